@@ -381,7 +381,8 @@ static void q4k_fit(const uint16_t* x, q4k_super* o, uint16_t* y)
             if (q > 15.0f) q = 15.0f;
             o->q[32 * j + i] = (uint8_t)q;
             if (y) {
-                float sq = s * q;
+                /* q is an unsigned integer code: dequantize from the integer */
+                float sq = s * (float)o->q[32 * j + i];
                 y[32 * j + i] = qfo_f32_to_bf16(sq - mm);
             }
         }

@@ -451,3 +451,16 @@ def test_ste_clipped_mask_is_saturation(fmt):
     assert np.array_equal(gx, np.where(keep, gb, 0).astype(np.uint16))
     if fmt == "nvfp4":
         assert (~keep).sum() > 0                               # saturation does occur
+
+
+def test_q4k_negative_values_rounding_to_code_zero_dequantize_to_positive_zero():
+    """Q4_K codes are unsigned integers: a sub-block whose stored min is 0 but that
+    holds small negative values dequantizes them from the integer code 0 to +0."""
+    x = np.zeros(256, np.float32)
+    x[:32] = np.linspace(0, 1, 32, dtype=np.float32)
+    x[5] = -1e-4                                              # rounds to q = 0, m stays 0
+    xb = oracle.f32_to_bf16(x)
+    d, dm, sc, m, q = oracle.q4k_fit_one(xb)
+    assert m[0] == 0 and q[5] == 0
+    y, _ = oracle.q4k(xb.reshape(1, 256))
+    assert y[5] == 0x0000
