@@ -458,7 +458,9 @@ def test_q4k_negative_values_rounding_to_code_zero_dequantize_to_positive_zero()
     holds small negative values dequantizes them from the integer code 0 to +0."""
     x = np.zeros(256, np.float32)
     x[:32] = np.linspace(0, 1, 32, dtype=np.float32)
-    x[5] = -1e-4                                              # rounds to q = 0, m stays 0
+    x[5] = -1e-4                                              # rounds to q = 0
+    x[32:64] = -1.0                                           # a large min elsewhere: dmin = 1/63,
+                                                              # so the first sub-block's m is 0
     xb = oracle.f32_to_bf16(x)
     d, dm, sc, m, q = oracle.q4k_fit_one(xb)
     assert m[0] == 0 and q[5] == 0
