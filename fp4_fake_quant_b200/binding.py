@@ -1,0 +1,167 @@
+"""Python binding of libqf.so: argument marshalling only.
+
+Every function here has the name of the C entry point it calls (include/qf.h)
+and does nothing but check tensor dtypes/devices, lay out the ``qf_tensor``
+array and pass raw device pointers plus the current CUDA stream.  All
+arithmetic runs in the library's sm_100a kernels; there is no fallback: if
+libqf.so is missing or fails to load, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libqf.so")
+
+QF_NVFP4, QF_MXFP4, QF_Q4K = 0, 1, 2
+FORMATS = {"nvfp4": QF_NVFP4, "mxfp4": QF_MXFP4, "q4k": QF_Q4K}
+BLOCK = {QF_NVFP4: 16, QF_MXFP4: 32, QF_Q4K: 256}
+STATUS = {0: "QF_OK", 1: "QF_ERR_INVALID_ARG", 2: "QF_ERR_SHAPE", 3: "QF_ERR_ALIGN",
+          4: "QF_ERR_UNSUPPORTED", 5: "QF_ERR_CUDA"}
+
+
+class QfTensor(ctypes.Structure):
+    """Mirror of ``qf_tensor`` (include/qf.h)."""
+    _fields_ = [("x", ctypes.c_void_p), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("group", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("y", ctypes.c_void_p), ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
+
+
+class QfError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libqf.so not built ({LIB_PATH}); run `python -m fp4_fake_quant_b200._build`"
+                          " or __graft_entry__.build()")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, I64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+    T = ctypes.POINTER(QfTensor)
+    lib.qf_amax_tied.argtypes = [T, I, P, I, P, P]
+    lib.qf_fakequant.argtypes = [I, T, I, P, I, P, P]
+    lib.qf_pack.argtypes = [I, T, I, P, I, P, P]
+    lib.qf_ste_backward.argtypes = [I, P, P, I64, I, T, P, I, P]
+    for f in (lib.qf_amax_tied, lib.qf_fakequant, lib.qf_pack, lib.qf_ste_backward):
+        f.restype = I
+    lib.qf_status_string.argtypes = [I]
+    lib.qf_status_string.restype = ctypes.c_char_p
+    lib.qf_last_error.argtypes = []
+    lib.qf_last_error.restype = ctypes.c_char_p
+    lib.qf_version.argtypes = []
+    lib.qf_version.restype = I
+    return lib
+
+
+lib = _load()
+
+# the entry points declared in include/qf.h
+EXPORTS = ("qf_amax_tied", "qf_fakequant", "qf_pack", "qf_ste_backward", "qf_status_string",
+           "qf_last_error", "qf_version")
+
+
+def _check(status: int) -> None:
+    if status != 0:
+        raise QfError(status, lib.qf_last_error().decode())
+
+
+def _fmt(f) -> int:
+    return FORMATS[f] if isinstance(f, str) else int(f)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors passed to libqf must be CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libqf must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _desc(xs: Sequence[torch.Tensor], ys=None, codes=None, scales=None, groups=None):
+    n = len(xs)
+    arr = (QfTensor * max(n, 1))()
+    for i, x in enumerate(xs):
+        if x.dtype != torch.bfloat16:
+            raise TypeError("x must be bfloat16")
+        rows, cols = (x.shape[0], x.shape[1]) if x.dim() == 2 else (1, x.numel()) if x.dim() == 1 \
+            else (x.numel() // x.shape[-1], x.shape[-1])
+        d = arr[i]
+        d.x = _ptr(x)
+        d.rows, d.cols = rows, cols
+        d.group = int(groups[i]) if groups is not None else 0
+        d.reserved = 0
+        d.y = _ptr(ys[i]) if ys is not None and ys[i] is not None else None
+        d.codes = _ptr(codes[i]) if codes is not None and codes[i] is not None else None
+        d.scales = _ptr(scales[i]) if scales is not None and scales[i] is not None else None
+    return arr, n
+
+
+def output_sizes(fmt, numel: int):
+    """Bytes of (codes, scales) for one tensor of ``numel`` elements."""
+    f = _fmt(fmt)
+    if f == QF_Q4K:
+        return (numel // 256) * 144, 0
+    return numel // 2, numel // BLOCK[f]
+
+
+def alloc_outputs(fmt, x: torch.Tensor, want_y: bool = True):
+    """Allocate (y, codes, scales) for one input tensor (torch allocations; plumbing)."""
+    ncodes, nscales = output_sizes(fmt, x.numel())
+    y = torch.empty_like(x) if want_y else None
+    codes = torch.empty(ncodes, dtype=torch.uint8, device=x.device)
+    scales = torch.empty(nscales, dtype=torch.uint8, device=x.device) if nscales else None
+    return y, codes, scales
+
+
+def qf_amax_tied(xs: Sequence[torch.Tensor], groups: Sequence[int], group_amax: torch.Tensor,
+                 tracked: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    arr, n = _desc(xs, groups=groups)
+    _check(lib.qf_amax_tied(arr, n, _ptr(group_amax), group_amax.numel(), _ptr(tracked),
+                            _stream(stream)))
+    return group_amax
+
+
+def qf_fakequant(fmt, xs: Sequence[torch.Tensor], ys=None, codes=None, scales=None, groups=None,
+                 group_amax: Optional[torch.Tensor] = None,
+                 group_scale_out: Optional[torch.Tensor] = None, stream=None) -> None:
+    arr, n = _desc(xs, ys, codes, scales, groups)
+    ng = group_amax.numel() if group_amax is not None else 0
+    _check(lib.qf_fakequant(_fmt(fmt), arr, n, _ptr(group_amax), ng, _ptr(group_scale_out),
+                            _stream(stream)))
+
+
+def qf_pack(fmt, xs: Sequence[torch.Tensor], codes, scales=None, groups=None,
+            group_amax: Optional[torch.Tensor] = None,
+            group_scale_out: Optional[torch.Tensor] = None, stream=None) -> None:
+    arr, n = _desc(xs, None, codes, scales, groups)
+    ng = group_amax.numel() if group_amax is not None else 0
+    _check(lib.qf_pack(_fmt(fmt), arr, n, _ptr(group_amax), ng, _ptr(group_scale_out),
+                       _stream(stream)))
+
+
+def qf_ste_backward(grad_y: torch.Tensor, grad_x: torch.Tensor, mode: int = 0, fmt="nvfp4",
+                    x: Optional[torch.Tensor] = None, group: int = 0,
+                    group_amax: Optional[torch.Tensor] = None, stream=None) -> None:
+    fwd = None
+    if mode == 1:
+        arr, _ = _desc([x], groups=[group])
+        fwd = arr
+    ng = group_amax.numel() if group_amax is not None else 0
+    _check(lib.qf_ste_backward(_fmt(fmt), _ptr(grad_y), _ptr(grad_x), grad_y.numel(), mode, fwd,
+                               _ptr(group_amax), ng, _stream(stream)))

@@ -1,0 +1,329 @@
+// qf_api.cu -- the C ABI of libqf.so (declared in include/qf.h): host-side argument
+// validation, descriptor tables and kernel launches.  No memory is allocated; all
+// work is enqueued on the caller's stream.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <vector>
+
+#include "qf.h"
+#include "qf_device.cuh"
+
+namespace {
+
+using qf::DevTensor;
+using qf::Table;
+using qf::kThreads;
+
+constexpr int kSmallT = 8;      // descriptor table sizes (kernel-parameter bytes: ~0.6 KB / ~27 KB)
+constexpr int kLargeT = 384;
+constexpr int kFp4U = 4;        // 256-element sub-tiles per warp unit
+constexpr int kQ4kU = 2;        // super-blocks per warp unit
+constexpr int kAmaxU = 8;
+
+thread_local char g_err[512] = "";
+
+qf_status fail(qf_status s, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+qf_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(QF_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int block_of(qf_format f) { return f == QF_NVFP4 ? 16 : f == QF_MXFP4 ? 32 : 256; }
+
+// Resident CTAs per SM for a kernel on the current device, and the SM count.
+struct Launch { int sms; int per_sm; };
+template <typename K>
+qf_status launch_shape(K kernel, Launch* L) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    e = cudaDeviceGetAttribute(&L->sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&L->per_sm, kernel, kThreads, 0);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+    if (L->per_sm < 1) L->per_sm = 1;
+    return QF_OK;
+}
+
+// Persistent grid: enough CTAs to fill every SM, never more than there is work.
+int grid_for(const Launch& L, int64_t units) {
+    const int64_t warps_per_cta = kThreads / 32;
+    int64_t want = (units + warps_per_cta - 1) / warps_per_cta;
+    int64_t cap = int64_t(L.sms) * L.per_sm;
+    return (int)std::max<int64_t>(1, std::min(want, cap));
+}
+
+template <int MAXT>
+void fill_table(Table<MAXT>& P, const std::vector<DevTensor>& v, size_t begin, size_t count,
+                int64_t unit_elems) {
+    memset(&P, 0, sizeof P);
+    int64_t u = 0;
+    for (size_t i = 0; i < count; ++i) {
+        DevTensor d = v[begin + i];
+        d.unit_begin = u;
+        u += (d.numel + unit_elems - 1) / unit_elems;
+        d.unit_end = u;
+        P.t[i] = d;
+    }
+    P.total_units = u;
+    P.n = (int)count;
+}
+
+// Launch `kernel<MAXT>` over v in chunks of at most kLargeT tensors.
+template <typename KS, typename KL>
+qf_status launch_chunks(KS small_kernel, KL large_kernel, const std::vector<DevTensor>& v,
+                        int64_t unit_elems, const float* amax, float* scale_out, float* tracked,
+                        int n_groups, cudaStream_t s) {
+    Launch Ls, Ll;
+    qf_status st = launch_shape(small_kernel, &Ls);
+    if (st != QF_OK) return st;
+    st = launch_shape(large_kernel, &Ll);
+    if (st != QF_OK) return st;
+    if (v.empty() && scale_out) {
+        // nothing to quantize, but the per-group tensor scales are still reported
+        Table<kSmallT> P;
+        memset(&P, 0, sizeof P);
+        P.group_amax = amax;
+        P.group_scale_out = scale_out;
+        P.n_groups = n_groups;
+        small_kernel<<<1, kThreads, 0, s>>>(P);
+    }
+    for (size_t b = 0; b < v.size(); b += kLargeT) {
+        const size_t cnt = std::min<size_t>(kLargeT, v.size() - b);
+        float* so = b == 0 ? scale_out : nullptr;
+        if (cnt <= (size_t)kSmallT) {
+            Table<kSmallT> P;
+            fill_table(P, v, b, cnt, unit_elems);
+            P.group_amax = amax; P.group_scale_out = so; P.tracked = tracked; P.n_groups = n_groups;
+            small_kernel<<<grid_for(Ls, P.total_units), kThreads, 0, s>>>(P);
+        } else {
+            Table<kLargeT> Q;              // ~27 KB kernel parameter
+            fill_table(Q, v, b, cnt, unit_elems);
+            Q.group_amax = amax; Q.group_scale_out = so; Q.tracked = tracked; Q.n_groups = n_groups;
+            large_kernel<<<grid_for(Ll, Q.total_units), kThreads, 0, s>>>(Q);
+        }
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+    return QF_OK;
+}
+
+// Validate one tensor; `need_cols_multiple` is 0 for qf_amax_tied.
+qf_status check_tensor(const qf_tensor& t, int i, int need_cols_multiple, int n_groups,
+                       bool check_group) {
+    if (t.rows < 0 || t.cols < 0) return fail(QF_ERR_SHAPE, "tensor %d: negative size", i);
+    if (t.cols > 0 && t.rows > INT64_MAX / 4 / t.cols)
+        return fail(QF_ERR_SHAPE, "tensor %d: rows*cols overflows", i);
+    if (need_cols_multiple && t.cols % need_cols_multiple != 0)
+        return fail(QF_ERR_SHAPE, "tensor %d: cols=%lld is not a multiple of %d", i,
+                    (long long)t.cols, need_cols_multiple);
+    if (t.reserved != 0) return fail(QF_ERR_INVALID_ARG, "tensor %d: reserved field not 0", i);
+    const int64_t numel = t.rows * t.cols;
+    if (numel > 0 && t.x == nullptr) return fail(QF_ERR_INVALID_ARG, "tensor %d: x is NULL", i);
+    if (!aligned16(t.x)) return fail(QF_ERR_ALIGN, "tensor %d: x not 16-byte aligned", i);
+    if (check_group && (t.group < 0 || t.group >= n_groups))
+        return fail(QF_ERR_INVALID_ARG, "tensor %d: group %d outside [0, %d)", i, t.group, n_groups);
+    return QF_OK;
+}
+
+qf_status fakequant_impl(qf_format f, const qf_tensor* t, int n, const float* d_group_amax,
+                         int n_groups, float* d_group_scale_out, void* stream, bool pack_only) {
+    g_err[0] = 0;
+    if (f != QF_NVFP4 && f != QF_MXFP4 && f != QF_Q4K)
+        return fail(QF_ERR_UNSUPPORTED, "unknown format %d", (int)f);
+    if (n < 0) return fail(QF_ERR_INVALID_ARG, "n = %d < 0", n);
+    if (n > 0 && t == nullptr) return fail(QF_ERR_INVALID_ARG, "tensor array is NULL");
+    const bool nv = f == QF_NVFP4;
+    if (nv) {
+        if (n_groups <= 0) return fail(QF_ERR_INVALID_ARG, "NVFP4 needs n_groups > 0");
+        if (d_group_amax == nullptr) return fail(QF_ERR_INVALID_ARG, "NVFP4 needs d_group_amax");
+    }
+    std::vector<DevTensor> v;
+    v.reserve(n);
+    for (int i = 0; i < n; ++i) {
+        qf_status st = check_tensor(t[i], i, block_of(f), n_groups, nv);
+        if (st != QF_OK) return st;
+        const int64_t numel = t[i].rows * t[i].cols;
+        if (numel == 0) continue;
+        void* y = pack_only ? nullptr : t[i].y;
+        void* scales = f == QF_Q4K ? nullptr : t[i].scales;
+        if (!y && !t[i].codes && !scales)
+            return fail(QF_ERR_INVALID_ARG, "tensor %d: no output (y, codes, scales all NULL)", i);
+        if (!aligned16(y) || !aligned16(t[i].codes))
+            return fail(QF_ERR_ALIGN, "tensor %d: y / codes not 16-byte aligned", i);
+        DevTensor d{};
+        d.x = static_cast<const uint16_t*>(t[i].x);
+        d.y = static_cast<uint16_t*>(y);
+        d.codes = static_cast<uint8_t*>(t[i].codes);
+        d.scales = static_cast<uint8_t*>(scales);
+        d.numel = numel;
+        d.group = nv ? t[i].group : 0;
+        v.push_back(d);
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    float* so = nv ? d_group_scale_out : nullptr;
+    const float* am = nv ? d_group_amax : nullptr;
+    const int ng = nv ? n_groups : 0;
+    if (v.empty() && !so) return QF_OK;
+    switch (f) {
+        case QF_NVFP4:
+            return launch_chunks(qf::k_fp4<true, kFp4U, kSmallT, 0>, qf::k_fp4<true, kFp4U, kLargeT, 0>,
+                                 v, 256 * kFp4U, am, so, nullptr, ng, s);
+        case QF_MXFP4:
+            return launch_chunks(qf::k_fp4<false, kFp4U, kSmallT, 0>,
+                                 qf::k_fp4<false, kFp4U, kLargeT, 0>, v, 256 * kFp4U, am, so,
+                                 nullptr, ng, s);
+        default:
+            return launch_chunks(qf::k_q4k<kQ4kU, kSmallT, 0>, qf::k_q4k<kQ4kU, kLargeT, 0>, v,
+                                 256 * kQ4kU, am, so, nullptr, ng, s);
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+qf_status qf_amax_tied(const qf_tensor* t, int n, float* d_group_amax, int n_groups,
+                       float* d_tracked, void* stream) {
+    g_err[0] = 0;
+    if (n < 0) return fail(QF_ERR_INVALID_ARG, "n = %d < 0", n);
+    if (n > 0 && t == nullptr) return fail(QF_ERR_INVALID_ARG, "tensor array is NULL");
+    if (n_groups <= 0) return fail(QF_ERR_INVALID_ARG, "n_groups = %d <= 0", n_groups);
+    if (d_group_amax == nullptr) return fail(QF_ERR_INVALID_ARG, "d_group_amax is NULL");
+    std::vector<DevTensor> v;
+    bool ragged = false;
+    for (int i = 0; i < n; ++i) {
+        qf_status st = check_tensor(t[i], i, 0, n_groups, true);
+        if (st != QF_OK) return st;
+        const int64_t numel = t[i].rows * t[i].cols;
+        if (numel == 0) continue;
+        DevTensor d{};
+        d.x = static_cast<const uint16_t*>(t[i].x);
+        d.numel = numel;
+        d.group = t[i].group;
+        ragged |= (numel & 7) != 0;
+        v.push_back(d);
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(d_group_amax, 0, sizeof(float) * (size_t)n_groups, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+    if (v.empty()) return QF_OK;
+    qf_status st = launch_chunks(qf::k_amax<kAmaxU, kSmallT>, qf::k_amax<kAmaxU, kLargeT>, v,
+                                 256 * kAmaxU, d_group_amax, nullptr, d_tracked, n_groups, s);
+    if (st != QF_OK || !ragged) return st;
+    // scalar tails of tensors whose size is not a multiple of 8 elements
+    for (size_t b = 0; b < v.size(); b += kSmallT) {
+        const size_t cnt = std::min<size_t>(kSmallT, v.size() - b);
+        Table<kSmallT> P;
+        fill_table(P, v, b, cnt, 256 * kAmaxU);
+        P.group_amax = d_group_amax;
+        P.tracked = d_tracked;
+        P.n_groups = n_groups;
+        qf::k_amax_tail<kSmallT><<<(unsigned)cnt, 32, 0, s>>>(P);
+    }
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+    return QF_OK;
+}
+
+qf_status qf_fakequant(qf_format f, const qf_tensor* t, int n, const float* d_group_amax,
+                       int n_groups, float* d_group_scale_out, void* stream) {
+    return fakequant_impl(f, t, n, d_group_amax, n_groups, d_group_scale_out, stream, false);
+}
+
+qf_status qf_pack(qf_format f, const qf_tensor* t, int n, const float* d_group_amax,
+                  int n_groups, float* d_group_scale_out, void* stream) {
+    return fakequant_impl(f, t, n, d_group_amax, n_groups, d_group_scale_out, stream, true);
+}
+
+qf_status qf_ste_backward(qf_format f, const void* grad_y, void* grad_x, int64_t numel, int mode,
+                          const qf_tensor* fwd, const float* d_group_amax, int n_groups,
+                          void* stream) {
+    g_err[0] = 0;
+    if (mode != 0 && mode != 1) return fail(QF_ERR_UNSUPPORTED, "unknown STE mode %d", mode);
+    if (numel < 0) return fail(QF_ERR_SHAPE, "numel = %lld < 0", (long long)numel);
+    if (numel > 0 && (grad_y == nullptr || grad_x == nullptr))
+        return fail(QF_ERR_INVALID_ARG, "grad_y / grad_x is NULL");
+    if (!aligned16(grad_y) || !aligned16(grad_x))
+        return fail(QF_ERR_ALIGN, "grad_y / grad_x not 16-byte aligned");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (mode == 0) {
+        if (numel == 0 || grad_x == grad_y) return QF_OK;
+        Launch L;
+        qf_status st = launch_shape(qf::k_copy, &L);
+        if (st != QF_OK) return st;
+        const int64_t vec = (numel + 7) / 8;
+        const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(
+            (vec + kThreads - 1) / kThreads, int64_t(L.sms) * L.per_sm));
+        qf::k_copy<<<grid, kThreads, 0, s>>>(static_cast<const uint16_t*>(grad_y),
+                                             static_cast<uint16_t*>(grad_x), numel);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+        return QF_OK;
+    }
+    if (f != QF_NVFP4 && f != QF_MXFP4 && f != QF_Q4K)
+        return fail(QF_ERR_UNSUPPORTED, "unknown format %d", (int)f);
+    if (fwd == nullptr) return fail(QF_ERR_INVALID_ARG, "clipped STE needs the forward tensor");
+    const bool nv = f == QF_NVFP4;
+    if (nv && (n_groups <= 0 || d_group_amax == nullptr))
+        return fail(QF_ERR_INVALID_ARG, "NVFP4 clipped STE needs d_group_amax and n_groups > 0");
+    qf_status st = check_tensor(*fwd, 0, block_of(f), n_groups, nv);
+    if (st != QF_OK) return st;
+    if (fwd->rows * fwd->cols != numel)
+        return fail(QF_ERR_SHAPE, "numel %lld != rows*cols of the forward tensor",
+                    (long long)numel);
+    // grad_x == grad_y is allowed: each element is read before the same thread writes it
+    if (numel == 0) return QF_OK;
+    std::vector<DevTensor> v(1);
+    v[0] = DevTensor{};
+    v[0].x = static_cast<const uint16_t*>(fwd->x);
+    v[0].g = static_cast<const uint16_t*>(grad_y);
+    v[0].y = static_cast<uint16_t*>(grad_x);
+    v[0].numel = numel;
+    v[0].group = nv ? fwd->group : 0;
+    const float* am = nv ? d_group_amax : nullptr;
+    switch (f) {
+        case QF_NVFP4:
+            return launch_chunks(qf::k_fp4<true, kFp4U, kSmallT, 1>, qf::k_fp4<true, kFp4U, kLargeT, 1>,
+                                 v, 256 * kFp4U, am, nullptr, nullptr, n_groups, s);
+        case QF_MXFP4:
+            return launch_chunks(qf::k_fp4<false, kFp4U, kSmallT, 1>,
+                                 qf::k_fp4<false, kFp4U, kLargeT, 1>, v, 256 * kFp4U, nullptr,
+                                 nullptr, nullptr, 0, s);
+        default:
+            return launch_chunks(qf::k_q4k<kQ4kU, kSmallT, 1>, qf::k_q4k<kQ4kU, kLargeT, 1>, v,
+                                 256 * kQ4kU, nullptr, nullptr, nullptr, 0, s);
+    }
+}
+
+const char* qf_status_string(qf_status s) {
+    switch (s) {
+        case QF_OK: return "QF_OK";
+        case QF_ERR_INVALID_ARG: return "QF_ERR_INVALID_ARG: invalid argument";
+        case QF_ERR_SHAPE: return "QF_ERR_SHAPE: invalid or unsupported shape";
+        case QF_ERR_ALIGN: return "QF_ERR_ALIGN: pointer not 16-byte aligned";
+        case QF_ERR_UNSUPPORTED: return "QF_ERR_UNSUPPORTED: unknown format or mode";
+        case QF_ERR_CUDA: return "QF_ERR_CUDA: a CUDA call failed";
+    }
+    return "unknown qf_status";
+}
+
+const char* qf_last_error(void) { return g_err; }
+
+int qf_version(void) { return (1 << 16) | 0; }
+
+}  // extern "C"

@@ -1,0 +1,484 @@
+// qf_device.cuh -- sm_100a kernels of the deployment-aligned simulated-quantization
+// hot path (QATFactory project page: Method, "Framework overview" / "Numerics",
+// "Supported formats" table).
+//
+// Design (HBM-bound streaming codec, no tensor cores):
+//   * A call covers n tensors.  Their descriptors travel in a __grid_constant__
+//     kernel parameter (no device allocation, no copy), each tensor split into
+//     fixed-size "units" of elements; a unit is the work of one warp iteration.
+//   * Persistent grid: (#SMs x resident CTAs) CTAs; warp w takes units w, w+W, ...
+//   * Lane l of a warp holds 8 consecutive BF16 (one 16-byte load) of each
+//     256-element sub-tile, so every load and every BF16 store is a fully
+//     coalesced 512-byte warp transaction.  Block statistics are reduced across
+//     the 2 (NVFP4), 4 (MXFP4) or 32 (Q4_K super-block) lanes that share a block
+//     with warp shuffles.
+//   * Blackwell's native conversions do the format rounding:
+//     cvt.rn.satfinite.e2m1x2.f32, cvt.rn.satfinite.e4m3x2.f32, cvt.rn.bf16x2.f32
+//     and the reverse cvt.rn.f16x2.{e2m1x2,e4m3x2}.
+//   * Every scale step is one IEEE binary32 operation with round-to-nearest-even
+//     (__fdiv_rn, __frcp_rn, __fmul_rn, __fadd_rn); the library is built without
+//     FMA contraction so the rounding order is the one the header documents.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+namespace qf {
+
+constexpr int kThreads = 256;
+constexpr unsigned kFull = 0xFFFFFFFFu;
+
+// One tensor of a launch.
+struct DevTensor {
+    const uint16_t* x;      // BF16 input
+    uint16_t* y;            // BF16 dequant out / STE grad_x (nullable)
+    uint8_t* codes;         // packed nibbles / Q4_K blocks (nullable)
+    uint8_t* scales;        // E4M3 / E8M0 bytes (nullable)
+    const uint16_t* g;      // STE: upstream gradient
+    int64_t numel;
+    int64_t unit_begin;     // first global unit of this tensor
+    int64_t unit_end;       // one past its last unit
+    int32_t group;          // NVFP4 tie group
+    int32_t pad;
+};
+
+template <int MAXT>
+struct Table {
+    DevTensor t[MAXT];
+    int64_t total_units;
+    const float* group_amax;    // NVFP4 tie-group amax (read) / qf_amax_tied output
+    float* group_scale_out;     // NVFP4 s_t per group (nullable)
+    float* tracked;             // qf_amax_tied running amax (nullable)
+    int32_t n;
+    int32_t n_groups;
+};
+
+// ------------------------------------------------------------------ PTX helpers
+// Two FP32 -> one byte of two E2M1 codes: `hi` in bits 4-7, `lo` in bits 0-3.
+__device__ __forceinline__ uint32_t cvt_e2m1x2(float hi, float lo) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
+        : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+// One byte of two E2M1 codes -> f16x2 (bits 4-7 -> upper half).
+__device__ __forceinline__ uint32_t cvt_e2m1x2_f16x2(uint32_t b) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+        : "=r"(r) : "r"(b));
+    return r;
+}
+// Two FP32 -> two E4M3 bytes (hi in bits 8-15), round to nearest even, saturating.
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float hi, float lo) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+__device__ __forceinline__ uint32_t cvt_e4m3x2_f16x2(uint32_t v) {
+    uint32_t r;
+    uint16_t h = (uint16_t)v;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(h));
+    return r;
+}
+// Two FP32 -> BF16x2 (hi in the upper half), round to nearest even.
+__device__ __forceinline__ uint32_t cvt_bf16x2(float hi, float lo) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+__device__ __forceinline__ float f16_lo(uint32_t h2) {
+    return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+}
+__device__ __forceinline__ float f16_hi(uint32_t h2) {
+    return __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
+}
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// 16-byte streaming load (read-only path, no L1 allocation, 256-byte L2 prefetch).
+__device__ __forceinline__ uint4 ld_stream(const uint16_t* p) {
+    uint4 v;
+    asm("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
+        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ void st_v4(void* p, uint4 v) { *reinterpret_cast<uint4*>(p) = v; }
+
+// bf16x2 helpers on raw bits
+__device__ __forceinline__ uint32_t bmax2(uint32_t a, uint32_t b) {
+    __nv_bfloat162 r = __hmax2(*reinterpret_cast<__nv_bfloat162*>(&a),
+                               *reinterpret_cast<__nv_bfloat162*>(&b));
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t bmin2(uint32_t a, uint32_t b) {
+    __nv_bfloat162 r = __hmin2(*reinterpret_cast<__nv_bfloat162*>(&a),
+                               *reinterpret_cast<__nv_bfloat162*>(&b));
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+// max |x| over the lane's 8 BF16 values, as non-negative BF16 bits
+__device__ __forceinline__ uint32_t abs_max8(uint4 v) {
+    uint32_t m = bmax2(bmax2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
+                       bmax2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
+    return max(m & 0xFFFFu, m >> 16);
+}
+
+// Walk the descriptor table forward to the tensor that owns unit u (units are
+// visited in increasing order by each warp, so this is amortised O(1)).
+template <int MAXT>
+__device__ __forceinline__ int find_tensor(const Table<MAXT>& P, int ti, int64_t u) {
+    while (u >= P.t[ti].unit_end) ++ti;
+    return ti;
+}
+
+// NVFP4 tensor scale of a tie group: s_t = amax_g / (6 * 448).
+__device__ __forceinline__ float nv_tensor_scale(float amax_g) { return __fdiv_rn(amax_g, 2688.0f); }
+
+// ------------------------------------------------------------------ NVFP4 / MXFP4
+// Per-lane result of the FP4 codec for 8 elements.
+struct Fp4Lane {
+    uint32_t codes;     // 8 nibbles, element k in bits 4k..4k+3
+    uint32_t scale;     // block scale byte
+    uint4 y;            // 8 BF16
+    float q[8];         // scaled values (for the clipped STE)
+};
+
+// MODE 0: codes + scales + (optionally) dequant.  Block statistics by shuffles.
+template <bool NV, bool WANT_Y>
+__device__ __forceinline__ void fp4_lane(uint4 v, float s_t, float six_st, Fp4Lane& o) {
+    uint32_t a = abs_max8(v);
+    a = max(a, __shfl_xor_sync(kFull, a, 1));
+    if (!NV) a = max(a, __shfl_xor_sync(kFull, a, 2));
+    float S, inv;
+    if (NV) {
+        // E4M3 block scale of the 16-element block held by this lane pair
+        uint32_t sb = 0;
+        S = 0.0f;
+        inv = 0.0f;
+        if (s_t != 0.0f) {
+            float ratio = __fdiv_rn(__uint_as_float(a << 16), six_st);
+            sb = cvt_e4m3x2(0.0f, ratio) & 0xFFu;
+            S = __fmul_rn(f16_lo(cvt_e4m3x2_f16x2(sb)), s_t);
+            inv = (S == 0.0f) ? 0.0f : __frcp_rn(S);
+        }
+        o.scale = sb;
+    } else {
+        // E8M0: e = floor(log2 amax) - 2 clamped to >= -127; byte = e + 127 = max(E - 2, 0)
+        uint32_t E = a >> 7;
+        uint32_t c = E > 2u ? E - 2u : 0u;
+        o.scale = c;
+        inv = __uint_as_float((254u - c) << 23);                      // 2^-e
+        S = c ? __uint_as_float(c << 23) : __uint_as_float(0x00200000u);   // 2^e
+    }
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        o.q[2 * k] = __fmul_rn(bf16_lo(w[k]), inv);
+        o.q[2 * k + 1] = __fmul_rn(bf16_hi(w[k]), inv);
+    }
+    if (NV && __builtin_expect(isinf(inv), 0)) {
+        // 1/S overflowed (S < 2^-128): a zero keeps its own sign instead of 0 * inf
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            if (bf16_lo(w[k]) == 0.0f) o.q[2 * k] = bf16_lo(w[k]);
+            if (bf16_hi(w[k]) == 0.0f) o.q[2 * k + 1] = bf16_hi(w[k]);
+        }
+    }
+    uint32_t b[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) b[k] = cvt_e2m1x2(o.q[2 * k + 1], o.q[2 * k]);
+    o.codes = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
+    if (WANT_Y) {
+        uint32_t yw[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            uint32_t h2 = cvt_e2m1x2_f16x2(b[k]);
+            yw[k] = cvt_bf16x2(__fmul_rn(f16_hi(h2), S), __fmul_rn(f16_lo(h2), S));
+        }
+        o.y = make_uint4(yw[0], yw[1], yw[2], yw[3]);
+    }
+}
+
+// Fused NVFP4 / MXFP4 fake-quant + pack (MODE 0) or clipped STE (MODE 1).
+// A unit is U sub-tiles of 256 elements.
+template <bool NV, int U, int MAXT, int MODE>
+__global__ void __launch_bounds__(kThreads) k_fp4(const __grid_constant__ Table<MAXT> P) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = (int64_t(blockIdx.x) * kThreads + threadIdx.x) >> 5;
+    const int64_t nwarps = (int64_t(gridDim.x) * kThreads) >> 5;
+    constexpr int kUnit = 256 * U;
+    if (NV && MODE == 0 && blockIdx.x == 0 && P.group_scale_out) {
+        for (int g = threadIdx.x; g < P.n_groups; g += kThreads)
+            P.group_scale_out[g] = nv_tensor_scale(P.group_amax[g]);
+    }
+    int ti = 0, cur = -1;
+    float s_t = 0.0f, six_st = 0.0f;
+    for (int64_t u = warp; u < P.total_units; u += nwarps) {
+        ti = find_tensor(P, ti, u);
+        const DevTensor& T = P.t[ti];
+        if (NV && ti != cur) {
+            s_t = nv_tensor_scale(P.group_amax[T.group]);
+            six_st = __fmul_rn(6.0f, s_t);
+            cur = ti;
+        }
+        const int64_t e0 = (u - T.unit_begin) * kUnit;
+        uint4 v[U], gv[U];
+        bool ok[U];
+#pragma unroll
+        for (int s = 0; s < U; ++s) {
+            const int64_t e = e0 + s * 256 + lane * 8;
+            ok[s] = e < T.numel;
+            v[s] = ok[s] ? ld_stream(T.x + e) : make_uint4(0, 0, 0, 0);
+            if (MODE == 1) gv[s] = ok[s] ? ld_stream(T.g + e) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int s = 0; s < U; ++s) {
+            const int64_t e = e0 + s * 256 + lane * 8;
+            Fp4Lane o;
+            if (MODE == 0) {
+                if (T.y) fp4_lane<NV, true>(v[s], s_t, six_st, o);
+                else fp4_lane<NV, false>(v[s], s_t, six_st, o);
+                if (ok[s]) {
+                    if (T.y) st_v4(T.y + e, o.y);
+                    if (T.codes) *reinterpret_cast<uint32_t*>(T.codes + (e >> 1)) = o.codes;
+                    if (T.scales && (lane & (NV ? 1 : 3)) == 0)
+                        T.scales[e >> (NV ? 4 : 5)] = (uint8_t)o.scale;
+                }
+            } else {
+                fp4_lane<NV, false>(v[s], s_t, six_st, o);
+                if (ok[s]) {
+                    const uint32_t gw[4] = {gv[s].x, gv[s].y, gv[s].z, gv[s].w};
+                    uint32_t r[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        uint32_t lo = fabsf(o.q[2 * k]) <= 6.0f ? (gw[k] & 0xFFFFu) : 0u;
+                        uint32_t hi = fabsf(o.q[2 * k + 1]) <= 6.0f ? (gw[k] & 0xFFFF0000u) : 0u;
+                        r[k] = lo | hi;
+                    }
+                    st_v4(T.y + e, make_uint4(r[0], r[1], r[2], r[3]));
+                }
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------ Q4_K
+// One warp per 256-element super-block: lane l holds elements 8l..8l+7, i.e.
+// sub-block j = l / 4.
+struct Q4kLane {
+    uint4 y;
+    uint32_t qs;        // this lane's 4 bytes of the 128-byte code area
+    uint32_t hdr;       // lanes 0..3: word l of the 16-byte header
+    float v[8];         // scaled values (for the clipped STE)
+};
+
+template <bool WANT_Y>
+__device__ __forceinline__ void q4k_lane(uint4 xv, int lane, Q4kLane& o) {
+    const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w};
+    // sub-block max and min: pack (max, -min) as bf16x2 and reduce both with one max
+    uint32_t mx = bmax2(bmax2(w[0], w[1]), bmax2(w[2], w[3]));
+    uint32_t mn = bmin2(bmin2(w[0], w[1]), bmin2(w[2], w[3]));
+    uint32_t hi = bmax2(mx, mx >> 16) & 0xFFFFu;            // bf16 bits of max
+    uint32_t lo = bmin2(mn, mn >> 16) & 0xFFFFu;            // bf16 bits of min
+    uint32_t pk = (hi << 16) | (lo ^ 0x8000u);              // (max, -min)
+    pk = bmax2(pk, __shfl_xor_sync(kFull, pk, 1));
+    pk = bmax2(pk, __shfl_xor_sync(kFull, pk, 2));
+    const float hi_f = bf16_hi(pk);
+    const float negmin = bf16_lo(pk);
+    const float min_j = negmin > 0.0f ? negmin : 0.0f;
+    const float scale_j = __fdiv_rn(__fadd_rn(hi_f, min_j), 15.0f);
+    float ms = scale_j, mm = min_j;
+#pragma unroll
+    for (int o2 = 4; o2 < 32; o2 <<= 1) {
+        ms = fmaxf(ms, __shfl_xor_sync(kFull, ms, o2));
+        mm = fmaxf(mm, __shfl_xor_sync(kFull, mm, o2));
+    }
+    const __half dh = __float2half_rn(__fdiv_rn(ms, 63.0f));
+    const __half dmh = __float2half_rn(__fdiv_rn(mm, 63.0f));
+    const float d = __half2float(dh), dmin = __half2float(dmh);
+    const int sc = d == 0.0f ? 0 : min(__float2int_rn(__fdiv_rn(scale_j, d)), 63);
+    const int m = dmin == 0.0f ? 0 : min(__float2int_rn(__fdiv_rn(min_j, dmin)), 63);
+    const float s = __fmul_rn(d, (float)sc);
+    const float mmv = __fmul_rn(dmin, (float)m);
+    const float inv = s == 0.0f ? 0.0f : __frcp_rn(s);
+    // elements: q = clamp(RNE((x + mm) * inv), 0, 15) via the 1.5*2^23 rounding constant
+    uint32_t qb[8];
+    float yk[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const float xk = (k & 1) ? bf16_hi(w[k >> 1]) : bf16_lo(w[k >> 1]);
+        const float t = __fmul_rn(__fadd_rn(xk, mmv), inv);
+        o.v[k] = t;
+        const float r = __fadd_rn(fminf(fmaxf(t, 0.0f), 15.0f), 12582912.0f);
+        qb[k] = __float_as_uint(r) & 15u;
+        // r - 1.5*2^23 is the integer code q as a float (exact)
+        yk[k] = __fsub_rn(__fmul_rn(s, __fsub_rn(r, 12582912.0f)), mmv);
+    }
+    if (WANT_Y)
+        o.y = make_uint4(cvt_bf16x2(yk[1], yk[0]), cvt_bf16x2(yk[3], yk[2]),
+                         cvt_bf16x2(yk[5], yk[4]), cvt_bf16x2(yk[7], yk[6]));
+    // codes: byte p of chunk c = q[2c][p] | q[2c+1][p] << 4; pair lane l with l ^ 4
+    const uint32_t B0 = qb[0] | (qb[1] << 8) | (qb[2] << 16) | (qb[3] << 24);
+    const uint32_t B1 = qb[4] | (qb[5] << 8) | (qb[6] << 16) | (qb[7] << 24);
+    const bool odd = (lane >> 2) & 1;
+    const uint32_t recv = __shfl_xor_sync(kFull, odd ? B0 : B1, 4);
+    o.qs = odd ? (recv | (B1 << 4)) : (B0 | (recv << 4));
+    // header: d, dmin, then 12 bytes of 6-bit scales and mins
+    const uint32_t smv = (uint32_t)sc | ((uint32_t)m << 8);
+    const uint32_t A = __shfl_sync(kFull, smv, 4 * (lane & 7));          // lane l<8: sub-block l
+    const uint32_t Bv = __shfl_sync(kFull, A, (lane & 3) + 4);            // sub-block (l&3)+4
+    const uint32_t scA = A & 0xFF, mA = A >> 8, scB = Bv & 0xFF, mB = Bv >> 8;
+    const uint32_t pb = ((scA & 63) | ((scB >> 4) << 6)) |
+                        (((mA & 63) | ((mB >> 4) << 6)) << 8) |
+                        (((scB & 15) | ((mB & 15) << 4)) << 16);
+    // transpose: word 1+r gathers byte r of lanes 0..3
+    const uint32_t p0 = __shfl_sync(kFull, pb, 0), p1 = __shfl_sync(kFull, pb, 1);
+    const uint32_t p2 = __shfl_sync(kFull, pb, 2), p3 = __shfl_sync(kFull, pb, 3);
+    // lane 1..3 takes byte slot r = lane-1 of lanes 0..3 (lane 0 writes d, dmin)
+    const uint32_t r = ((uint32_t)(lane & 3) + 3u) & 3u;
+    const uint32_t sel = r | ((r + 4u) << 4);               // byte r of each operand
+    const uint32_t w01 = __byte_perm(p0, p1, sel);
+    const uint32_t w23 = __byte_perm(p2, p3, sel);
+    const uint32_t word = __byte_perm(w01, w23, 0x5410u);
+    o.hdr = (lane & 3) == 0
+                ? ((uint32_t)__half_as_ushort(dh) | ((uint32_t)__half_as_ushort(dmh) << 16))
+                : word;
+}
+
+template <int U, int MAXT, int MODE>
+__global__ void __launch_bounds__(kThreads) k_q4k(const __grid_constant__ Table<MAXT> P) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = (int64_t(blockIdx.x) * kThreads + threadIdx.x) >> 5;
+    const int64_t nwarps = (int64_t(gridDim.x) * kThreads) >> 5;
+    constexpr int kUnit = 256 * U;
+    int ti = 0;
+    for (int64_t u = warp; u < P.total_units; u += nwarps) {
+        ti = find_tensor(P, ti, u);
+        const DevTensor& T = P.t[ti];
+        const int64_t e0 = (u - T.unit_begin) * kUnit;
+        uint4 v[U], gv[U];
+        bool ok[U];
+#pragma unroll
+        for (int s = 0; s < U; ++s) {
+            const int64_t e = e0 + s * 256 + lane * 8;
+            ok[s] = (e0 + s * 256) < T.numel;            // a whole super-block or nothing
+            v[s] = ok[s] ? ld_stream(T.x + e) : make_uint4(0, 0, 0, 0);
+            if (MODE == 1) gv[s] = ok[s] ? ld_stream(T.g + e) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int s = 0; s < U; ++s) {
+            if (!ok[s]) continue;                          // warp-uniform
+            const int64_t sb = (e0 >> 8) + s;              // super-block index in the tensor
+            const int64_t e = e0 + s * 256 + lane * 8;
+            Q4kLane o;
+            if (MODE == 0) {
+                if (T.y) q4k_lane<true>(v[s], lane, o);
+                else q4k_lane<false>(v[s], lane, o);
+                if (T.y) st_v4(T.y + e, o.y);
+                if (T.codes) {
+                    uint8_t* blk = T.codes + sb * 144;
+                    const int off = 16 + 32 * (lane >> 3) + 8 * (lane & 3) + 4 * ((lane >> 2) & 1);
+                    *reinterpret_cast<uint32_t*>(blk + off) = o.qs;
+                    if (lane < 4) *reinterpret_cast<uint32_t*>(blk + 4 * lane) = o.hdr;
+                }
+            } else {
+                q4k_lane<false>(v[s], lane, o);
+                const uint32_t gw[4] = {gv[s].x, gv[s].y, gv[s].z, gv[s].w};
+                uint32_t r[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float a = o.v[2 * k], b = o.v[2 * k + 1];
+                    uint32_t lo = (a >= 0.0f && a <= 15.0f) ? (gw[k] & 0xFFFFu) : 0u;
+                    uint32_t hi = (b >= 0.0f && b <= 15.0f) ? (gw[k] & 0xFFFF0000u) : 0u;
+                    r[k] = lo | hi;
+                }
+                st_v4(T.y + e, make_uint4(r[0], r[1], r[2], r[3]));
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------ tied amax
+// Running max|x| per lane while the warp stays in one tie group; on a group
+// change (and at the end) the warp reduces and lane 0 does one atomicMax on the
+// group's FP32 bits (non-negative floats order like their bit patterns).
+template <int U, int MAXT>
+__global__ void __launch_bounds__(kThreads) k_amax(const __grid_constant__ Table<MAXT> P) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = (int64_t(blockIdx.x) * kThreads + threadIdx.x) >> 5;
+    const int64_t nwarps = (int64_t(gridDim.x) * kThreads) >> 5;
+    constexpr int kUnit = 256 * U;
+    float* amax = const_cast<float*>(P.group_amax);
+    int ti = 0, g = -1;
+    uint32_t run = 0;          // bf16x2 running max of |x|
+    auto flush = [&](int grp) {
+        uint32_t a = max(run & 0xFFFFu, run >> 16);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) a = max(a, __shfl_xor_sync(kFull, a, o));
+        if (lane == 0 && grp >= 0) {
+            atomicMax(reinterpret_cast<unsigned int*>(amax) + grp, a << 16);
+            if (P.tracked) atomicMax(reinterpret_cast<unsigned int*>(P.tracked) + grp, a << 16);
+        }
+        run = 0;
+    };
+    for (int64_t u = warp; u < P.total_units; u += nwarps) {
+        ti = find_tensor(P, ti, u);
+        const DevTensor& T = P.t[ti];
+        if (T.group != g) {
+            if (g >= 0) flush(g);
+            g = T.group;
+        }
+        const int64_t e0 = (u - T.unit_begin) * kUnit;
+        uint4 v[U];
+#pragma unroll
+        for (int s = 0; s < U; ++s) {
+            const int64_t e = e0 + s * 256 + lane * 8;
+            v[s] = (e + 8 <= T.numel) ? ld_stream(T.x + e) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int s = 0; s < U; ++s) {
+            run = bmax2(run, bmax2(bmax2(v[s].x & 0x7FFF7FFFu, v[s].y & 0x7FFF7FFFu),
+                                   bmax2(v[s].z & 0x7FFF7FFFu, v[s].w & 0x7FFF7FFFu)));
+        }
+    }
+    if (g >= 0) flush(g);
+}
+
+// amax of tensors whose element count is not a multiple of 8 handles the
+// scalar tail here (one thread per leftover element; at most 7 per tensor).
+template <int MAXT>
+__global__ void k_amax_tail(const __grid_constant__ Table<MAXT> P) {
+    const int ti = blockIdx.x;
+    if (ti >= P.n) return;
+    const DevTensor& T = P.t[ti];
+    const int64_t start = T.numel & ~int64_t(7);
+    const int64_t e = start + threadIdx.x;
+    if (threadIdx.x < 8 && e < T.numel) {
+        const uint32_t a = (uint32_t)(T.x[e] & 0x7FFFu) << 16;
+        atomicMax(reinterpret_cast<unsigned int*>(const_cast<float*>(P.group_amax)) + T.group, a);
+        if (P.tracked) atomicMax(reinterpret_cast<unsigned int*>(P.tracked) + T.group, a);
+    }
+}
+
+// ------------------------------------------------------------------ STE identity
+__global__ void __launch_bounds__(kThreads) k_copy(const uint16_t* __restrict__ src,
+                                                   uint16_t* __restrict__ dst, int64_t n) {
+    const int64_t nvec = n >> 3;
+    const int64_t stride = int64_t(gridDim.x) * kThreads;
+    int64_t i = int64_t(blockIdx.x) * kThreads + threadIdx.x;
+    for (; i + 3 * stride < nvec; i += 4 * stride) {
+        uint4 a = ld_stream(src + 8 * i), b = ld_stream(src + 8 * (i + stride));
+        uint4 c = ld_stream(src + 8 * (i + 2 * stride)), d = ld_stream(src + 8 * (i + 3 * stride));
+        st_v4(dst + 8 * i, a);
+        st_v4(dst + 8 * (i + stride), b);
+        st_v4(dst + 8 * (i + 2 * stride), c);
+        st_v4(dst + 8 * (i + 3 * stride), d);
+    }
+    for (; i < nvec; i += stride) st_v4(dst + 8 * i, ld_stream(src + 8 * i));
+    if (blockIdx.x == 0 && threadIdx.x < (n & 7)) {
+        const int64_t e = (nvec << 3) + threadIdx.x;
+        dst[e] = src[e];
+    }
+}
+
+}  // namespace qf

@@ -1,0 +1,206 @@
+/*
+ * qf.h -- C ABI of the B200 (sm_100a) deployment-aligned simulated-quantization
+ * library (libqf.so).
+ *
+ * The library implements the hot path of quantization-aware training as
+ * described on the QATFactory project page ("QATFactory: A Versatile,
+ * Deployment-Aligned Framework for Quantization-aware Training and Distillation
+ * of LLMs"): weights, and optionally activations, are rounded onto a deployment
+ * format's grid in the forward pass (quantize-dequantize), a straight-through
+ * estimator carries the gradient to the latent weight in the backward pass, and
+ * the codes and scales are packed in the inference engine's layout.
+ *
+ * Formats ("Supported formats" table of the project page):
+ *   NVFP4  E2M1 elements, 16-element blocks, E4M3 block scale, FP32 tensor scale,
+ *          symmetric, 4.50 bits/weight
+ *   MXFP4  E2M1 elements, 32-element blocks, E8M0 block scale, symmetric,
+ *          4.25 bits/weight
+ *   Q4_K   unsigned 4-bit elements, 32-element sub-blocks in 256-element
+ *          super-blocks, 6-bit sub-block scale and min, FP16 super-block d and
+ *          dmin, asymmetric, 4.50 bits/weight
+ *
+ * Conventions common to every call
+ *   - A tensor is a row-major, contiguous BF16 matrix [rows, cols].  Blocks run
+ *     along cols (the contiguous dimension, the GEMM reduction dimension along
+ *     which the engines scale); cols must be a multiple of the format's block
+ *     (16, 32 or 256).  Since blocks never straddle rows, element i of the
+ *     tensor (flat index) belongs to block i / block_size.
+ *   - Every pointer in a qf_tensor and every d_* pointer is a DEVICE pointer on
+ *     the current CUDA device, owned by the caller.  The library allocates no
+ *     memory and keeps no pointer after a call returns.  The qf_tensor array
+ *     itself is HOST memory, read during the call only.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every call
+ *     is asynchronous on that stream.
+ *   - Arguments are validated on the host before anything is launched; an
+ *     invalid call returns an error status and launches nothing.  A CUDA launch
+ *     failure returns QF_ERR_CUDA.  Kernels never trap and contain no waits.
+ *     qf_last_error() gives a one-line description of the last failure on the
+ *     calling thread.
+ *   - Calls on the same stream are ordered; calls whose outputs overlap and that
+ *     run concurrently on different streams race.
+ *   - Numerics are fixed bit for bit (see each call); every result is
+ *     deterministic and independent of launch configuration.
+ */
+#ifndef QF_H
+#define QF_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    QF_NVFP4 = 0,
+    QF_MXFP4 = 1,
+    QF_Q4K = 2
+} qf_format;
+
+typedef enum {
+    QF_OK = 0,
+    QF_ERR_INVALID_ARG = 1,   /* null pointer, bad count, group out of range, no output */
+    QF_ERR_SHAPE = 2,         /* negative or overflowing size, cols not a block multiple */
+    QF_ERR_ALIGN = 3,         /* x / y / codes not 16-byte aligned */
+    QF_ERR_UNSUPPORTED = 4,   /* unknown format or mode */
+    QF_ERR_CUDA = 5           /* a CUDA call failed (see qf_last_error) */
+} qf_status;
+
+#define QF_NVFP4_BLOCK 16
+#define QF_MXFP4_BLOCK 32
+#define QF_Q4K_SUBBLOCK 32
+#define QF_Q4K_SUPERBLOCK 256
+#define QF_Q4K_BLOCK_BYTES 144
+
+/*
+ * One tensor of a call.
+ *   x       BF16 [rows, cols], 16-byte aligned.  May be NULL only if rows*cols == 0.
+ *   rows    >= 0
+ *   cols    >= 0, a multiple of the format's block size
+ *   group   NVFP4 tie group in [0, n_groups): every tensor of a group shares one
+ *           FP32 tensor scale (the projections an engine fuses, e.g. Q, K and V,
+ *           or gate and up -- project page, Method, "Numerics").  Ignored by
+ *           MXFP4 and Q4_K.
+ *   reserved  must be 0
+ *   y       BF16 [rows, cols] dequantized output, 16-byte aligned, or NULL
+ *   codes   packed output, 16-byte aligned, or NULL:
+ *             NVFP4 / MXFP4: rows*cols/2 bytes; element 2i of the flat tensor in
+ *               bits 0-3 of byte i, element 2i+1 in bits 4-7; each nibble is an
+ *               E2M1 code (bit 3 = sign).
+ *             Q4_K: (rows*cols/256) blocks of 144 bytes, one per super-block in
+ *               flat order: FP16 d, FP16 dmin, 12 bytes of 6-bit scales/mins,
+ *               128 bytes of 4-bit codes (the GGUF Q4_K block layout).
+ *   scales  block scales, any alignment, or NULL (ignored by Q4_K, whose scales
+ *           live inside its blocks):
+ *             NVFP4: rows*cols/16 E4M3 bytes, MXFP4: rows*cols/32 E8M0 bytes,
+ *             row-major (flat block order).
+ */
+typedef struct qf_tensor {
+    const void* x;
+    int64_t rows;
+    int64_t cols;
+    int32_t group;
+    int32_t reserved;
+    void* y;
+    void* codes;
+    void* scales;
+} qf_tensor;
+
+/*
+ * qf_amax_tied -- tied NVFP4 tensor amax (project page, Method, "Numerics": the
+ * projections that vLLM and SGLang fuse share one tensor scale; "Export": NVFP4
+ * activation scales are tracked during training and saved).
+ *
+ *   d_group_amax[g] = max over the tensors i with t[i].group == g of max |x_i|
+ *                     (FP32, exact); 0 for a group with no tensor.  Overwritten.
+ *   d_tracked       NULL, or FP32[n_groups]: updated in place to
+ *                     max(d_tracked[g], d_group_amax[g])  (the running amax a
+ *                     training loop keeps for activations; pass it as the
+ *                     d_group_amax of qf_fakequant to quantize with it).
+ *   Only x, rows, cols and group of each tensor are read; cols may be any value
+ *   >= 0 here.  n == 0 only clears d_group_amax.
+ * Errors: t == NULL with n > 0, n < 0, n_groups <= 0, d_group_amax == NULL,
+ *   group out of range -> QF_ERR_INVALID_ARG; bad sizes -> QF_ERR_SHAPE;
+ *   x not 16-byte aligned -> QF_ERR_ALIGN.
+ */
+qf_status qf_amax_tied(const qf_tensor* t, int n, float* d_group_amax, int n_groups,
+                       float* d_tracked, void* stream);
+
+/*
+ * qf_fakequant -- the fused forward pass: block statistics, block-scale encode,
+ * element encode, dequantize and pack in one read of x (project page, Method,
+ * "Framework overview": a lossy quantize-dequantize that reproduces inference
+ * numerics; "QARL"/"Export": packing in the engine's layout).  n == 1 is one
+ * tensor; n > 1 is one grouped launch over all n tensors (e.g. every expert of
+ * an MoE layer), bitwise identical to n single calls.
+ *
+ * Numerics (IEEE binary32, round to nearest even, no fused multiply-add):
+ *   NVFP4: s_t = amax_g / 2688 (= amax_g / (6 * 448)), amax_g = d_group_amax[group];
+ *          per 16-block: sb = E4M3_satfinite(amax_b / (6 * s_t)) (sb = 0 if s_t == 0),
+ *          S = f32(sb) * s_t, inv = 1 / S (0 if S == 0),
+ *          code = E2M1_satfinite(x * inv) (a zero x stays a zero of its sign),
+ *          y = BF16(f32(code) * S).
+ *   MXFP4: per 32-block: e = clamp(floor(log2 amax_b) - 2, -127, 127)
+ *          (-127 for an all-zero block), scale byte = e + 127,
+ *          code = E2M1_satfinite(x * 2^-e), y = BF16(f32(code) * 2^e).
+ *   Q4_K:  per 32-sub-block j: min_j = max(-min x, 0), scale_j = (max x + min_j) / 15;
+ *          d = FP16(max_j scale_j / 63), dmin = FP16(max_j min_j / 63);
+ *          sc_j = min(RNE(scale_j / d), 63) (0 if d == 0), m_j likewise with dmin;
+ *          s_j = d * sc_j, mm_j = dmin * m_j, inv_j = 1 / s_j (0 if s_j == 0);
+ *          q = clamp(RNE((x + mm_j) * inv_j), 0, 15), y = BF16(s_j * q - mm_j).
+ *   E2M1 codes carry the sign bit of their input (a negative value that rounds
+ *   to zero gives code 8).
+ *
+ *   d_group_amax       NVFP4: FP32[n_groups] device array of tie-group amaxes
+ *                      (from qf_amax_tied).  Ignored by MXFP4 / Q4_K (may be NULL).
+ *   n_groups           NVFP4: number of entries of d_group_amax (> 0).
+ *   d_group_scale_out  NVFP4: NULL, or FP32[n_groups] receiving each s_t.
+ * Every tensor needs at least one of y, codes, scales non-NULL.
+ * Errors: unknown format -> QF_ERR_UNSUPPORTED; see qf_tensor for the rest.
+ */
+qf_status qf_fakequant(qf_format f, const qf_tensor* t, int n, const float* d_group_amax,
+                       int n_groups, float* d_group_scale_out, void* stream);
+
+/*
+ * qf_pack -- the engine-layout export and weight sync (project page, Method,
+ * "QARL": after each step the learner packs its weights in the engine's layout
+ * and syncs them; "Export").  Identical to qf_fakequant except that y is never
+ * written (it may be non-NULL and is ignored); each tensor needs codes or scales.
+ * The bytes written are those qf_fakequant writes.
+ */
+qf_status qf_pack(qf_format f, const qf_tensor* t, int n, const float* d_group_amax,
+                  int n_groups, float* d_group_scale_out, void* stream);
+
+/*
+ * qf_ste_backward -- straight-through estimator backward (project page, Method,
+ * "Framework overview": the STE updates the continuous latent weights; Bengio,
+ * Leonard and Courville 2013, cited by the paper).
+ *   mode 0 (identity):  grad_x = grad_y, numel BF16 elements.  grad_x == grad_y
+ *                       is allowed and launches nothing.  f, fwd and
+ *                       d_group_amax are ignored.
+ *   mode 1 (clipped):   grad_x = grad_y where the forward pass did not saturate
+ *                       the element, +0 elsewhere: NVFP4/MXFP4 |x * inv| <= 6,
+ *                       Q4_K 0 <= (x + mm_j) * inv_j <= 15, with the scales the
+ *                       forward pass of format f derives for fwd->x.  fwd gives x,
+ *                       rows, cols and (NVFP4) group; numel == rows * cols;
+ *                       d_group_amax as for qf_fakequant (NVFP4 only).
+ *   grad_y, grad_x: BF16 device arrays, 16-byte aligned.
+ * Errors: mode not 0/1 or unknown format -> QF_ERR_UNSUPPORTED; the rest as above.
+ */
+qf_status qf_ste_backward(qf_format f, const void* grad_y, void* grad_x, int64_t numel,
+                          int mode, const qf_tensor* fwd, const float* d_group_amax,
+                          int n_groups, void* stream);
+
+/* Static description of a status code. */
+const char* qf_status_string(qf_status s);
+
+/* One-line description of the last failed call on the calling thread ("" if none). */
+const char* qf_last_error(void);
+
+/* ABI version: (major << 16) | minor. */
+int qf_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QF_H */

@@ -1,0 +1,145 @@
+"""The C ABI boundary on the host (no GPU needed): libqf.so loads, exports every
+entry point include/qf.h declares, and rejects invalid calls with the documented
+status codes before touching CUDA."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qf.h")
+
+
+@pytest.fixture(scope="module")
+def qf():
+    from fp4_fake_quant_b200 import _build
+    _build.build()
+    import fp4_fake_quant_b200 as mod
+    return mod
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(qf_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_hot_path_calls():
+    names = declared_functions()
+    for n in ("qf_amax_tied", "qf_fakequant", "qf_pack", "qf_ste_backward"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(qf):
+    out = subprocess.run(["nm", "-D", "--defined-only", qf.binding.LIB_PATH],
+                         capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r" T (qf_\w+)", out))
+    for n in declared_functions():
+        assert n in exported, n
+        assert hasattr(qf.lib, n)
+    assert set(qf.EXPORTS) == set(declared_functions())
+
+
+def test_header_compiles_as_c():
+    src = '#include "qf.h"\nint main(void){ qf_tensor t = {0}; (void)t; return (int)QF_OK; }\n'
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.dirname(HEADER),
+                        "-x", "c", "-", "-fsyntax-only"], input=src, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+
+
+def test_struct_layout_matches_header(qf):
+    T = qf.binding.QfTensor
+    assert ctypes.sizeof(T) == 56
+    assert T.y.offset == 32 and T.codes.offset == 40 and T.scales.offset == 48
+
+
+def test_status_strings(qf):
+    for s in range(6):
+        assert qf.lib.qf_status_string(s).decode().startswith("QF_")
+    assert qf.lib.qf_version() >> 16 == 1
+
+
+def _tensor(qf, x=0x1000, rows=4, cols=64, group=0, y=0x2000, codes=0x3000, scales=0x4000,
+            reserved=0):
+    arr = (qf.binding.QfTensor * 1)()
+    t = arr[0]
+    t.x, t.rows, t.cols, t.group, t.reserved = x, rows, cols, group, reserved
+    t.y, t.codes, t.scales = y, codes, scales
+    return arr
+
+
+def _fq(qf, f, arr, n=1, amax=None, ng=0, pack=False):
+    fn = qf.lib.qf_pack if pack else qf.lib.qf_fakequant
+    return fn(f, arr, n, amax, ng, None, None)
+
+
+@pytest.mark.parametrize("pack", [False, True])
+def test_validation_codes(qf, pack):
+    OK, INV, SHAPE, ALIGN, UNSUP = 0, 1, 2, 3, 4
+    assert _fq(qf, 7, _tensor(qf), pack=pack) == UNSUP
+    assert _fq(qf, 1, _tensor(qf), n=-1, pack=pack) == INV
+    assert _fq(qf, 1, None, n=1, pack=pack) == INV
+    assert _fq(qf, 1, _tensor(qf), n=0, pack=pack) == OK              # nothing to do
+    assert _fq(qf, 1, _tensor(qf, cols=48), pack=pack) == SHAPE        # 48 % 32
+    assert _fq(qf, 2, _tensor(qf, cols=512 + 32), pack=pack) == SHAPE  # Q4_K needs 256
+    assert _fq(qf, 0, _tensor(qf, cols=24), amax=0x5000, ng=1, pack=pack) == SHAPE
+    assert _fq(qf, 1, _tensor(qf, rows=-1), pack=pack) == SHAPE
+    assert _fq(qf, 1, _tensor(qf, rows=1 << 40, cols=1 << 30), pack=pack) == SHAPE
+    assert _fq(qf, 1, _tensor(qf, x=0x1008), pack=pack) == ALIGN
+    assert _fq(qf, 1, _tensor(qf, codes=0x3004), pack=pack) == ALIGN
+    assert _fq(qf, 1, _tensor(qf, x=0), pack=pack) == INV
+    assert _fq(qf, 1, _tensor(qf, reserved=1), pack=pack) == INV
+    assert _fq(qf, 1, _tensor(qf, y=0, codes=0, scales=0), pack=pack) == INV
+    # Q4_K ignores `scales`: a pack with no codes has no output
+    assert _fq(qf, 2, _tensor(qf, cols=256, codes=0), pack=True) == INV
+    # NVFP4 needs the group amax and a valid group
+    assert _fq(qf, 0, _tensor(qf), amax=None, ng=1, pack=pack) == INV
+    assert _fq(qf, 0, _tensor(qf), amax=0x5000, ng=0, pack=pack) == INV
+    assert _fq(qf, 0, _tensor(qf, group=1), amax=0x5000, ng=1, pack=pack) == INV
+    assert _fq(qf, 0, _tensor(qf, group=-1), amax=0x5000, ng=1, pack=pack) == INV
+    # empty tensors are skipped without needing outputs
+    assert _fq(qf, 1, _tensor(qf, rows=0, y=0, codes=0, scales=0), pack=pack) == OK
+    assert qf.lib.qf_last_error() == b""
+
+
+def test_valid_call_without_a_gpu_reports_cuda_error(qf):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert _fq(qf, 1, _tensor(qf)) == 5
+    assert qf.lib.qf_last_error().decode()
+
+
+def test_amax_and_ste_validation(qf):
+    INV, SHAPE, ALIGN, UNSUP = 1, 2, 3, 4
+    lib = qf.lib
+    arr = _tensor(qf, cols=7)                       # any cols is fine for the amax
+    assert lib.qf_amax_tied(arr, 1, None, 1, None, None) == INV
+    assert lib.qf_amax_tied(arr, 1, 0x5000, 0, None, None) == INV
+    assert lib.qf_amax_tied(_tensor(qf, group=2), 1, 0x5000, 2, None, None) == INV
+    assert lib.qf_amax_tied(_tensor(qf, x=0x1002), 1, 0x5000, 1, None, None) == ALIGN
+    assert lib.qf_amax_tied(None, 1, 0x5000, 1, None, None) == INV
+    assert lib.qf_ste_backward(0, 0x1000, 0x2000, 64, 2, None, None, 0, None) == UNSUP
+    assert lib.qf_ste_backward(0, 0x1000, 0x2000, -1, 0, None, None, 0, None) == SHAPE
+    assert lib.qf_ste_backward(0, 0x1008, 0x2000, 64, 0, None, None, 0, None) == ALIGN
+    assert lib.qf_ste_backward(0, 0, 0x2000, 64, 0, None, None, 0, None) == INV
+    assert lib.qf_ste_backward(0, 0x1000, 0x1000, 64, 0, None, None, 0, None) == 0  # aliased
+    assert lib.qf_ste_backward(9, 0x1000, 0x2000, 256, 1, _tensor(qf), None, 0, None) == UNSUP
+    assert lib.qf_ste_backward(1, 0x1000, 0x2000, 256, 1, None, None, 0, None) == INV
+    assert lib.qf_ste_backward(1, 0x1000, 0x2000, 255, 1, _tensor(qf), None, 0, None) == SHAPE
+    assert lib.qf_ste_backward(0, 0x1000, 0x2000, 256, 1, _tensor(qf), None, 1, None) == INV
+
+
+def test_product_path_has_no_oracle_dependency():
+    """The library and its binding never import, link or read the oracle."""
+    pkg = os.path.join(ROOT, "fp4_fake_quant_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "oracle" not in text.lower(), f
+    out = subprocess.run(["ldd", os.path.join(pkg, "libqf.so")], capture_output=True,
+                         text=True).stdout
+    assert "oracle" not in out
