@@ -165,3 +165,37 @@ def qf_ste_backward(grad_y: torch.Tensor, grad_x: torch.Tensor, mode: int = 0, f
     ng = group_amax.numel() if group_amax is not None else 0
     _check(lib.qf_ste_backward(_fmt(fmt), _ptr(grad_y), _ptr(grad_x), grad_y.numel(), mode, fwd,
                                _ptr(group_amax), ng, _stream(stream)))
+
+
+class Prepared:
+    """A call whose ``qf_tensor`` array and pointers are marshalled once.
+
+    Training loops re-quantize the same weight buffers every step; a prepared call
+    skips rebuilding the descriptor array (which for a grouped launch over hundreds
+    of MoE expert tensors costs more host time than the kernel takes).  The tensors
+    are kept alive by this object; calling it enqueues the same C entry point on
+    the current (or given) stream."""
+
+    def __init__(self, fn, args_before_stream, keep):
+        self._fn = fn
+        self._args = args_before_stream
+        self._keep = keep
+
+    def __call__(self, stream=None) -> None:
+        _check(self._fn(*self._args, _stream(stream)))
+
+
+def prepare_fakequant(fmt, xs, ys=None, codes=None, scales=None, groups=None, group_amax=None,
+                      group_scale_out=None, pack_only: bool = False) -> Prepared:
+    arr, n = _desc(xs, None if pack_only else ys, codes, scales, groups)
+    ng = group_amax.numel() if group_amax is not None else 0
+    fn = lib.qf_pack if pack_only else lib.qf_fakequant
+    keep = (arr, list(xs), ys, codes, scales, group_amax, group_scale_out)
+    return Prepared(fn, (_fmt(fmt), arr, n, _ptr(group_amax), ng, _ptr(group_scale_out)), keep)
+
+
+def prepare_amax_tied(xs, groups, group_amax, tracked=None) -> Prepared:
+    arr, n = _desc(xs, groups=groups)
+    keep = (arr, list(xs), group_amax, tracked)
+    return Prepared(lib.qf_amax_tied, (arr, n, _ptr(group_amax), group_amax.numel(), _ptr(tracked)),
+                    keep)

@@ -21,7 +21,6 @@ using qf::kThreads;
 constexpr int kSmallT = 8;      // descriptor table sizes (kernel-parameter bytes: ~0.6 KB / ~27 KB)
 constexpr int kLargeT = 384;
 constexpr int kFp4U = 4;        // 256-element sub-tiles per warp unit
-constexpr int kQ4kU = 2;        // super-blocks per warp unit
 constexpr int kAmaxU = 8;
 
 thread_local char g_err[512] = "";
@@ -188,8 +187,8 @@ qf_status fakequant_impl(qf_format f, const qf_tensor* t, int n, const float* d_
                                  qf::k_fp4<false, kFp4U, kLargeT, 0>, v, 256 * kFp4U, am, so,
                                  nullptr, ng, s);
         default:
-            return launch_chunks(qf::k_q4k<kQ4kU, kSmallT, 0>, qf::k_q4k<kQ4kU, kLargeT, 0>, v,
-                                 256 * kQ4kU, am, so, nullptr, ng, s);
+            return launch_chunks(qf::k_q4k<kSmallT, 0>, qf::k_q4k<kLargeT, 0>, v,
+                                 1024, am, so, nullptr, ng, s);
     }
 }
 
@@ -305,8 +304,8 @@ qf_status qf_ste_backward(qf_format f, const void* grad_y, void* grad_x, int64_t
                                  qf::k_fp4<false, kFp4U, kLargeT, 1>, v, 256 * kFp4U, nullptr,
                                  nullptr, nullptr, 0, s);
         default:
-            return launch_chunks(qf::k_q4k<kQ4kU, kSmallT, 1>, qf::k_q4k<kQ4kU, kLargeT, 1>, v,
-                                 256 * kQ4kU, nullptr, nullptr, nullptr, 0, s);
+            return launch_chunks(qf::k_q4k<kSmallT, 1>, qf::k_q4k<kLargeT, 1>, v,
+                                 1024, nullptr, nullptr, nullptr, 0, s);
     }
 }
 

@@ -199,8 +199,30 @@ __device__ __forceinline__ void fp4_lane(uint4 v, float s_t, float six_st, Fp4La
     }
 }
 
+// Loads of one warp unit (U sub-tiles of 256 elements): v = x, gv = upstream gradient
+// (STE only).  Lanes past the end of the tensor load zeros.
+template <int U, int MODE>
+struct UnitLoad {
+    uint4 v[U];
+    uint4 gv[MODE == 1 ? U : 1];
+};
+
+template <int U, int MODE>
+__device__ __forceinline__ void load_unit(const DevTensor& T, int64_t e0, int lane,
+                                          UnitLoad<U, MODE>& L) {
+#pragma unroll
+    for (int s = 0; s < U; ++s) {
+        const int64_t e = e0 + s * 256 + lane * 8;
+        const bool ok = e < T.numel;
+        L.v[s] = ok ? ld_stream(T.x + e) : make_uint4(0, 0, 0, 0);
+        if (MODE == 1) L.gv[s] = ok ? ld_stream(T.g + e) : make_uint4(0, 0, 0, 0);
+    }
+}
+
 // Fused NVFP4 / MXFP4 fake-quant + pack (MODE 0) or clipped STE (MODE 1).
-// A unit is U sub-tiles of 256 elements.
+// A unit is U sub-tiles of 256 elements.  The loads of a warp's next unit are
+// issued before the current one is computed, so every warp keeps a unit of
+// reads in flight while it converts.
 template <bool NV, int U, int MAXT, int MODE>
 __global__ void __launch_bounds__(kThreads) k_fp4(const __grid_constant__ Table<MAXT> P) {
     const int lane = threadIdx.x & 31;
@@ -211,43 +233,47 @@ __global__ void __launch_bounds__(kThreads) k_fp4(const __grid_constant__ Table<
         for (int g = threadIdx.x; g < P.n_groups; g += kThreads)
             P.group_scale_out[g] = nv_tensor_scale(P.group_amax[g]);
     }
-    int ti = 0, cur = -1;
+    int64_t u = warp;
+    if (u >= P.total_units) return;
+    int ti = find_tensor(P, 0, u);
+    UnitLoad<U, MODE> cur;
+    load_unit<U, MODE>(P.t[ti], (u - P.t[ti].unit_begin) * kUnit, lane, cur);
+    int cur_t = -1;
     float s_t = 0.0f, six_st = 0.0f;
-    for (int64_t u = warp; u < P.total_units; u += nwarps) {
-        ti = find_tensor(P, ti, u);
+    while (true) {
+        // prefetch the next unit of this warp
+        const int64_t un = u + nwarps;
+        int tn = ti;
+        UnitLoad<U, MODE> nxt;
+        if (un < P.total_units) {
+            tn = find_tensor(P, ti, un);
+            load_unit<U, MODE>(P.t[tn], (un - P.t[tn].unit_begin) * kUnit, lane, nxt);
+        }
         const DevTensor& T = P.t[ti];
-        if (NV && ti != cur) {
+        if (NV && ti != cur_t) {
             s_t = nv_tensor_scale(P.group_amax[T.group]);
             six_st = __fmul_rn(6.0f, s_t);
-            cur = ti;
+            cur_t = ti;
         }
         const int64_t e0 = (u - T.unit_begin) * kUnit;
-        uint4 v[U], gv[U];
-        bool ok[U];
 #pragma unroll
         for (int s = 0; s < U; ++s) {
             const int64_t e = e0 + s * 256 + lane * 8;
-            ok[s] = e < T.numel;
-            v[s] = ok[s] ? ld_stream(T.x + e) : make_uint4(0, 0, 0, 0);
-            if (MODE == 1) gv[s] = ok[s] ? ld_stream(T.g + e) : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int s = 0; s < U; ++s) {
-            const int64_t e = e0 + s * 256 + lane * 8;
+            const bool ok = e < T.numel;
             Fp4Lane o;
             if (MODE == 0) {
-                if (T.y) fp4_lane<NV, true>(v[s], s_t, six_st, o);
-                else fp4_lane<NV, false>(v[s], s_t, six_st, o);
-                if (ok[s]) {
+                if (T.y) fp4_lane<NV, true>(cur.v[s], s_t, six_st, o);
+                else fp4_lane<NV, false>(cur.v[s], s_t, six_st, o);
+                if (ok) {
                     if (T.y) st_v4(T.y + e, o.y);
                     if (T.codes) *reinterpret_cast<uint32_t*>(T.codes + (e >> 1)) = o.codes;
                     if (T.scales && (lane & (NV ? 1 : 3)) == 0)
                         T.scales[e >> (NV ? 4 : 5)] = (uint8_t)o.scale;
                 }
             } else {
-                fp4_lane<NV, false>(v[s], s_t, six_st, o);
-                if (ok[s]) {
-                    const uint32_t gw[4] = {gv[s].x, gv[s].y, gv[s].z, gv[s].w};
+                fp4_lane<NV, false>(cur.v[s], s_t, six_st, o);
+                if (ok) {
+                    const uint32_t gw[4] = {cur.gv[s].x, cur.gv[s].y, cur.gv[s].z, cur.gv[s].w};
                     uint32_t r[4];
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
@@ -259,141 +285,196 @@ __global__ void __launch_bounds__(kThreads) k_fp4(const __grid_constant__ Table<
                 }
             }
         }
+        if (un >= P.total_units) break;
+        u = un;
+        ti = tn;
+        cur = nxt;
     }
 }
 
 // ------------------------------------------------------------------ Q4_K
-// One warp per 256-element super-block: lane l holds elements 8l..8l+7, i.e.
-// sub-block j = l / 4.
-struct Q4kLane {
-    uint4 y;
-    uint32_t qs;        // this lane's 4 bytes of the 128-byte code area
-    uint32_t hdr;       // lanes 0..3: word l of the 16-byte header
-    float v[8];         // scaled values (for the clipped STE)
-};
+// One lane per 32-element sub-block: a warp iteration covers 4 super-blocks (1024
+// elements) and lane l owns sub-block j = l / 4 of super-block b = l % 4, so the
+// per-sub-block and per-super-block scalar work (divides, FP16 and integer
+// conversions) is amortised over 32 elements instead of 8.  Global loads and
+// stores stay fully coalesced: the warp stages its 2 KB through shared memory
+// (one 528-byte row per super-block, 16 bytes of padding so that the lanes'
+// 16-byte accesses hit distinct banks) and transposes there.
+constexpr int kQ4kRow = 528;
+constexpr int kQ4kWarpBytes = 4 * kQ4kRow;
+constexpr float kRound = 12582912.0f;      // 1.5 * 2^23: v + kRound rounds v to an integer (RNE)
 
-template <bool WANT_Y>
-__device__ __forceinline__ void q4k_lane(uint4 xv, int lane, Q4kLane& o) {
-    const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w};
-    // sub-block max and min: pack (max, -min) as bf16x2 and reduce both with one max
-    uint32_t mx = bmax2(bmax2(w[0], w[1]), bmax2(w[2], w[3]));
-    uint32_t mn = bmin2(bmin2(w[0], w[1]), bmin2(w[2], w[3]));
-    uint32_t hi = bmax2(mx, mx >> 16) & 0xFFFFu;            // bf16 bits of max
-    uint32_t lo = bmin2(mn, mn >> 16) & 0xFFFFu;            // bf16 bits of min
-    uint32_t pk = (hi << 16) | (lo ^ 0x8000u);              // (max, -min)
-    pk = bmax2(pk, __shfl_xor_sync(kFull, pk, 1));
-    pk = bmax2(pk, __shfl_xor_sync(kFull, pk, 2));
-    const float hi_f = bf16_hi(pk);
-    const float negmin = bf16_lo(pk);
-    const float min_j = negmin > 0.0f ? negmin : 0.0f;
-    const float scale_j = __fdiv_rn(__fadd_rn(hi_f, min_j), 15.0f);
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
+    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w) : "memory");
+}
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z),
+                 "=r"(v.w) : "r"(addr) : "memory");
+    return v;
+}
+
+// Per-lane fit of one sub-block (32 BF16 in w[16]); returns the super-block's FP16
+// d / dmin bits, this sub-block's 6-bit sc / m, its s = d*sc, mm = dmin*m, inv = 1/s.
+struct Q4kFit { uint32_t dbits, dminbits, sc, m; float s, mm, inv; };
+
+__device__ __forceinline__ Q4kFit q4k_fit(const uint32_t (&w)[16]) {
+    uint32_t mx = w[0], mn = w[0];
+#pragma unroll
+    for (int k = 1; k < 16; ++k) { mx = bmax2(mx, w[k]); mn = bmin2(mn, w[k]); }
+    const float hi = fmaxf(bf16_lo(mx), bf16_hi(mx));
+    const float lo = fminf(bf16_lo(mn), bf16_hi(mn));
+    const float min_j = lo < 0.0f ? -lo : 0.0f;
+    const float scale_j = __fdiv_rn(__fadd_rn(hi, min_j), 15.0f);
     float ms = scale_j, mm = min_j;
 #pragma unroll
-    for (int o2 = 4; o2 < 32; o2 <<= 1) {
-        ms = fmaxf(ms, __shfl_xor_sync(kFull, ms, o2));
-        mm = fmaxf(mm, __shfl_xor_sync(kFull, mm, o2));
+    for (int o = 4; o < 32; o <<= 1) {               // the 8 lanes of this super-block
+        ms = fmaxf(ms, __shfl_xor_sync(kFull, ms, o));
+        mm = fmaxf(mm, __shfl_xor_sync(kFull, mm, o));
     }
     const __half dh = __float2half_rn(__fdiv_rn(ms, 63.0f));
     const __half dmh = __float2half_rn(__fdiv_rn(mm, 63.0f));
     const float d = __half2float(dh), dmin = __half2float(dmh);
-    const int sc = d == 0.0f ? 0 : min(__float2int_rn(__fdiv_rn(scale_j, d)), 63);
-    const int m = dmin == 0.0f ? 0 : min(__float2int_rn(__fdiv_rn(min_j, dmin)), 63);
-    const float s = __fmul_rn(d, (float)sc);
-    const float mmv = __fmul_rn(dmin, (float)m);
-    const float inv = s == 0.0f ? 0.0f : __frcp_rn(s);
-    // elements: q = clamp(RNE((x + mm) * inv), 0, 15) via the 1.5*2^23 rounding constant
-    uint32_t qb[8];
-    float yk[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        const float xk = (k & 1) ? bf16_hi(w[k >> 1]) : bf16_lo(w[k >> 1]);
-        const float t = __fmul_rn(__fadd_rn(xk, mmv), inv);
-        o.v[k] = t;
-        const float r = __fadd_rn(fminf(fmaxf(t, 0.0f), 15.0f), 12582912.0f);
-        qb[k] = __float_as_uint(r) & 15u;
-        // r - 1.5*2^23 is the integer code q as a float (exact)
-        yk[k] = __fsub_rn(__fmul_rn(s, __fsub_rn(r, 12582912.0f)), mmv);
-    }
-    if (WANT_Y)
-        o.y = make_uint4(cvt_bf16x2(yk[1], yk[0]), cvt_bf16x2(yk[3], yk[2]),
-                         cvt_bf16x2(yk[5], yk[4]), cvt_bf16x2(yk[7], yk[6]));
-    // codes: byte p of chunk c = q[2c][p] | q[2c+1][p] << 4; pair lane l with l ^ 4
-    const uint32_t B0 = qb[0] | (qb[1] << 8) | (qb[2] << 16) | (qb[3] << 24);
-    const uint32_t B1 = qb[4] | (qb[5] << 8) | (qb[6] << 16) | (qb[7] << 24);
-    const bool odd = (lane >> 2) & 1;
-    const uint32_t recv = __shfl_xor_sync(kFull, odd ? B0 : B1, 4);
-    o.qs = odd ? (recv | (B1 << 4)) : (B0 | (recv << 4));
-    // header: d, dmin, then 12 bytes of 6-bit scales and mins
-    const uint32_t smv = (uint32_t)sc | ((uint32_t)m << 8);
-    const uint32_t A = __shfl_sync(kFull, smv, 4 * (lane & 7));          // lane l<8: sub-block l
-    const uint32_t Bv = __shfl_sync(kFull, A, (lane & 3) + 4);            // sub-block (l&3)+4
-    const uint32_t scA = A & 0xFF, mA = A >> 8, scB = Bv & 0xFF, mB = Bv >> 8;
-    const uint32_t pb = ((scA & 63) | ((scB >> 4) << 6)) |
-                        (((mA & 63) | ((mB >> 4) << 6)) << 8) |
-                        (((scB & 15) | ((mB & 15) << 4)) << 16);
-    // transpose: word 1+r gathers byte r of lanes 0..3
-    const uint32_t p0 = __shfl_sync(kFull, pb, 0), p1 = __shfl_sync(kFull, pb, 1);
-    const uint32_t p2 = __shfl_sync(kFull, pb, 2), p3 = __shfl_sync(kFull, pb, 3);
-    // lane 1..3 takes byte slot r = lane-1 of lanes 0..3 (lane 0 writes d, dmin)
-    const uint32_t r = ((uint32_t)(lane & 3) + 3u) & 3u;
-    const uint32_t sel = r | ((r + 4u) << 4);               // byte r of each operand
-    const uint32_t w01 = __byte_perm(p0, p1, sel);
-    const uint32_t w23 = __byte_perm(p2, p3, sel);
-    const uint32_t word = __byte_perm(w01, w23, 0x5410u);
-    o.hdr = (lane & 3) == 0
-                ? ((uint32_t)__half_as_ushort(dh) | ((uint32_t)__half_as_ushort(dmh) << 16))
-                : word;
+    Q4kFit f;
+    f.dbits = __half_as_ushort(dh);
+    f.dminbits = __half_as_ushort(dmh);
+    f.sc = d == 0.0f ? 0u : (uint32_t)min(__float2int_rn(__fdiv_rn(scale_j, d)), 63);
+    f.m = dmin == 0.0f ? 0u : (uint32_t)min(__float2int_rn(__fdiv_rn(min_j, dmin)), 63);
+    f.s = __fmul_rn(d, (float)f.sc);
+    f.mm = __fmul_rn(dmin, (float)f.m);
+    f.inv = f.s == 0.0f ? 0.0f : __frcp_rn(f.s);
+    return f;
 }
 
-template <int U, int MAXT, int MODE>
+// MODE 0: dequant (y) and/or 144-byte blocks (codes).  MODE 1: clipped STE, y = grad_x.
+template <int MAXT, int MODE>
 __global__ void __launch_bounds__(kThreads) k_q4k(const __grid_constant__ Table<MAXT> P) {
+    __shared__ __align__(16) uint8_t stage[kThreads / 32][kQ4kWarpBytes];
     const int lane = threadIdx.x & 31;
+    const int b = lane & 3, j = lane >> 2;              // super-block of 4, sub-block of 8
+    const uint32_t sm = (uint32_t)__cvta_generic_to_shared(stage[threadIdx.x >> 5]);
+    const uint32_t sm_lane = sm + 16u * lane;           // coalesced view: row k at + k*528
+    const uint32_t sm_mine = sm + b * kQ4kRow + 64u * j; // this lane's 64-byte sub-block
     const int64_t warp = (int64_t(blockIdx.x) * kThreads + threadIdx.x) >> 5;
     const int64_t nwarps = (int64_t(gridDim.x) * kThreads) >> 5;
-    constexpr int kUnit = 256 * U;
     int ti = 0;
     for (int64_t u = warp; u < P.total_units; u += nwarps) {
         ti = find_tensor(P, ti, u);
         const DevTensor& T = P.t[ti];
-        const int64_t e0 = (u - T.unit_begin) * kUnit;
-        uint4 v[U], gv[U];
-        bool ok[U];
+        const int64_t e0 = (u - T.unit_begin) * 1024;
+        const int64_t left = (T.numel - e0) >> 8;
+        const int nsb = left < 4 ? (int)left : 4;          // super-blocks in this unit
+        uint4 v[4];
 #pragma unroll
-        for (int s = 0; s < U; ++s) {
-            const int64_t e = e0 + s * 256 + lane * 8;
-            ok[s] = (e0 + s * 256) < T.numel;            // a whole super-block or nothing
-            v[s] = ok[s] ? ld_stream(T.x + e) : make_uint4(0, 0, 0, 0);
-            if (MODE == 1) gv[s] = ok[s] ? ld_stream(T.g + e) : make_uint4(0, 0, 0, 0);
+        for (int k = 0; k < 4; ++k)
+            v[k] = k < nsb ? ld_stream(T.x + e0 + 256 * k + 8 * lane) : make_uint4(0, 0, 0, 0);
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 4; ++k) sts128(sm_lane + k * kQ4kRow, v[k]);
+        __syncwarp();
+        uint32_t w[16];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const uint4 t = lds128(sm_mine + 16 * p);
+            w[4 * p] = t.x; w[4 * p + 1] = t.y; w[4 * p + 2] = t.z; w[4 * p + 3] = t.w;
         }
+        const Q4kFit f = q4k_fit(w);
+        const bool have = b < nsb;
+        const int64_t sb = (e0 >> 8) + b;                // this lane's super-block in the tensor
+        if (MODE == 0) {
+            // elements: q = clamp(RNE((x + mm) * inv), 0, 15); y = BF16(s*q - mm)
+            uint32_t qw[8];                              // q of elements 4t..4t+3, one per byte
+            uint32_t yw[16];
 #pragma unroll
-        for (int s = 0; s < U; ++s) {
-            if (!ok[s]) continue;                          // warp-uniform
-            const int64_t sb = (e0 >> 8) + s;              // super-block index in the tensor
-            const int64_t e = e0 + s * 256 + lane * 8;
-            Q4kLane o;
-            if (MODE == 0) {
-                if (T.y) q4k_lane<true>(v[s], lane, o);
-                else q4k_lane<false>(v[s], lane, o);
-                if (T.y) st_v4(T.y + e, o.y);
-                if (T.codes) {
-                    uint8_t* blk = T.codes + sb * 144;
-                    const int off = 16 + 32 * (lane >> 3) + 8 * (lane & 3) + 4 * ((lane >> 2) & 1);
-                    *reinterpret_cast<uint32_t*>(blk + off) = o.qs;
-                    if (lane < 4) *reinterpret_cast<uint32_t*>(blk + 4 * lane) = o.hdr;
-                }
-            } else {
-                q4k_lane<false>(v[s], lane, o);
-                const uint32_t gw[4] = {gv[s].x, gv[s].y, gv[s].z, gv[s].w};
-                uint32_t r[4];
+            for (int k = 0; k < 16; ++k) {
+                float r[2];
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float a = o.v[2 * k], b = o.v[2 * k + 1];
-                    uint32_t lo = (a >= 0.0f && a <= 15.0f) ? (gw[k] & 0xFFFFu) : 0u;
-                    uint32_t hi = (b >= 0.0f && b <= 15.0f) ? (gw[k] & 0xFFFF0000u) : 0u;
-                    r[k] = lo | hi;
+                for (int h = 0; h < 2; ++h) {
+                    const float x = h ? bf16_hi(w[k]) : bf16_lo(w[k]);
+                    const float t = __fmul_rn(__fadd_rn(x, f.mm), f.inv);
+                    r[h] = __fadd_rn(fminf(fmaxf(t, 0.0f), 15.0f), kRound);
                 }
-                st_v4(T.y + e, make_uint4(r[0], r[1], r[2], r[3]));
+                if (k & 1) qw[k >> 1] = __byte_perm(qw[k >> 1], __byte_perm(__float_as_uint(r[0]),
+                                                    __float_as_uint(r[1]), 0x0040), 0x5410);
+                else qw[k >> 1] = __byte_perm(__float_as_uint(r[0]), __float_as_uint(r[1]), 0x0040);
+                yw[k] = cvt_bf16x2(__fsub_rn(__fmul_rn(f.s, __fsub_rn(r[1], kRound)), f.mm),
+                                   __fsub_rn(__fmul_rn(f.s, __fsub_rn(r[0], kRound)), f.mm));
             }
+            if (T.y) {
+                // stage y back through this lane's own 64 bytes, then store coalesced
+#pragma unroll
+                for (int p = 0; p < 4; ++p)
+                    sts128(sm_mine + 16 * p, make_uint4(yw[4 * p], yw[4 * p + 1], yw[4 * p + 2],
+                                                        yw[4 * p + 3]));
+                __syncwarp();
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    if (k < nsb) st_v4(T.y + e0 + 256 * k + 8 * lane, lds128(sm_lane + k * kQ4kRow));
+            }
+            if (T.codes) {
+                // codes: byte l of chunk c = q[2c][l] | q[2c+1][l] << 4; the even sub-block's
+                // lane writes bytes 0-15 of the chunk, the odd one bytes 16-31 (partner = lane ^ 4)
+                const bool odd = j & 1;
+                uint32_t out[4];
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    const uint32_t recv = __shfl_xor_sync(kFull, odd ? qw[t] : qw[4 + t], 4);
+                    out[t] = odd ? (recv | (qw[4 + t] << 4)) : (qw[t] | (recv << 4));
+                }
+                uint8_t* blk = T.codes + sb * 144;
+                if (have) st_v4(blk + 16 + 16 * j, make_uint4(out[0], out[1], out[2], out[3]));
+                // header: d, dmin, then the 12 bytes of 6-bit scales and mins
+                const uint32_t smv = f.sc | (f.m << 8);
+                const uint32_t o4 = __shfl_xor_sync(kFull, smv, 16);      // sub-block j ^ 4
+                const uint32_t scB = o4 & 0xFF, mB = o4 >> 8;
+                const uint32_t pk = ((f.sc & 63) | ((scB >> 4) << 6)) |
+                                    (((f.m & 63) | ((mB >> 4) << 6)) << 8) |
+                                    (((scB & 15) | ((mB & 15) << 4)) << 16);
+                const uint32_t p1 = __shfl_sync(kFull, pk, b + 4);
+                const uint32_t p2 = __shfl_sync(kFull, pk, b + 8);
+                const uint32_t p3 = __shfl_sync(kFull, pk, b + 12);
+                if (j == 0 && have) {
+                    const uint32_t l1 = __byte_perm(pk, p1, 0x0040), h1 = __byte_perm(p2, p3, 0x0040);
+                    const uint32_t l2 = __byte_perm(pk, p1, 0x0051), h2 = __byte_perm(p2, p3, 0x0051);
+                    const uint32_t l3 = __byte_perm(pk, p1, 0x0062), h3 = __byte_perm(p2, p3, 0x0062);
+                    st_v4(blk, make_uint4(f.dbits | (f.dminbits << 16), __byte_perm(l1, h1, 0x5410),
+                                          __byte_perm(l2, h2, 0x5410), __byte_perm(l3, h3, 0x5410)));
+                }
+            }
+        } else {
+            // clipped STE: keep grad where 0 <= (x + mm) * inv <= 15
+            uint32_t keep = 0;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const float t0 = __fmul_rn(__fadd_rn(bf16_lo(w[k]), f.mm), f.inv);
+                const float t1 = __fmul_rn(__fadd_rn(bf16_hi(w[k]), f.mm), f.inv);
+                keep |= (uint32_t)(t0 >= 0.0f && t0 <= 15.0f) << (2 * k);
+                keep |= (uint32_t)(t1 >= 0.0f && t1 <= 15.0f) << (2 * k + 1);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                v[k] = k < nsb ? ld_stream(T.g + e0 + 256 * k + 8 * lane) : make_uint4(0, 0, 0, 0);
+            __syncwarp();
+#pragma unroll
+            for (int k = 0; k < 4; ++k) sts128(sm_lane + k * kQ4kRow, v[k]);
+            __syncwarp();
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                uint4 g = lds128(sm_mine + 16 * p);
+                uint32_t* gw = reinterpret_cast<uint32_t*>(&g);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int k = 4 * p + q;
+                    gw[q] = (((keep >> (2 * k)) & 1u) ? (gw[q] & 0xFFFFu) : 0u) |
+                            (((keep >> (2 * k + 1)) & 1u) ? (gw[q] & 0xFFFF0000u) : 0u);
+                }
+                sts128(sm_mine + 16 * p, g);
+            }
+            __syncwarp();
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                if (k < nsb) st_v4(T.y + e0 + 256 * k + 8 * lane, lds128(sm_lane + k * kQ4kRow));
         }
     }
 }
@@ -405,9 +486,13 @@ __global__ void __launch_bounds__(kThreads) k_q4k(const __grid_constant__ Table<
 template <int U, int MAXT>
 __global__ void __launch_bounds__(kThreads) k_amax(const __grid_constant__ Table<MAXT> P) {
     const int lane = threadIdx.x & 31;
-    const int64_t warp = (int64_t(blockIdx.x) * kThreads + threadIdx.x) >> 5;
-    const int64_t nwarps = (int64_t(gridDim.x) * kThreads) >> 5;
     constexpr int kUnit = 256 * U;
+    constexpr int kWarps = kThreads / 32;
+    // each CTA reduces one contiguous range of units, so a warp stays inside one
+    // tensor (one tie group) for many units and flushes its max rarely
+    const int64_t per_cta = (P.total_units + gridDim.x - 1) / gridDim.x;
+    const int64_t u_begin = int64_t(blockIdx.x) * per_cta;
+    const int64_t u_end = min(u_begin + per_cta, P.total_units);
     float* amax = const_cast<float*>(P.group_amax);
     int ti = 0, g = -1;
     uint32_t run = 0;          // bf16x2 running max of |x|
@@ -421,7 +506,7 @@ __global__ void __launch_bounds__(kThreads) k_amax(const __grid_constant__ Table
         }
         run = 0;
     };
-    for (int64_t u = warp; u < P.total_units; u += nwarps) {
+    for (int64_t u = u_begin + (threadIdx.x >> 5); u < u_end; u += kWarps) {
         ti = find_tensor(P, ti, u);
         const DevTensor& T = P.t[ti];
         if (T.group != g) {
