@@ -135,6 +135,19 @@ def traffic_for(kernel: str, workload: str):
     return None
 
 
+def max_over_ranks(vals, device):
+    """Element-wise max over all ranks (device timings are reported as the slowest rank)."""
+    t = torch.tensor(vals, dtype=torch.float64, device=device)
+    if torch.distributed.is_initialized() and torch.distributed.get_world_size() > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def weak_scaling_value(step_bytes: float, world: int, ms_per_step: float) -> float:
+    """Whole-job GB/s: every rank processes its own step of `step_bytes` per slowest step."""
+    return world * step_bytes / (ms_per_step * 1e-3) / 1e9
+
+
 # ----------------------------------------------------------------------------- workloads
 _CACHE = {}
 
@@ -247,12 +260,9 @@ def run_ours(args, rank, world, local_rank):
     step_ms = [a.elapsed_time(c) for a, b, c in ev]
     fq_ms = [b.elapsed_time(c) for a, b, c in ev]
     total_ms = sum(step_ms) if flush_buf is not None else ev[0][0].elapsed_time(ev[-1][2])
-    t = torch.tensor([total_ms, float(np.mean(fq_ms))], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    total_ms, kern_ms = float(t[0]), float(t[1])
+    total_ms, kern_ms = max_over_ranks([total_ms, float(np.mean(fq_ms))], dev)
     ms_per_step = total_ms / args.steps
-    value = world * step_bytes / (ms_per_step * 1e-3) / 1e9
+    value = weak_scaling_value(step_bytes, world, ms_per_step)
 
     # end to end through the public API with pinned host buffers
     outs_h = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in W["outs"]]
@@ -275,13 +285,11 @@ def run_ours(args, rank, world, local_rank):
         e2e_step()
     b.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = torch.tensor([a.elapsed_time(b) / e2e_steps], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(e2e_ms, op=torch.distributed.ReduceOp.MAX)
-    e2e = {"value": world * step_bytes / (float(e2e_ms) * 1e-3) / 1e9, "unit": UNIT,
+    e2e_ms = max_over_ranks([a.elapsed_time(b) / e2e_steps], dev)[0]
+    e2e = {"value": weak_scaling_value(step_bytes, world, e2e_ms), "unit": UNIT,
            "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in W["xs"]),
            "d2h_bytes_per_step": sum(o.numel() * o.element_size() for o in W["outs"]),
-           "steps": e2e_steps, "ms_per_step": float(e2e_ms)}
+           "steps": e2e_steps, "ms_per_step": e2e_ms}
 
     peak, peak_kind = peaks()
     achieved = W["fq_bytes"] / (kern_ms * 1e-3) / 1e9

@@ -20,7 +20,7 @@ using qf::kThreads;
 
 constexpr int kSmallT = 8;      // descriptor table sizes (kernel-parameter bytes: ~0.6 KB / ~27 KB)
 constexpr int kLargeT = 384;
-constexpr int kFp4U = 4;        // 256-element sub-tiles per warp unit
+constexpr int kFp4U = QF_FP4_U;  // 256-element sub-tiles per warp unit
 constexpr int kAmaxU = 8;
 
 thread_local char g_err[512] = "";
@@ -41,27 +41,29 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 int block_of(qf_format f) { return f == QF_NVFP4 ? 16 : f == QF_MXFP4 ? 32 : 256; }
 
-// Resident CTAs per SM for a kernel on the current device, and the SM count.
-struct Launch { int sms; int per_sm; };
+// Launch shape of one kernel: SM count, resident CTAs per SM, CTA size, waves.
+struct Launch { int sms; int per_sm; int threads; int waves; };
 template <typename K>
-qf_status launch_shape(K kernel, Launch* L) {
+qf_status launch_shape(K kernel, int threads, int waves, Launch* L) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
     e = cudaDeviceGetAttribute(&L->sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&L->per_sm, kernel, kThreads, 0);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&L->per_sm, kernel, threads, 0);
     if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
     if (L->per_sm < 1) L->per_sm = 1;
+    L->threads = threads;
+    L->waves = waves;
     return QF_OK;
 }
 
-// Persistent grid: enough CTAs to fill every SM, never more than there is work.
+// Grid: one warp per unit, capped at `waves` CTAs per resident slot (1 = persistent).
 int grid_for(const Launch& L, int64_t units) {
-    const int64_t warps_per_cta = kThreads / 32;
+    const int64_t warps_per_cta = L.threads / 32;
     int64_t want = (units + warps_per_cta - 1) / warps_per_cta;
-    int64_t cap = int64_t(L.sms) * L.per_sm;
-    return (int)std::max<int64_t>(1, std::min(want, cap));
+    int64_t cap = int64_t(L.sms) * L.per_sm * L.waves;
+    return (int)std::max<int64_t>(1, std::min<int64_t>(std::min<int64_t>(want, cap), INT32_MAX));
 }
 
 template <int MAXT>
@@ -82,13 +84,13 @@ void fill_table(Table<MAXT>& P, const std::vector<DevTensor>& v, size_t begin, s
 
 // Launch `kernel<MAXT>` over v in chunks of at most kLargeT tensors.
 template <typename KS, typename KL>
-qf_status launch_chunks(KS small_kernel, KL large_kernel, const std::vector<DevTensor>& v,
-                        int64_t unit_elems, const float* amax, float* scale_out, float* tracked,
-                        int n_groups, cudaStream_t s) {
+qf_status launch_chunks(KS small_kernel, KL large_kernel, int threads, int waves,
+                        const std::vector<DevTensor>& v, int64_t unit_elems, const float* amax,
+                        float* scale_out, float* tracked, int n_groups, cudaStream_t s) {
     Launch Ls, Ll;
-    qf_status st = launch_shape(small_kernel, &Ls);
+    qf_status st = launch_shape(small_kernel, threads, waves, &Ls);
     if (st != QF_OK) return st;
-    st = launch_shape(large_kernel, &Ll);
+    st = launch_shape(large_kernel, threads, waves, &Ll);
     if (st != QF_OK) return st;
     if (v.empty() && scale_out) {
         // nothing to quantize, but the per-group tensor scales are still reported
@@ -97,7 +99,7 @@ qf_status launch_chunks(KS small_kernel, KL large_kernel, const std::vector<DevT
         P.group_amax = amax;
         P.group_scale_out = scale_out;
         P.n_groups = n_groups;
-        small_kernel<<<1, kThreads, 0, s>>>(P);
+        small_kernel<<<1, threads, 0, s>>>(P);
     }
     for (size_t b = 0; b < v.size(); b += kLargeT) {
         const size_t cnt = std::min<size_t>(kLargeT, v.size() - b);
@@ -106,12 +108,12 @@ qf_status launch_chunks(KS small_kernel, KL large_kernel, const std::vector<DevT
             Table<kSmallT> P;
             fill_table(P, v, b, cnt, unit_elems);
             P.group_amax = amax; P.group_scale_out = so; P.tracked = tracked; P.n_groups = n_groups;
-            small_kernel<<<grid_for(Ls, P.total_units), kThreads, 0, s>>>(P);
+            small_kernel<<<grid_for(Ls, P.total_units), threads, 0, s>>>(P);
         } else {
             Table<kLargeT> Q;              // ~27 KB kernel parameter
             fill_table(Q, v, b, cnt, unit_elems);
             Q.group_amax = amax; Q.group_scale_out = so; Q.tracked = tracked; Q.n_groups = n_groups;
-            large_kernel<<<grid_for(Ll, Q.total_units), kThreads, 0, s>>>(Q);
+            large_kernel<<<grid_for(Ll, Q.total_units), threads, 0, s>>>(Q);
         }
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
@@ -137,6 +139,43 @@ qf_status check_tensor(const qf_tensor& t, int i, int need_cols_multiple, int n_
     if (check_group && (t.group < 0 || t.group >= n_groups))
         return fail(QF_ERR_INVALID_ARG, "tensor %d: group %d outside [0, %d)", i, t.group, n_groups);
     return QF_OK;
+}
+
+// The kernels of each format with their launch shapes.
+template <int MAXT, int MODE>
+constexpr auto nv_kernel() {
+    return qf::k_fp4<true, kFp4U, MAXT, MODE, QF_NV_THREADS, QF_NV_PREFETCH>;
+}
+template <int MAXT, int MODE>
+constexpr auto mx_kernel() {
+    return qf::k_fp4<false, kFp4U, MAXT, MODE, QF_MX_THREADS, QF_MX_PREFETCH>;
+}
+template <int MAXT, int MODE>
+constexpr auto q4k_kernel() {
+    return qf::k_q4k<MAXT, MODE, QF_Q4K_THREADS>;
+}
+
+qf_status launch_format(qf_format f, int mode, const std::vector<DevTensor>& v, const float* am,
+                        float* so, int ng, cudaStream_t s) {
+    if (f == QF_NVFP4) {
+        if (mode == 0)
+            return launch_chunks(nv_kernel<kSmallT, 0>(), nv_kernel<kLargeT, 0>(), QF_NV_THREADS,
+                                 QF_NV_WAVES, v, 256 * kFp4U, am, so, nullptr, ng, s);
+        return launch_chunks(nv_kernel<kSmallT, 1>(), nv_kernel<kLargeT, 1>(), QF_NV_THREADS,
+                             QF_NV_WAVES, v, 256 * kFp4U, am, nullptr, nullptr, ng, s);
+    }
+    if (f == QF_MXFP4) {
+        if (mode == 0)
+            return launch_chunks(mx_kernel<kSmallT, 0>(), mx_kernel<kLargeT, 0>(), QF_MX_THREADS,
+                                 QF_MX_WAVES, v, 256 * kFp4U, nullptr, nullptr, nullptr, 0, s);
+        return launch_chunks(mx_kernel<kSmallT, 1>(), mx_kernel<kLargeT, 1>(), QF_MX_THREADS,
+                             QF_MX_WAVES, v, 256 * kFp4U, nullptr, nullptr, nullptr, 0, s);
+    }
+    if (mode == 0)
+        return launch_chunks(q4k_kernel<kSmallT, 0>(), q4k_kernel<kLargeT, 0>(), QF_Q4K_THREADS,
+                             QF_Q4K_WAVES, v, 1024, nullptr, nullptr, nullptr, 0, s);
+    return launch_chunks(q4k_kernel<kSmallT, 1>(), q4k_kernel<kLargeT, 1>(), QF_Q4K_THREADS,
+                         QF_Q4K_WAVES, v, 1024, nullptr, nullptr, nullptr, 0, s);
 }
 
 qf_status fakequant_impl(qf_format f, const qf_tensor* t, int n, const float* d_group_amax,
@@ -178,18 +217,7 @@ qf_status fakequant_impl(qf_format f, const qf_tensor* t, int n, const float* d_
     const float* am = nv ? d_group_amax : nullptr;
     const int ng = nv ? n_groups : 0;
     if (v.empty() && !so) return QF_OK;
-    switch (f) {
-        case QF_NVFP4:
-            return launch_chunks(qf::k_fp4<true, kFp4U, kSmallT, 0>, qf::k_fp4<true, kFp4U, kLargeT, 0>,
-                                 v, 256 * kFp4U, am, so, nullptr, ng, s);
-        case QF_MXFP4:
-            return launch_chunks(qf::k_fp4<false, kFp4U, kSmallT, 0>,
-                                 qf::k_fp4<false, kFp4U, kLargeT, 0>, v, 256 * kFp4U, am, so,
-                                 nullptr, ng, s);
-        default:
-            return launch_chunks(qf::k_q4k<kSmallT, 0>, qf::k_q4k<kLargeT, 0>, v,
-                                 1024, am, so, nullptr, ng, s);
-    }
+    return launch_format(f, 0, v, am, so, ng, s);
 }
 
 }  // namespace
@@ -221,8 +249,10 @@ qf_status qf_amax_tied(const qf_tensor* t, int n, float* d_group_amax, int n_gro
     cudaError_t e = cudaMemsetAsync(d_group_amax, 0, sizeof(float) * (size_t)n_groups, s);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
     if (v.empty()) return QF_OK;
-    qf_status st = launch_chunks(qf::k_amax<kAmaxU, kSmallT>, qf::k_amax<kAmaxU, kLargeT>, v,
-                                 256 * kAmaxU, d_group_amax, nullptr, d_tracked, n_groups, s);
+    qf_status st = launch_chunks(qf::k_amax<kAmaxU, kSmallT, QF_AMAX_THREADS>,
+                                 qf::k_amax<kAmaxU, kLargeT, QF_AMAX_THREADS>, QF_AMAX_THREADS,
+                                 QF_AMAX_WAVES, v, 256 * kAmaxU, d_group_amax, nullptr, d_tracked,
+                                 n_groups, s);
     if (st != QF_OK || !ragged) return st;
     // scalar tails of tensors whose size is not a multiple of 8 elements
     for (size_t b = 0; b < v.size(); b += kSmallT) {
@@ -263,7 +293,7 @@ qf_status qf_ste_backward(qf_format f, const void* grad_y, void* grad_x, int64_t
     if (mode == 0) {
         if (numel == 0 || grad_x == grad_y) return QF_OK;
         Launch L;
-        qf_status st = launch_shape(qf::k_copy, &L);
+        qf_status st = launch_shape(qf::k_copy, kThreads, 1, &L);
         if (st != QF_OK) return st;
         const int64_t vec = (numel + 7) / 8;
         const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(
@@ -295,18 +325,7 @@ qf_status qf_ste_backward(qf_format f, const void* grad_y, void* grad_x, int64_t
     v[0].numel = numel;
     v[0].group = nv ? fwd->group : 0;
     const float* am = nv ? d_group_amax : nullptr;
-    switch (f) {
-        case QF_NVFP4:
-            return launch_chunks(qf::k_fp4<true, kFp4U, kSmallT, 1>, qf::k_fp4<true, kFp4U, kLargeT, 1>,
-                                 v, 256 * kFp4U, am, nullptr, nullptr, n_groups, s);
-        case QF_MXFP4:
-            return launch_chunks(qf::k_fp4<false, kFp4U, kSmallT, 1>,
-                                 qf::k_fp4<false, kFp4U, kLargeT, 1>, v, 256 * kFp4U, nullptr,
-                                 nullptr, nullptr, 0, s);
-        default:
-            return launch_chunks(qf::k_q4k<kSmallT, 1>, qf::k_q4k<kLargeT, 1>, v,
-                                 1024, nullptr, nullptr, nullptr, 0, s);
-    }
+    return launch_format(f, 1, v, am, nullptr, n_groups, s);
 }
 
 const char* qf_status_string(qf_status s) {

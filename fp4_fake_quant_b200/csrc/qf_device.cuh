@@ -24,9 +24,55 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+// Build-time launch-shape knobs, per kernel (the defaults are the shipped configuration,
+// chosen by measurement on B200).  *_WAVES is the grid size in units of "one CTA per
+// resident slot": 1 is a persistent grid, a large value one CTA per chunk of work.
+#ifndef QF_MX_THREADS
+#define QF_MX_THREADS 256
+#endif
+#ifndef QF_MX_WAVES
+#define QF_MX_WAVES 1000
+#endif
+#ifndef QF_MX_PREFETCH
+#define QF_MX_PREFETCH 0
+#endif
+#ifndef QF_NV_THREADS
+#define QF_NV_THREADS 256
+#endif
+#ifndef QF_NV_WAVES
+#define QF_NV_WAVES 4
+#endif
+#ifndef QF_NV_PREFETCH
+#define QF_NV_PREFETCH 1
+#endif
+#ifndef QF_FP4_U
+#define QF_FP4_U 4              // 256-element sub-tiles per FP4 warp unit
+#endif
+#ifndef QF_FP4_LD
+#define QF_FP4_LD 1             // load policy, see ld_stream
+#endif
+#ifndef QF_Q4K_THREADS
+#define QF_Q4K_THREADS 512
+#endif
+#ifndef QF_Q4K_WAVES
+#define QF_Q4K_WAVES 1
+#endif
+#ifndef QF_AMAX_THREADS
+#define QF_AMAX_THREADS 256
+#endif
+#ifndef QF_AMAX_WAVES
+#define QF_AMAX_WAVES 1
+#endif
+#ifndef QF_AMAX_LD
+#define QF_AMAX_LD 0
+#endif
+#ifndef QF_ST_POLICY
+#define QF_ST_POLICY 0          // 0: default write-back stores, 1: streaming (.cs) stores
+#endif
+
 namespace qf {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 256;          // CTA size of the small helper kernels
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
 // One tensor of a launch.
@@ -96,14 +142,30 @@ __device__ __forceinline__ float f16_hi(uint32_t h2) {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// 16-byte streaming load (read-only path, no L1 allocation, 256-byte L2 prefetch).
+// 16-byte streaming load on the read-only path.  LD = 0: no L1 allocation and a
+// 256-byte L2 prefetch; 1: plain non-coherent load; 2: no L1 allocation.
+template <int LD = 0>
 __device__ __forceinline__ uint4 ld_stream(const uint16_t* p) {
     uint4 v;
-    asm("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
-        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    if (LD == 0)
+        asm("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
+            : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    else if (LD == 1)
+        asm("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+            : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    else
+        asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+            : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
     return v;
 }
-__device__ __forceinline__ void st_v4(void* p, uint4 v) { *reinterpret_cast<uint4*>(p) = v; }
+__device__ __forceinline__ void st_v4(void* p, uint4 v) {
+#if QF_ST_POLICY == 1
+    asm volatile("st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
+                 "r"(v.w) : "memory");
+#else
+    *reinterpret_cast<uint4*>(p) = v;
+#endif
+}
 
 // bf16x2 helpers on raw bits
 __device__ __forceinline__ uint32_t bmax2(uint32_t a, uint32_t b) {
@@ -123,8 +185,21 @@ __device__ __forceinline__ uint32_t abs_max8(uint4 v) {
     return max(m & 0xFFFFu, m >> 16);
 }
 
-// Walk the descriptor table forward to the tensor that owns unit u (units are
-// visited in increasing order by each warp, so this is amortised O(1)).
+// The tensor that owns unit u, by binary search over the units' first indices
+// (for a warp's first unit).
+template <int MAXT>
+__device__ __forceinline__ int locate_tensor(const Table<MAXT>& P, int64_t u) {
+    int lo = 0, hi = P.n - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (P.t[mid].unit_begin <= u) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
+// Walk the descriptor table forward to the tensor that owns unit u (a warp visits
+// its units in increasing order, so after locate_tensor this is amortised O(1)).
 template <int MAXT>
 __device__ __forceinline__ int find_tensor(const Table<MAXT>& P, int ti, int64_t u) {
     while (u >= P.t[ti].unit_end) ++ti;
@@ -210,12 +285,13 @@ struct UnitLoad {
 template <int U, int MODE>
 __device__ __forceinline__ void load_unit(const DevTensor& T, int64_t e0, int lane,
                                           UnitLoad<U, MODE>& L) {
+    constexpr int LD = QF_FP4_LD;
 #pragma unroll
     for (int s = 0; s < U; ++s) {
         const int64_t e = e0 + s * 256 + lane * 8;
         const bool ok = e < T.numel;
-        L.v[s] = ok ? ld_stream(T.x + e) : make_uint4(0, 0, 0, 0);
-        if (MODE == 1) L.gv[s] = ok ? ld_stream(T.g + e) : make_uint4(0, 0, 0, 0);
+        L.v[s] = ok ? ld_stream<LD>(T.x + e) : make_uint4(0, 0, 0, 0);
+        if (MODE == 1) L.gv[s] = ok ? ld_stream<LD>(T.g + e) : make_uint4(0, 0, 0, 0);
     }
 }
 
@@ -223,19 +299,19 @@ __device__ __forceinline__ void load_unit(const DevTensor& T, int64_t e0, int la
 // A unit is U sub-tiles of 256 elements.  The loads of a warp's next unit are
 // issued before the current one is computed, so every warp keeps a unit of
 // reads in flight while it converts.
-template <bool NV, int U, int MAXT, int MODE>
-__global__ void __launch_bounds__(kThreads) k_fp4(const __grid_constant__ Table<MAXT> P) {
+template <bool NV, int U, int MAXT, int MODE, int THREADS, int PREFETCH>
+__global__ void __launch_bounds__(THREADS) k_fp4(const __grid_constant__ Table<MAXT> P) {
     const int lane = threadIdx.x & 31;
-    const int64_t warp = (int64_t(blockIdx.x) * kThreads + threadIdx.x) >> 5;
-    const int64_t nwarps = (int64_t(gridDim.x) * kThreads) >> 5;
+    const int64_t warp = (int64_t(blockIdx.x) * THREADS + threadIdx.x) >> 5;
+    const int64_t nwarps = (int64_t(gridDim.x) * THREADS) >> 5;
     constexpr int kUnit = 256 * U;
     if (NV && MODE == 0 && blockIdx.x == 0 && P.group_scale_out) {
-        for (int g = threadIdx.x; g < P.n_groups; g += kThreads)
+        for (int g = threadIdx.x; g < P.n_groups; g += THREADS)
             P.group_scale_out[g] = nv_tensor_scale(P.group_amax[g]);
     }
     int64_t u = warp;
     if (u >= P.total_units) return;
-    int ti = find_tensor(P, 0, u);
+    int ti = locate_tensor(P, u);
     UnitLoad<U, MODE> cur;
     load_unit<U, MODE>(P.t[ti], (u - P.t[ti].unit_begin) * kUnit, lane, cur);
     int cur_t = -1;
@@ -245,7 +321,7 @@ __global__ void __launch_bounds__(kThreads) k_fp4(const __grid_constant__ Table<
         const int64_t un = u + nwarps;
         int tn = ti;
         UnitLoad<U, MODE> nxt;
-        if (un < P.total_units) {
+        if (PREFETCH && un < P.total_units) {
             tn = find_tensor(P, ti, un);
             load_unit<U, MODE>(P.t[tn], (un - P.t[tn].unit_begin) * kUnit, lane, nxt);
         }
@@ -287,8 +363,13 @@ __global__ void __launch_bounds__(kThreads) k_fp4(const __grid_constant__ Table<
         }
         if (un >= P.total_units) break;
         u = un;
-        ti = tn;
-        cur = nxt;
+        if (PREFETCH) {
+            ti = tn;
+            cur = nxt;
+        } else {
+            ti = find_tensor(P, ti, u);
+            load_unit<U, MODE>(P.t[ti], (u - P.t[ti].unit_begin) * kUnit, lane, cur);
+        }
     }
 }
 
@@ -348,17 +429,17 @@ __device__ __forceinline__ Q4kFit q4k_fit(const uint32_t (&w)[16]) {
 }
 
 // MODE 0: dequant (y) and/or 144-byte blocks (codes).  MODE 1: clipped STE, y = grad_x.
-template <int MAXT, int MODE>
-__global__ void __launch_bounds__(kThreads) k_q4k(const __grid_constant__ Table<MAXT> P) {
-    __shared__ __align__(16) uint8_t stage[kThreads / 32][kQ4kWarpBytes];
+template <int MAXT, int MODE, int THREADS>
+__global__ void __launch_bounds__(THREADS) k_q4k(const __grid_constant__ Table<MAXT> P) {
+    __shared__ __align__(16) uint8_t stage[THREADS / 32][kQ4kWarpBytes];
     const int lane = threadIdx.x & 31;
     const int b = lane & 3, j = lane >> 2;              // super-block of 4, sub-block of 8
     const uint32_t sm = (uint32_t)__cvta_generic_to_shared(stage[threadIdx.x >> 5]);
     const uint32_t sm_lane = sm + 16u * lane;           // coalesced view: row k at + k*528
     const uint32_t sm_mine = sm + b * kQ4kRow + 64u * j; // this lane's 64-byte sub-block
-    const int64_t warp = (int64_t(blockIdx.x) * kThreads + threadIdx.x) >> 5;
-    const int64_t nwarps = (int64_t(gridDim.x) * kThreads) >> 5;
-    int ti = 0;
+    const int64_t warp = (int64_t(blockIdx.x) * THREADS + threadIdx.x) >> 5;
+    const int64_t nwarps = (int64_t(gridDim.x) * THREADS) >> 5;
+    int ti = warp < P.total_units ? locate_tensor(P, warp) : 0;
     for (int64_t u = warp; u < P.total_units; u += nwarps) {
         ti = find_tensor(P, ti, u);
         const DevTensor& T = P.t[ti];
@@ -368,7 +449,7 @@ __global__ void __launch_bounds__(kThreads) k_q4k(const __grid_constant__ Table<
         uint4 v[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-            v[k] = k < nsb ? ld_stream(T.x + e0 + 256 * k + 8 * lane) : make_uint4(0, 0, 0, 0);
+            v[k] = k < nsb ? ld_stream<0>(T.x + e0 + 256 * k + 8 * lane) : make_uint4(0, 0, 0, 0);
         __syncwarp();
 #pragma unroll
         for (int k = 0; k < 4; ++k) sts128(sm_lane + k * kQ4kRow, v[k]);
@@ -454,7 +535,7 @@ __global__ void __launch_bounds__(kThreads) k_q4k(const __grid_constant__ Table<
             }
 #pragma unroll
             for (int k = 0; k < 4; ++k)
-                v[k] = k < nsb ? ld_stream(T.g + e0 + 256 * k + 8 * lane) : make_uint4(0, 0, 0, 0);
+                v[k] = k < nsb ? ld_stream<0>(T.g + e0 + 256 * k + 8 * lane) : make_uint4(0, 0, 0, 0);
             __syncwarp();
 #pragma unroll
             for (int k = 0; k < 4; ++k) sts128(sm_lane + k * kQ4kRow, v[k]);
@@ -483,18 +564,20 @@ __global__ void __launch_bounds__(kThreads) k_q4k(const __grid_constant__ Table<
 // Running max|x| per lane while the warp stays in one tie group; on a group
 // change (and at the end) the warp reduces and lane 0 does one atomicMax on the
 // group's FP32 bits (non-negative floats order like their bit patterns).
-template <int U, int MAXT>
-__global__ void __launch_bounds__(kThreads) k_amax(const __grid_constant__ Table<MAXT> P) {
+template <int U, int MAXT, int THREADS>
+__global__ void __launch_bounds__(THREADS) k_amax(const __grid_constant__ Table<MAXT> P) {
     const int lane = threadIdx.x & 31;
     constexpr int kUnit = 256 * U;
-    constexpr int kWarps = kThreads / 32;
+    constexpr int kWarps = THREADS / 32;
     // each CTA reduces one contiguous range of units, so a warp stays inside one
     // tensor (one tie group) for many units and flushes its max rarely
     const int64_t per_cta = (P.total_units + gridDim.x - 1) / gridDim.x;
     const int64_t u_begin = int64_t(blockIdx.x) * per_cta;
     const int64_t u_end = min(u_begin + per_cta, P.total_units);
     float* amax = const_cast<float*>(P.group_amax);
-    int ti = 0, g = -1;
+    const int64_t u_first = u_begin + (threadIdx.x >> 5);
+    int ti = u_first < u_end ? locate_tensor(P, u_first) : 0;
+    int g = -1;
     uint32_t run = 0;          // bf16x2 running max of |x|
     auto flush = [&](int grp) {
         uint32_t a = max(run & 0xFFFFu, run >> 16);
@@ -506,7 +589,7 @@ __global__ void __launch_bounds__(kThreads) k_amax(const __grid_constant__ Table
         }
         run = 0;
     };
-    for (int64_t u = u_begin + (threadIdx.x >> 5); u < u_end; u += kWarps) {
+    for (int64_t u = u_first; u < u_end; u += kWarps) {
         ti = find_tensor(P, ti, u);
         const DevTensor& T = P.t[ti];
         if (T.group != g) {
@@ -518,7 +601,7 @@ __global__ void __launch_bounds__(kThreads) k_amax(const __grid_constant__ Table
 #pragma unroll
         for (int s = 0; s < U; ++s) {
             const int64_t e = e0 + s * 256 + lane * 8;
-            v[s] = (e + 8 <= T.numel) ? ld_stream(T.x + e) : make_uint4(0, 0, 0, 0);
+            v[s] = (e + 8 <= T.numel) ? ld_stream<QF_AMAX_LD>(T.x + e) : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
         for (int s = 0; s < U; ++s) {
@@ -552,14 +635,14 @@ __global__ void __launch_bounds__(kThreads) k_copy(const uint16_t* __restrict__ 
     const int64_t stride = int64_t(gridDim.x) * kThreads;
     int64_t i = int64_t(blockIdx.x) * kThreads + threadIdx.x;
     for (; i + 3 * stride < nvec; i += 4 * stride) {
-        uint4 a = ld_stream(src + 8 * i), b = ld_stream(src + 8 * (i + stride));
-        uint4 c = ld_stream(src + 8 * (i + 2 * stride)), d = ld_stream(src + 8 * (i + 3 * stride));
+        uint4 a = ld_stream<1>(src + 8 * i), b = ld_stream<1>(src + 8 * (i + stride));
+        uint4 c = ld_stream<1>(src + 8 * (i + 2 * stride)), d = ld_stream<1>(src + 8 * (i + 3 * stride));
         st_v4(dst + 8 * i, a);
         st_v4(dst + 8 * (i + stride), b);
         st_v4(dst + 8 * (i + 2 * stride), c);
         st_v4(dst + 8 * (i + 3 * stride), d);
     }
-    for (; i < nvec; i += stride) st_v4(dst + 8 * i, ld_stream(src + 8 * i));
+    for (; i < nvec; i += stride) st_v4(dst + 8 * i, ld_stream<1>(src + 8 * i));
     if (blockIdx.x == 0 && threadIdx.x < (n & 7)) {
         const int64_t e = (nvec << 3) + threadIdx.x;
         dst[e] = src[e];

@@ -212,3 +212,19 @@ def test_mx_exponent_matches_frexp_for_every_bf16():
     for e in (-127, -3, 0, 5, 125):
         byte = np.uint8(e + 127)
         assert float(np.array([byte]).view(ml_dtypes.float8_e8m0fnu).astype(np.float64)[0]) == 2.0 ** e
+
+
+def test_conversions_are_monotone_in_magnitude():
+    """Every oracle conversion is a non-decreasing step function of the binary32 bit
+    pattern within one sign (round-to-nearest is monotone); the exhaustive GPU check
+    of the hardware conversions relies on this."""
+    rng = np.random.default_rng(8)
+    pats = np.unique(np.concatenate([
+        rng.integers(0, 0x7F7FFFFF, 1_000_000, dtype=np.uint64).astype(np.uint32),
+        np.arange(0x3E000000, 0x3E000000 + 200_000, dtype=np.uint32)]))
+    for sign in (0, 0x80000000):
+        x = (pats | np.uint32(sign)).view(np.float32)
+        for conv, mask in ((oracle.e2m1_from_f32, 0x7), (oracle.e4m3_from_f32, 0x7F),
+                           (oracle.f32_to_bf16, 0x7FFF), (oracle.f32_to_f16, 0x7FFF)):
+            m = (conv(x).astype(np.int64)) & mask
+            assert np.all(np.diff(m) >= 0)
