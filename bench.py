@@ -206,7 +206,7 @@ def make_workload(name: str, qf, dev, seed_shift: int = 0):
         W["fq"] = qf.prepare_fakequant(fmt, xs, Y, C, S, groups, amax, so)
         W["step_bytes"] = W["fq_bytes"] + 2 * numel
         W["launches"] = 2 * chunks
-        W["kernel"] = "k_fp4_nvfp4"
+        W["kernel"] = "k_nv"
     else:
         W["pre"] = None
         W["fq"] = qf.prepare_fakequant(fmt, xs, Y, C, S)

@@ -146,6 +146,10 @@ template <int MAXT, int MODE>
 constexpr auto nv_kernel() {
     return qf::k_fp4<true, kFp4U, MAXT, MODE, QF_NV_THREADS, QF_NV_PREFETCH>;
 }
+template <int MAXT>
+constexpr auto nv_block_kernel() {
+    return qf::k_nv<QF_NVB_U, MAXT, QF_NVB_THREADS, QF_NVB_PREFETCH>;
+}
 template <int MAXT, int MODE>
 constexpr auto mx_kernel() {
     return qf::k_fp4<false, kFp4U, MAXT, MODE, QF_MX_THREADS, QF_MX_PREFETCH>;
@@ -159,8 +163,9 @@ qf_status launch_format(qf_format f, int mode, const std::vector<DevTensor>& v, 
                         float* so, int ng, cudaStream_t s) {
     if (f == QF_NVFP4) {
         if (mode == 0)
-            return launch_chunks(nv_kernel<kSmallT, 0>(), nv_kernel<kLargeT, 0>(), QF_NV_THREADS,
-                                 QF_NV_WAVES, v, 256 * kFp4U, am, so, nullptr, ng, s);
+            return launch_chunks(nv_block_kernel<kSmallT>(), nv_block_kernel<kLargeT>(),
+                                 QF_NVB_THREADS, QF_NVB_WAVES, v, 512 * QF_NVB_U, am, so, nullptr,
+                                 ng, s);
         return launch_chunks(nv_kernel<kSmallT, 1>(), nv_kernel<kLargeT, 1>(), QF_NV_THREADS,
                              QF_NV_WAVES, v, 256 * kFp4U, am, nullptr, nullptr, ng, s);
     }

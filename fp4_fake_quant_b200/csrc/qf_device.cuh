@@ -45,6 +45,18 @@
 #ifndef QF_NV_PREFETCH
 #define QF_NV_PREFETCH 1
 #endif
+#ifndef QF_NVB_THREADS
+#define QF_NVB_THREADS 256      // NVFP4 fused pass, one lane per block
+#endif
+#ifndef QF_NVB_WAVES
+#define QF_NVB_WAVES 1000
+#endif
+#ifndef QF_NVB_PREFETCH
+#define QF_NVB_PREFETCH 0
+#endif
+#ifndef QF_NVB_U
+#define QF_NVB_U 4              // 512-element sub-tiles per warp unit
+#endif
 #ifndef QF_FP4_U
 #define QF_FP4_U 4              // 256-element sub-tiles per FP4 warp unit
 #endif
@@ -373,6 +385,122 @@ __global__ void __launch_bounds__(THREADS) k_fp4(const __grid_constant__ Table<M
     }
 }
 
+// ------------------------------------------------------------------ NVFP4, lane per block
+// NVFP4 fake-quant + pack with one lane per 16-element block: a warp sub-tile is 32
+// consecutive blocks (512 elements, 1 KB of BF16) and lane l owns block l, so the
+// E4M3 block scale (one IEEE divide, one reciprocal) is computed once per block and
+// the block max needs no shuffle.  A lane reads its block's 32 bytes with two 16-byte
+// loads (together they cover whole sectors; the second is served from L1) and writes
+// 32 bytes of BF16, 8 bytes of codes and 1 scale byte: the warp's code and scale
+// stores are contiguous 256- and 32-byte runs.
+template <int U, int MAXT, int THREADS, int PREFETCH>
+__global__ void __launch_bounds__(THREADS) k_nv(const __grid_constant__ Table<MAXT> P) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = (int64_t(blockIdx.x) * THREADS + threadIdx.x) >> 5;
+    const int64_t nwarps = (int64_t(gridDim.x) * THREADS) >> 5;
+    constexpr int kUnit = 512 * U;
+    if (blockIdx.x == 0 && P.group_scale_out) {
+        for (int g = threadIdx.x; g < P.n_groups; g += THREADS)
+            P.group_scale_out[g] = nv_tensor_scale(P.group_amax[g]);
+    }
+    int64_t u = warp;
+    if (u >= P.total_units) return;
+    int ti = locate_tensor(P, u);
+    uint4 cur[2 * U], nxt[2 * U];
+    auto load = [&](const DevTensor& T, int64_t e0, uint4 (&v)[2 * U]) {
+#pragma unroll
+        for (int s = 0; s < U; ++s) {
+            const int64_t e = e0 + s * 512 + lane * 16;
+            const bool ok = e < T.numel;
+            v[2 * s] = ok ? ld_stream<QF_FP4_LD>(T.x + e) : make_uint4(0, 0, 0, 0);
+            v[2 * s + 1] = ok ? ld_stream<QF_FP4_LD>(T.x + e + 8) : make_uint4(0, 0, 0, 0);
+        }
+    };
+    load(P.t[ti], (u - P.t[ti].unit_begin) * kUnit, cur);
+    int cur_t = -1;
+    float s_t = 0.0f, six_st = 0.0f;
+    while (true) {
+        const int64_t un = u + nwarps;
+        int tn = ti;
+        if (PREFETCH && un < P.total_units) {
+            tn = find_tensor(P, ti, un);
+            load(P.t[tn], (un - P.t[tn].unit_begin) * kUnit, nxt);
+        }
+        const DevTensor& T = P.t[ti];
+        if (ti != cur_t) {
+            s_t = nv_tensor_scale(P.group_amax[T.group]);
+            six_st = __fmul_rn(6.0f, s_t);
+            cur_t = ti;
+        }
+        const int64_t e0 = (u - T.unit_begin) * kUnit;
+#pragma unroll
+        for (int s = 0; s < U; ++s) {
+            const int64_t e = e0 + s * 512 + lane * 16;
+            const uint32_t w[8] = {cur[2 * s].x, cur[2 * s].y, cur[2 * s].z, cur[2 * s].w,
+                                   cur[2 * s + 1].x, cur[2 * s + 1].y, cur[2 * s + 1].z,
+                                   cur[2 * s + 1].w};
+            uint32_t m = bmax2(bmax2(bmax2(w[0] & 0x7FFF7FFFu, w[1] & 0x7FFF7FFFu),
+                                     bmax2(w[2] & 0x7FFF7FFFu, w[3] & 0x7FFF7FFFu)),
+                               bmax2(bmax2(w[4] & 0x7FFF7FFFu, w[5] & 0x7FFF7FFFu),
+                                     bmax2(w[6] & 0x7FFF7FFFu, w[7] & 0x7FFF7FFFu)));
+            const uint32_t a = max(m & 0xFFFFu, m >> 16);
+            uint32_t sb = 0;
+            float S = 0.0f, inv = 0.0f;
+            if (s_t != 0.0f) {
+                const float ratio = __fdiv_rn(__uint_as_float(a << 16), six_st);
+                sb = cvt_e4m3x2(0.0f, ratio) & 0xFFu;
+                S = __fmul_rn(f16_lo(cvt_e4m3x2_f16x2(sb)), s_t);
+                inv = (S == 0.0f) ? 0.0f : __frcp_rn(S);
+            }
+            float q[16];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                q[2 * k] = __fmul_rn(bf16_lo(w[k]), inv);
+                q[2 * k + 1] = __fmul_rn(bf16_hi(w[k]), inv);
+            }
+            if (__builtin_expect(isinf(inv), 0)) {
+                // 1/S overflowed (S < 2^-128): a zero keeps its own sign instead of 0 * inf
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    if (bf16_lo(w[k]) == 0.0f) q[2 * k] = bf16_lo(w[k]);
+                    if (bf16_hi(w[k]) == 0.0f) q[2 * k + 1] = bf16_hi(w[k]);
+                }
+            }
+            uint32_t b[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) b[k] = cvt_e2m1x2(q[2 * k + 1], q[2 * k]);
+            if (e < T.numel) {
+                if (T.y) {
+                    uint32_t yw[8];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const uint32_t h2 = cvt_e2m1x2_f16x2(b[k]);
+                        yw[k] = cvt_bf16x2(__fmul_rn(f16_hi(h2), S), __fmul_rn(f16_lo(h2), S));
+                    }
+                    st_v4(T.y + e, make_uint4(yw[0], yw[1], yw[2], yw[3]));
+                    st_v4(T.y + e + 8, make_uint4(yw[4], yw[5], yw[6], yw[7]));
+                }
+                if (T.codes) {
+                    const uint32_t lo = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
+                    const uint32_t hi = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
+                    *reinterpret_cast<uint2*>(T.codes + (e >> 1)) = make_uint2(lo, hi);
+                }
+                if (T.scales) T.scales[e >> 4] = (uint8_t)sb;
+            }
+        }
+        if (un >= P.total_units) break;
+        u = un;
+        if (PREFETCH) {
+            ti = tn;
+#pragma unroll
+            for (int i = 0; i < 2 * U; ++i) cur[i] = nxt[i];
+        } else {
+            ti = find_tensor(P, ti, u);
+            load(P.t[ti], (u - P.t[ti].unit_begin) * kUnit, cur);
+        }
+    }
+}
+
 // ------------------------------------------------------------------ Q4_K
 // One lane per 32-element sub-block: a warp iteration covers 4 super-blocks (1024
 // elements) and lane l owns sub-block j = l / 4 of super-block b = l % 4, so the
@@ -479,8 +607,11 @@ __global__ void __launch_bounds__(THREADS) k_q4k(const __grid_constant__ Table<M
                 if (k & 1) qw[k >> 1] = __byte_perm(qw[k >> 1], __byte_perm(__float_as_uint(r[0]),
                                                     __float_as_uint(r[1]), 0x0040), 0x5410);
                 else qw[k >> 1] = __byte_perm(__float_as_uint(r[0]), __float_as_uint(r[1]), 0x0040);
-                yw[k] = cvt_bf16x2(__fsub_rn(__fmul_rn(f.s, __fsub_rn(r[1], kRound)), f.mm),
-                                   __fsub_rn(__fmul_rn(f.s, __fsub_rn(r[0], kRound)), f.mm));
+                // y = RN(s*q - mm): s = d*sc has at most 17 significant bits and q at most 4,
+                // so s*q is exact and one fused multiply-add rounds exactly once, as the
+                // separate multiply and subtract do
+                yw[k] = cvt_bf16x2(__fmaf_rn(f.s, __fsub_rn(r[1], kRound), -f.mm),
+                                   __fmaf_rn(f.s, __fsub_rn(r[0], kRound), -f.mm));
             }
             if (T.y) {
                 // stage y back through this lane's own 64 bytes, then store coalesced
