@@ -5,10 +5,11 @@
  * The library implements the hot path of quantization-aware training as
  * described on the QATFactory project page ("QATFactory: A Versatile,
  * Deployment-Aligned Framework for Quantization-aware Training and Distillation
- * of LLMs"): weights, and optionally activations, are rounded onto a deployment
- * format's grid in the forward pass (quantize-dequantize), a straight-through
- * estimator carries the gradient to the latent weight in the backward pass, and
- * the codes and scales are packed in the inference engine's layout.
+ * of LLMs"): in the forward pass every weight (and, if wanted, activation)
+ * becomes the nearest value a deployment format can hold (quantize, then
+ * dequantize); in the backward pass the gradient passes straight through to the
+ * full-precision weight; and the codes and scales are written in the byte
+ * layout the inference engine loads.
  *
  * Formats ("Supported formats" table of the project page):
  *   NVFP4  E2M1 elements, 16-element blocks, E4M3 block scale, FP32 tensor scale,
@@ -106,9 +107,10 @@ typedef struct qf_tensor {
 } qf_tensor;
 
 /*
- * qf_amax_tied -- tied NVFP4 tensor amax (project page, Method, "Numerics": the
- * projections that vLLM and SGLang fuse share one tensor scale; "Export": NVFP4
- * activation scales are tracked during training and saved).
+ * qf_amax_tied -- tied NVFP4 tensor amax (project page, Method, "Numerics": a
+ * projection group that vLLM or SGLang runs as one fused GEMM uses a common
+ * tensor scale; "Export": the NVFP4 activation amax is kept from training, so
+ * serving needs no calibration).
  *
  *   d_group_amax[g] = max over the tensors i with t[i].group == g of max |x_i|
  *                     (FP32, exact); 0 for a group with no tensor.  Overwritten.
@@ -128,8 +130,8 @@ qf_status qf_amax_tied(const qf_tensor* t, int n, float* d_group_amax, int n_gro
 /*
  * qf_fakequant -- the fused forward pass: block statistics, block-scale encode,
  * element encode, dequantize and pack in one read of x (project page, Method,
- * "Framework overview": a lossy quantize-dequantize that reproduces inference
- * numerics; "QARL"/"Export": packing in the engine's layout).  n == 1 is one
+ * "Framework overview": quantize then dequantize so training sees serving's
+ * numbers; "QARL"/"Export": the engine's byte layout).  n == 1 is one
  * tensor; n > 1 is one grouped launch over all n tensors (e.g. every expert of
  * an MoE layer), bitwise identical to n single calls.
  *
@@ -162,8 +164,8 @@ qf_status qf_fakequant(qf_format f, const qf_tensor* t, int n, const float* d_gr
 
 /*
  * qf_pack -- the engine-layout export and weight sync (project page, Method,
- * "QARL": after each step the learner packs its weights in the engine's layout
- * and syncs them; "Export").  Identical to qf_fakequant except that y is never
+ * "QARL": after every optimizer step the trainer writes its weights in the
+ * engine's byte layout and hands them over; "Export").  Identical to qf_fakequant except that y is never
  * written (it may be non-NULL and is ignored); each tensor needs codes or scales.
  * The bytes written are those qf_fakequant writes.
  */
@@ -172,7 +174,8 @@ qf_status qf_pack(qf_format f, const qf_tensor* t, int n, const float* d_group_a
 
 /*
  * qf_ste_backward -- straight-through estimator backward (project page, Method,
- * "Framework overview": the STE updates the continuous latent weights; Bengio,
+ * "Framework overview": the gradient reaches the full-precision weights
+ * unchanged by the rounding; Bengio,
  * Leonard and Courville 2013, cited by the paper).
  *   mode 0 (identity):  grad_x = grad_y, numel BF16 elements.  grad_x == grad_y
  *                       is allowed and launches nothing.  f, fwd and

@@ -9,22 +9,23 @@
  * Source of the method: "QATFactory: A Versatile, Deployment-Aligned Framework
  * for Quantization-aware Training and Distillation of LLMs", project page
  * (weilixu.com/QATFactory-web):
- *   [M-QDQ]   Method, "Framework overview": the forward pass applies a lossy
- *             quantize-dequantize that reproduces inference numerics; the backward
- *             pass is a straight-through estimator onto the latent weights.
- *   [M-NUM]   Method, "Numerics -- deployment-aligned simulated quantization":
- *             the engine is the numerical specification (values, block sizes,
- *             scaling rules); under NVFP4 the projections an engine fuses (QKV,
- *             gate/up) share one tensor scale; MXFP4 and Q4_K have no tensor scale.
+ *   [M-QDQ]   Method, "Framework overview": training quantizes and at once
+ *             dequantizes in the forward pass, so the model computes with the
+ *             numbers inference will use; gradients pass straight through to the
+ *             full-precision weights (a straight-through estimator).
+ *   [M-NUM]   Method, "Numerics": the serving engine defines the values, block
+ *             sizes and scaling rules; for NVFP4, projections the engine runs as
+ *             one fused GEMM (QKV, gate/up) use a common tensor scale, while
+ *             MXFP4 and Q4_K have no tensor-level scale at all.
  *   [T-FMT]   "Supported formats" table: NVFP4 = E2M1 elements, block 16, E4M3
  *             block scale + FP32 tensor scale, symmetric, 4.50 bits/weight;
  *             MXFP4 = E2M1, block 32, E8M0 block scale, symmetric, 4.25 b/w;
  *             Q4_K = unsigned INT4, block 32 in a 256 super-block, 6-bit block
- *             scales + FP16 super-block scales, asymmetric, 4.50 b/w.  Bits per
- *             weight include element codes and scale metadata.
- *   [M-EXP]   Method, "QARL" and "Export": weights are packed in the engine's
- *             layout; NVFP4 activation scales are tracked during training.
- *   [M-QAD]   Method, "QAD": MoE experts are quantized one at a time.
+ *             scales + FP16 super-block scales, asymmetric, 4.50 b/w.  The
+ *             bits-per-weight figures count the codes plus the scale bytes.
+ *   [M-EXP]   Method, "QARL" and "Export": weights are written in the byte layout
+ *             the engine loads; the NVFP4 activation amax is kept from training.
+ *   [M-QAD]   Method, "QAD": MoE experts are quantized in separate passes.
  *
  * Arithmetic: the pages fix FP32 as the tensor-scale type [T-FMT]; every scale
  * and element step below is IEEE binary32 with round-to-nearest-even and no

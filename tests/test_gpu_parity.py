@@ -110,7 +110,7 @@ def test_moe_grouped_equals_looped_and_oracle(fmt):
     am = oracle.tied_amax(ts, groups, ng) if fmt == "nvfp4" else None
     if fmt == "nvfp4":
         assert_same("moe amax", grouped["amax"].view(np.uint32), am.view(np.uint32))
-    # one expert at a time: each call sees only that expert's tensors
+    # each expert in its own call: the call sees only that expert's tensors
     for e in range(12):
         idx = [3 * e, 3 * e + 1, 3 * e + 2]
         sub = [ts[i] for i in idx]

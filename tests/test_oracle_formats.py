@@ -70,7 +70,7 @@ def test_bits_per_weight_and_block_sizes_match_format_table():
 
 # ----------------------------------------------------------------------------- tied scale
 def test_tied_tensor_scale_is_amax_of_concatenation():
-    """NVFP4: fused projections (QKV, gate/up) share one tensor scale (Method, Numerics)."""
+    """NVFP4: projections an engine fuses (QKV, gate/up) use a common tensor scale (Method, Numerics)."""
     wl = workloads.nvfp4_tied(rows_scale=1 / 64, with_grads=False)
     am = oracle.tied_amax(wl["tensors"], wl["groups"], wl["n_groups"])
     for g in range(2):
