@@ -79,6 +79,13 @@ def _load():
             "qfo_e4m3_from_f32": (ctypes.c_uint8, [F]),
             "qfo_mx_exponent": (ctypes.c_int, [F]),
             "qfo_amax_bf16": (F, [P, I64]),
+            "qfo_amax_x": (F, [P, ctypes.c_int, I64]),
+            "qfo_nvfp4_quant_x": (None, [P, ctypes.c_int, I64, I64, F, P, P, P, P]),
+            "qfo_mxfp4_quant_x": (None, [P, ctypes.c_int, I64, I64, P, P, P]),
+            "qfo_q4k_quant_x": (None, [P, ctypes.c_int, I64, I64, P, P]),
+            "qfo_q4k_fit_one_x": (None, [P, ctypes.c_int, P, P, P, P, P]),
+            "qfo_ste_backward_x": (None, [P, P, I64, ctypes.c_int, ctypes.c_int, P, ctypes.c_int,
+                                          I64, F]),
             "qfo_nvfp4_tensor_scale": (F, [F]),
             "qfo_nvfp4_quant": (None, [P, I64, I64, F, P, P, P, P]),
             "qfo_mxfp4_quant": (None, [P, I64, I64, P, P, P]),
@@ -118,6 +125,20 @@ def _bits(x) -> np.ndarray:
     import torch  # the input generators hand out torch bf16 tensors
     assert x.dtype == torch.bfloat16 and x.device.type == "cpu"
     return x.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def _xin(x):
+    """An input tensor and its element type: BF16 (numpy uint16 bits or torch bf16) -> 0,
+    FP32 (numpy float32 or torch float32) -> 1."""
+    if isinstance(x, np.ndarray):
+        if x.dtype == np.float32:
+            return np.ascontiguousarray(x), 1
+        return _bits(x), 0
+    import torch
+    if x.dtype == torch.float32:
+        assert x.device.type == "cpu"
+        return x.contiguous().numpy(), 1
+    return _bits(x), 0
 
 
 # ---------------------------------------------------------------- conversions
@@ -184,9 +205,9 @@ def change_points(which: str, lo: int, hi: int, cap: int = 1 << 18):
 
 # ---------------------------------------------------------------- the method
 def amax(x) -> float:
-    """max |x| of one BF16 tensor (FP32)."""
-    xb = _bits(x)
-    return float(_load().qfo_amax_bf16(_ptr(xb), xb.size))
+    """max |x| of one BF16 or FP32 tensor (FP32)."""
+    xb, xt = _xin(x)
+    return float(_load().qfo_amax_x(_ptr(xb), xt, xb.size))
 
 
 def tied_amax(tensors, groups, n_groups: int, tracked=None) -> np.ndarray:
@@ -206,7 +227,7 @@ def nvfp4_tensor_scale(amax_g: float) -> float:
 
 def nvfp4(x, amax_g: float, rows: int | None = None, cols: int | None = None):
     """NVFP4 quantize-dequantize + pack.  Returns (y_bits, codes, scales, s_t)."""
-    xb = _bits(x)
+    xb, xt = _xin(x)
     if rows is None:
         rows, cols = xb.shape
     n = rows * cols
@@ -214,47 +235,48 @@ def nvfp4(x, amax_g: float, rows: int | None = None, cols: int | None = None):
     codes = np.empty(n // 2, np.uint8)
     scales = np.empty(n // 16, np.uint8)
     st = ctypes.c_float()
-    _load().qfo_nvfp4_quant(_ptr(xb), rows, cols, float(amax_g), _ptr(y), _ptr(codes),
-                            _ptr(scales), ctypes.byref(st))
+    _load().qfo_nvfp4_quant_x(_ptr(xb), xt, rows, cols, float(amax_g), _ptr(y), _ptr(codes),
+                              _ptr(scales), ctypes.byref(st))
     return y, codes, scales, float(st.value)
 
 
 def mxfp4(x, rows: int | None = None, cols: int | None = None):
     """MXFP4 quantize-dequantize + pack.  Returns (y_bits, codes, scales)."""
-    xb = _bits(x)
+    xb, xt = _xin(x)
     if rows is None:
         rows, cols = xb.shape
     n = rows * cols
     y = np.empty(n, np.uint16)
     codes = np.empty(n // 2, np.uint8)
     scales = np.empty(n // 32, np.uint8)
-    _load().qfo_mxfp4_quant(_ptr(xb), rows, cols, _ptr(y), _ptr(codes), _ptr(scales))
+    _load().qfo_mxfp4_quant_x(_ptr(xb), xt, rows, cols, _ptr(y), _ptr(codes), _ptr(scales))
     return y, codes, scales
 
 
 def q4k(x, rows: int | None = None, cols: int | None = None):
     """Q4_K quantize-dequantize + pack.  Returns (y_bits, blocks[n/256, 144])."""
-    xb = _bits(x)
+    xb, xt = _xin(x)
     if rows is None:
         rows, cols = xb.shape
     n = rows * cols
     y = np.empty(n, np.uint16)
     blocks = np.empty((n // 256) * 144, np.uint8)
-    _load().qfo_q4k_quant(_ptr(xb), rows, cols, _ptr(y), _ptr(blocks))
+    _load().qfo_q4k_quant_x(_ptr(xb), xt, rows, cols, _ptr(y), _ptr(blocks))
     return y, blocks
 
 
 def q4k_fit_one(x256: np.ndarray):
     """Unpacked fit of one super-block: (d_bits, dmin_bits, sc[8], m[8], q[256])."""
-    xb = _bits(x256).reshape(-1)
+    xb, xt = _xin(x256)
+    xb = xb.reshape(-1)
     assert xb.size == 256
     d = ctypes.c_uint16()
     dm = ctypes.c_uint16()
     sc = np.empty(8, np.uint8)
     m = np.empty(8, np.uint8)
     q = np.empty(256, np.uint8)
-    _load().qfo_q4k_fit_one(_ptr(xb), ctypes.byref(d), ctypes.byref(dm), _ptr(sc), _ptr(m),
-                            _ptr(q))
+    _load().qfo_q4k_fit_one_x(_ptr(xb), xt, ctypes.byref(d), ctypes.byref(dm), _ptr(sc), _ptr(m),
+                              _ptr(q))
     return int(d.value), int(dm.value), sc, m, q
 
 
@@ -288,8 +310,8 @@ def ste_backward(grad_y, mode: int = 0, fmt: str = "nvfp4", x=None, amax_g: floa
     if mode == 0:
         _load().qfo_ste_backward(_ptr(gy), _ptr(gx), gy.size, 0, 0, None, 0, 0.0)
         return gx
-    xb = _bits(x)
+    xb, xt = _xin(x)
     cols = xb.shape[-1]
-    _load().qfo_ste_backward(_ptr(gy), _ptr(gx), gy.size, 1, FORMATS[fmt], _ptr(xb), cols,
-                             float(amax_g))
+    _load().qfo_ste_backward_x(_ptr(gy), _ptr(gx), gy.size, 1, FORMATS[fmt], _ptr(xb), xt, cols,
+                               float(amax_g))
     return gx

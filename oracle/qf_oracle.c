@@ -211,19 +211,40 @@ int qfo_mx_exponent(float amax)
 }
 
 /* ------------------------------------------------------------------------ */
+/* Input element types: BF16 weights/activations, or FP32 latent (master)    */
+/* weights (the memory table of the project page lists the student's         */
+/* trainable weights as FP32).  Every step below works on the element value.  */
+/* ------------------------------------------------------------------------ */
+enum { QFO_BF16 = 0, QFO_F32 = 1 };
+
+static float xval(const void* x, int xt, int64_t i)
+{
+    if (xt == QFO_F32) return ((const float*)x)[i];
+    return qfo_bf16_to_f32(((const uint16_t*)x)[i]);
+}
+
+static const void* xoff(const void* x, int xt, int64_t i)
+{
+    return xt == QFO_F32 ? (const void*)((const float*)x + i)
+                         : (const void*)((const uint16_t*)x + i);
+}
+
+/* ------------------------------------------------------------------------ */
 /* Tensor absolute maximum (exact: max is independent of order).             */
 /* [M-NUM]: the NVFP4 tensor scale of a tie group is taken from the amax of  */
 /* every tensor in the group; [M-EXP]: activation amax is tracked.           */
 /* ------------------------------------------------------------------------ */
-float qfo_amax_bf16(const uint16_t* x, int64_t n)
+float qfo_amax_x(const void* x, int xt, int64_t n)
 {
     float m = 0.0f;
     for (int64_t i = 0; i < n; ++i) {
-        float a = fabsf(qfo_bf16_to_f32(x[i]));
+        float a = fabsf(xval(x, xt, i));
         if (a > m) m = a;
     }
     return m;
 }
+
+float qfo_amax_bf16(const uint16_t* x, int64_t n) { return qfo_amax_x(x, QFO_BF16, n); }
 
 /* ------------------------------------------------------------------------ */
 /* NVFP4 block scale derivation, one 16-element block.                       */
@@ -263,20 +284,20 @@ float qfo_nvfp4_tensor_scale(float amax_g) { return amax_g / 2688.0f; }
 /*   s_t    the FP32 tensor scale                                            */
 /* [T-FMT] NVFP4 row; [M-NUM] tied tensor scale; [M-QDQ] quantize-dequantize.*/
 /* ------------------------------------------------------------------------ */
-void qfo_nvfp4_quant(const uint16_t* x, int64_t rows, int64_t cols, float amax_g,
-                     uint16_t* y, uint8_t* codes, uint8_t* scales, float* s_t_out)
+void qfo_nvfp4_quant_x(const void* x, int xt, int64_t rows, int64_t cols, float amax_g,
+                       uint16_t* y, uint8_t* codes, uint8_t* scales, float* s_t_out)
 {
     float s_t = qfo_nvfp4_tensor_scale(amax_g);
     if (s_t_out) *s_t_out = s_t;
     for (int64_t r = 0; r < rows; ++r) {
         for (int64_t b = 0; b < cols / 16; ++b) {
             const int64_t base = r * cols + b * 16;
-            float amax_b = qfo_amax_bf16(x + base, 16);
+            float amax_b = qfo_amax_x(xoff(x, xt, base), xt, 16);
             uint8_t sb; float S, inv;
             nvfp4_block_scale(amax_b, s_t, &sb, &S, &inv);
             if (scales) scales[base / 16] = sb;
             for (int i = 0; i < 16; ++i) {
-                float xv = qfo_bf16_to_f32(x[base + i]);
+                float xv = xval(x, xt, base + i);
                 uint8_t c = qfo_e2m1_from_f32(scaled(xv, inv));
                 if (y) y[base + i] = qfo_f32_to_bf16(qfo_e2m1_to_f32(c) * S);
                 if (codes) {
@@ -296,19 +317,19 @@ void qfo_nvfp4_quant(const uint16_t* x, int64_t rows, int64_t cols, float amax_g
 /*   y    = BF16(f32(code) * 2^e)        (exact)                             */
 /* Layout as NVFP4 with one E8M0 byte per 32 elements.  [T-FMT] MXFP4 row.   */
 /* ------------------------------------------------------------------------ */
-void qfo_mxfp4_quant(const uint16_t* x, int64_t rows, int64_t cols,
-                     uint16_t* y, uint8_t* codes, uint8_t* scales)
+void qfo_mxfp4_quant_x(const void* x, int xt, int64_t rows, int64_t cols,
+                       uint16_t* y, uint8_t* codes, uint8_t* scales)
 {
     for (int64_t r = 0; r < rows; ++r) {
         for (int64_t b = 0; b < cols / 32; ++b) {
             const int64_t base = r * cols + b * 32;
-            float amax_b = qfo_amax_bf16(x + base, 32);
+            float amax_b = qfo_amax_x(xoff(x, xt, base), xt, 32);
             int e = qfo_mx_exponent(amax_b);
             if (scales) scales[base / 32] = (uint8_t)(e + 127);
             float inv = ldexpf(1.0f, -e);
             float S = ldexpf(1.0f, e);
             for (int i = 0; i < 32; ++i) {
-                float xv = qfo_bf16_to_f32(x[base + i]);
+                float xv = xval(x, xt, base + i);
                 uint8_t c = qfo_e2m1_from_f32(xv * inv);
                 if (y) y[base + i] = qfo_f32_to_bf16(qfo_e2m1_to_f32(c) * S);
                 if (codes) {
@@ -346,13 +367,13 @@ typedef struct {
     uint8_t q[256];              /* 4-bit values */
 } q4k_super;
 
-static void q4k_fit(const uint16_t* x, q4k_super* o, uint16_t* y)
+static void q4k_fit(const void* x, int xt, q4k_super* o, uint16_t* y)
 {
     float scale[8], minv[8];
     for (int j = 0; j < 8; ++j) {
-        float mn = qfo_bf16_to_f32(x[32 * j]), hi = mn;
+        float mn = xval(x, xt, 32 * j), hi = mn;
         for (int i = 1; i < 32; ++i) {
-            float v = qfo_bf16_to_f32(x[32 * j + i]);
+            float v = xval(x, xt, 32 * j + i);
             if (v < mn) mn = v;
             if (v > hi) hi = v;
         }
@@ -376,7 +397,7 @@ static void q4k_fit(const uint16_t* x, q4k_super* o, uint16_t* y)
         float mm = dmin * (float)o->m[j];
         float inv = (s == 0.0f) ? 0.0f : 1.0f / s;
         for (int i = 0; i < 32; ++i) {
-            float v = (qfo_bf16_to_f32(x[32 * j + i]) + mm) * inv;
+            float v = (xval(x, xt, 32 * j + i) + mm) * inv;
             float q = nearbyintf(v);
             if (q < 0.0f) q = 0.0f;
             if (q > 15.0f) q = 15.0f;
@@ -425,25 +446,25 @@ static void q4k_pack(const q4k_super* o, uint8_t* blk)
 
 /* Q4_K quantize-dequantize + pack of one [rows, cols] matrix, cols % 256 == 0.
  * y: [rows*cols] BF16 (may be NULL); blocks: [rows*cols/256] x 144 bytes (may be NULL). */
-void qfo_q4k_quant(const uint16_t* x, int64_t rows, int64_t cols,
-                   uint16_t* y, uint8_t* blocks)
+void qfo_q4k_quant_x(const void* x, int xt, int64_t rows, int64_t cols,
+                     uint16_t* y, uint8_t* blocks)
 {
     q4k_super o;
     for (int64_t r = 0; r < rows; ++r) {
         for (int64_t b = 0; b < cols / 256; ++b) {
             const int64_t base = r * cols + b * 256;
-            q4k_fit(x + base, &o, y ? y + base : NULL);
+            q4k_fit(xoff(x, xt, base), xt, &o, y ? y + base : NULL);
             if (blocks) q4k_pack(&o, blocks + (base / 256) * 144);
         }
     }
 }
 
 /* Q4_K scale/min fit of one 256-element super-block, unpacked (for pins). */
-void qfo_q4k_fit_one(const uint16_t* x, uint16_t* d, uint16_t* dmin, uint8_t* sc,
-                     uint8_t* m, uint8_t* q)
+void qfo_q4k_fit_one_x(const void* x, int xt, uint16_t* d, uint16_t* dmin, uint8_t* sc,
+                       uint8_t* m, uint8_t* q)
 {
     q4k_super o;
-    q4k_fit(x, &o, NULL);
+    q4k_fit(x, xt, &o, NULL);
     *d = o.d; *dmin = o.dmin;
     memcpy(sc, o.sc, 8); memcpy(m, o.m, 8); memcpy(q, o.q, 256);
 }
@@ -511,8 +532,8 @@ void qfo_q4k_decode(const uint8_t* blocks, int64_t numel, uint16_t* y)
 /*   Q4_K: 0 <= (x + mm_j) * inv_j <= 15.                                    */
 /* fmt: 0 NVFP4, 1 MXFP4, 2 Q4_K.  amax_g is the NVFP4 tie-group amax.       */
 /* ------------------------------------------------------------------------ */
-void qfo_ste_backward(const uint16_t* grad_y, uint16_t* grad_x, int64_t numel, int mode,
-                      int fmt, const uint16_t* x, int64_t cols, float amax_g)
+void qfo_ste_backward_x(const uint16_t* grad_y, uint16_t* grad_x, int64_t numel, int mode,
+                        int fmt, const void* x, int xt, int64_t cols, float amax_g)
 {
     if (mode == 0) { for (int64_t i = 0; i < numel; ++i) grad_x[i] = grad_y[i]; return; }
     int64_t rows = cols ? numel / cols : 0;
@@ -520,37 +541,53 @@ void qfo_ste_backward(const uint16_t* grad_y, uint16_t* grad_x, int64_t numel, i
         float s_t = qfo_nvfp4_tensor_scale(amax_g);
         for (int64_t base = 0; base < rows * cols; base += 16) {
             uint8_t sb; float S, inv;
-            nvfp4_block_scale(qfo_amax_bf16(x + base, 16), s_t, &sb, &S, &inv);
+            nvfp4_block_scale(qfo_amax_x(xoff(x, xt, base), xt, 16), s_t, &sb, &S, &inv);
             for (int i = 0; i < 16; ++i) {
-                float q = scaled(qfo_bf16_to_f32(x[base + i]), inv);
+                float q = scaled(xval(x, xt, base + i), inv);
                 grad_x[base + i] = (fabsf(q) <= 6.0f) ? grad_y[base + i] : 0;
             }
         }
     } else if (fmt == 1) {
         for (int64_t base = 0; base < rows * cols; base += 32) {
-            float inv = ldexpf(1.0f, -qfo_mx_exponent(qfo_amax_bf16(x + base, 32)));
+            float inv = ldexpf(1.0f, -qfo_mx_exponent(qfo_amax_x(xoff(x, xt, base), xt, 32)));
             for (int i = 0; i < 32; ++i) {
-                float q = qfo_bf16_to_f32(x[base + i]) * inv;
+                float q = xval(x, xt, base + i) * inv;
                 grad_x[base + i] = (fabsf(q) <= 6.0f) ? grad_y[base + i] : 0;
             }
         }
     } else {
         q4k_super o;
         for (int64_t base = 0; base < rows * cols; base += 256) {
-            q4k_fit(x + base, &o, NULL);
+            q4k_fit(xoff(x, xt, base), xt, &o, NULL);
             float d = qfo_f16_to_f32(o.d), dmin = qfo_f16_to_f32(o.dmin);
             for (int j = 0; j < 8; ++j) {
                 float s = d * (float)o.sc[j], mm = dmin * (float)o.m[j];
                 float inv = (s == 0.0f) ? 0.0f : 1.0f / s;
                 for (int i = 0; i < 32; ++i) {
                     int64_t k = base + 32 * j + i;
-                    float v = (qfo_bf16_to_f32(x[k]) + mm) * inv;
+                    float v = (xval(x, xt, k) + mm) * inv;
                     grad_x[k] = (v >= 0.0f && v <= 15.0f) ? grad_y[k] : 0;
                 }
             }
         }
     }
 }
+
+/* BF16-input entry points (the common case). */
+void qfo_nvfp4_quant(const uint16_t* x, int64_t rows, int64_t cols, float amax_g,
+                     uint16_t* y, uint8_t* codes, uint8_t* scales, float* s_t_out)
+{ qfo_nvfp4_quant_x(x, QFO_BF16, rows, cols, amax_g, y, codes, scales, s_t_out); }
+void qfo_mxfp4_quant(const uint16_t* x, int64_t rows, int64_t cols,
+                     uint16_t* y, uint8_t* codes, uint8_t* scales)
+{ qfo_mxfp4_quant_x(x, QFO_BF16, rows, cols, y, codes, scales); }
+void qfo_q4k_quant(const uint16_t* x, int64_t rows, int64_t cols, uint16_t* y, uint8_t* blocks)
+{ qfo_q4k_quant_x(x, QFO_BF16, rows, cols, y, blocks); }
+void qfo_q4k_fit_one(const uint16_t* x, uint16_t* d, uint16_t* dmin, uint8_t* sc, uint8_t* m,
+                     uint8_t* q)
+{ qfo_q4k_fit_one_x(x, QFO_BF16, d, dmin, sc, m, q); }
+void qfo_ste_backward(const uint16_t* grad_y, uint16_t* grad_x, int64_t numel, int mode,
+                      int fmt, const uint16_t* x, int64_t cols, float amax_g)
+{ qfo_ste_backward_x(grad_y, grad_x, numel, mode, fmt, x, QFO_BF16, cols, amax_g); }
 
 /* ------------------------------------------------------------------------ */
 /* Array forms of the conversions, for exhaustive checks in the tests.       */

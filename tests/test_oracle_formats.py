@@ -466,3 +466,68 @@ def test_q4k_negative_values_rounding_to_code_zero_dequantize_to_positive_zero()
     assert m[0] == 0 and q[5] == 0
     y, _ = oracle.q4k(xb.reshape(1, 256))
     assert y[5] == 0x0000
+
+
+# ----------------------------------------------------------------------------- FP32 latent input
+def test_f32_input_equal_to_bf16_path_when_representable():
+    """FP32 master weights that happen to be BF16 values quantize exactly like the BF16 tensor."""
+    x = rand_bf16(16, 512, 31)
+    xf = x.float()
+    am = oracle.amax(x)
+    assert oracle.amax(xf) == am
+    for a, b in zip(oracle.nvfp4(x, am), oracle.nvfp4(xf, am)):
+        assert np.array_equal(a, b)
+    for a, b in zip(oracle.mxfp4(x), oracle.mxfp4(xf)):
+        assert np.array_equal(a, b)
+    for a, b in zip(oracle.q4k(x), oracle.q4k(xf)):
+        assert np.array_equal(a, b)
+
+
+def test_f32_nvfp4_on_grid_codes_round_trip():
+    """x = code * sb * s_t with an 18-bit s_t: exact in FP32 but not in BF16; the fit
+    recovers every code and block scale, and y = BF16(x)."""
+    rng = np.random.default_rng(41)
+    rows, cols = 8, 256
+    nb = rows * cols // 16
+    st = np.float32((1.0 + rng.integers(1, 1 << 17) / 2.0 ** 17) * 2.0 ** -10)
+    sb = rng.integers(0x08, 0x7F, size=nb).astype(np.uint8)
+    sb[3] = 0x7E
+    sbv = sb.view(ml_dtypes.float8_e4m3fn).astype(np.float64)
+    codes = rng.integers(0, 16, size=(nb, 16)).astype(np.uint8)
+    codes[np.arange(nb), rng.integers(0, 16, nb)] = 7
+    x64 = e2m1_val(codes) * sbv[:, None] * float(st)
+    x = x64.astype(np.float32)
+    assert np.array_equal(x.astype(np.float64), x64)                # exact in FP32
+    x = x.reshape(rows, cols)
+    am = oracle.amax(x)
+    y, c, s, st_out = oracle.nvfp4(x, am)
+    assert st_out == st
+    assert np.array_equal(s, sb) and np.array_equal(unpack_nibbles(c), codes.reshape(-1))
+    assert np.array_equal(y, oracle.f32_to_bf16(x.reshape(-1)))
+
+
+def test_f32_codes_brute_force_and_decoder():
+    rng = np.random.default_rng(43)
+    x = (rng.standard_normal((8, 512)) * 0.02).astype(np.float32)
+    x[2, 5] = 0.7                                                    # an outlier
+    xf = x.reshape(-1)
+    am = oracle.amax(x)
+    # NVFP4: nearest E2M1 of x * (1/S) with S from the block scale, ties to even
+    y, c, s, st = oracle.nvfp4(x, am)
+    S = (s.view(ml_dtypes.float8_e4m3fn).astype(np.float32) * np.float32(st)).astype(np.float32)
+    inv = np.where(S == 0, np.float32(0), np.float32(1) / S).astype(np.float32)
+    q = (xf.reshape(-1, 16) * inv[:, None]).astype(np.float32).reshape(-1)
+    lib = q.astype(ml_dtypes.float4_e2m1fn).astype(np.float32)
+    assert np.array_equal(e2m1_val(unpack_nibbles(c)).astype(np.float32), np.abs(lib) *
+                          np.where(q.view(np.uint32) >> 31, -1, 1))
+    assert np.array_equal(oracle.nvfp4_decode(c, s, st, xf.size), y)
+    # MXFP4 and Q4_K: the independent decoder reproduces the dequantized output
+    y, c, s = oracle.mxfp4(x)
+    assert np.array_equal(oracle.mxfp4_decode(c, s, xf.size), y)
+    e = s.astype(np.int64) - 127
+    qm = (xf.reshape(-1, 32).astype(np.float64) * np.exp2(-e.astype(np.float64))[:, None])
+    assert np.array_equal(e2m1_val(unpack_nibbles(c)).astype(np.float64),
+                          qm.reshape(-1).astype(np.float32).astype(ml_dtypes.float4_e2m1fn)
+                          .astype(np.float64))
+    y, b = oracle.q4k(x)
+    assert np.array_equal(oracle.q4k_decode(b, xf.size), y)
