@@ -49,7 +49,7 @@ UNIT = "GB/s"
 BYTES_PER_ELEM = {"nvfp4": 2 + 2 + 0.5 + 1 / 16, "mxfp4": 2 + 2 + 0.5 + 1 / 32,
                   "q4k": 2 + 2 + 144 / 256}
 WORKLOADS = ("w4a4", "nvfp4_tied", "q4k", "nvfp4_weight", "activation", "moe_nvfp4",
-             "moe_mxfp4", "moe_q4k")
+             "moe_mxfp4", "moe_q4k", "nvfp4_tied_f32", "q4k_f32")
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -167,6 +167,14 @@ def make_workload(name: str, qf, dev, seed_shift: int = 0):
         wl, fmt = workloads.q4k_weights(seed=2 + seed_shift), "q4k"
         desc = ("Q4_K weight-only: down 4096x14336 + up 14336x4096, N(0,0.015) x per-row "
                 "log-uniform[0.5,2]; one grouped fake-quant+pack launch (144-byte blocks)")
+    elif name == "q4k_f32":
+        wl, fmt = workloads.q4k_weights(seed=2 + seed_shift, dtype="f32"), "q4k"
+        desc = ("Q4_K from FP32 latent weights: down 4096x14336 + up 14336x4096; one grouped "
+                "fake-quant+pack launch (FP32 in, BF16 + 144-byte blocks out)")
+    elif name == "nvfp4_tied_f32":
+        wl, fmt = workloads.nvfp4_tied(seed=3 + seed_shift, with_grads=False, dtype="f32"), "nvfp4"
+        desc = ("NVFP4 tied projections from FP32 latent weights (Q/K/V, gate/up); tied amax "
+                "pass + one grouped fake-quant+pack launch (FP32 in, BF16 + codes out)")
     elif name == "nvfp4_weight":
         wl, fmt = workloads.nvfp4_weight(seed=0 + seed_shift), "nvfp4"
         desc = "NVFP4 weight 4096x4096 N(0,0.02), 0.1% x20 outliers; amax pass + fake-quant+pack"
@@ -190,10 +198,11 @@ def make_workload(name: str, qf, dev, seed_shift: int = 0):
     outs = [qf.alloc_outputs(fmt, x) for x in xs]
     Y, C, S = [o[0] for o in outs], [o[1] for o in outs], [o[2] for o in outs]
     numel = sum(x.numel() for x in xs)
+    in_b = xs[0].element_size()                      # 2 (BF16) or 4 (FP32 latent weights)
     chunks = (len(xs) + 383) // 384                  # launches per call (descriptor tables)
     W = dict(name=name, fmt=fmt, desc=desc, xs=xs, xs_h=xs_h, outs=[t for t in Y + C + S if
-             t is not None], numel=numel, fq_bytes=numel * BYTES_PER_ELEM[fmt],
-             n_tensors=len(xs))
+             t is not None], numel=numel, fq_bytes=numel * (BYTES_PER_ELEM[fmt] + in_b - 2),
+             n_tensors=len(xs), in_bytes=in_b)
     if fmt == "nvfp4":
         amax = torch.zeros(ng, dtype=torch.float32, device=dev)
         cur = torch.zeros(ng, dtype=torch.float32, device=dev)
@@ -204,7 +213,7 @@ def make_workload(name: str, qf, dev, seed_shift: int = 0):
         else:
             W["pre"] = qf.prepare_amax_tied(xs, groups, amax)
         W["fq"] = qf.prepare_fakequant(fmt, xs, Y, C, S, groups, amax, so)
-        W["step_bytes"] = W["fq_bytes"] + 2 * numel
+        W["step_bytes"] = W["fq_bytes"] + in_b * numel
         W["launches"] = 2 * chunks
         W["kernel"] = "k_nv"
     else:
@@ -232,7 +241,7 @@ def run_ours(args, rank, world, local_rank):
 
     W = make_workload(args.workload, qf, dev, seed_shift=1000 * rank)
     numel, step_bytes = W["numel"], W["step_bytes"]
-    in_bytes = 2 * numel
+    in_bytes = W["in_bytes"] * numel
     flush_buf = torch.empty(2 * l2, dtype=torch.uint8, device=dev) if in_bytes < 2 * l2 else None
     torch.cuda.synchronize()
 
@@ -305,9 +314,10 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic (seeded stand-ins for real weights and activations)",
         "config": {"workload": W["desc"], "format": W["fmt"], "tensors": W["n_tensors"],
                    "elements_per_step": numel, "bytes_per_step": step_bytes,
-                   "l2": (f"L2 flushed before every step ({in_bytes / 1e6:.0f} MB of BF16 input "
+                   "input": "fp32" if W["in_bytes"] == 4 else "bf16",
+                   "l2": (f"L2 flushed before every step ({in_bytes / 1e6:.0f} MB of input "
                           f"< 2x the {l2 / 1e6:.0f} MB L2)") if flush_buf is not None else
-                         (f"inputs larger than L2 ({in_bytes / 1e6:.0f} MB of BF16 vs "
+                         (f"inputs larger than L2 ({in_bytes / 1e6:.0f} MB of input vs "
                           f"{l2 / 1e6:.0f} MB); no flush between steps"),
                    "parallelism": f"replicas x{world} (weak scaling, no collective)"},
         "gelem_per_s": world * numel / (ms_per_step * 1e-3) / 1e9,
@@ -353,13 +363,15 @@ def per_format(qf, dev, args, l2):
         it = args.pf_iters
         t_fq = timed_calls(W["fq"], it, 3, flush)
         gbs = W["fq_bytes"] / (t_fq * 1e-3) / 1e9
-        d = {"format": W["fmt"], "tensors": W["n_tensors"], "elements": W["numel"],
+        d = {"format": W["fmt"], "input": "fp32" if W["in_bytes"] == 4 else "bf16",
+             "tensors": W["n_tensors"], "elements": W["numel"],
              "fused_us": t_fq * 1e3, "fused_GB/s": gbs, "fused_Gelem/s": W["numel"] / t_fq / 1e6,
              "fused_frac_of_hbm_peak": gbs / peak}
         if W["pre"] is not None:
             t_pre = timed_calls(W["pre"], it, 3, flush)
             t_step = timed_calls(lambda: run_step(W), it, 3, flush)
-            d.update({"amax_us": t_pre * 1e3, "amax_GB/s": 2 * W["numel"] / t_pre / 1e6,
+            d.update({"amax_us": t_pre * 1e3,
+                      "amax_GB/s": W["in_bytes"] * W["numel"] / t_pre / 1e6,
                       "step_us": t_step * 1e3,
                       "step_GB/s": W["step_bytes"] / t_step / 1e6})
         if name.startswith("moe_"):

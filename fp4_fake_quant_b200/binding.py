@@ -18,6 +18,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libqf.so")
 
 QF_NVFP4, QF_MXFP4, QF_Q4K = 0, 1, 2
+QF_X_BF16, QF_X_F32 = 0, 1
 FORMATS = {"nvfp4": QF_NVFP4, "mxfp4": QF_MXFP4, "q4k": QF_Q4K}
 BLOCK = {QF_NVFP4: 16, QF_MXFP4: 32, QF_Q4K: 256}
 STATUS = {0: "QF_OK", 1: "QF_ERR_INVALID_ARG", 2: "QF_ERR_SHAPE", 3: "QF_ERR_ALIGN",
@@ -27,7 +28,7 @@ STATUS = {0: "QF_OK", 1: "QF_ERR_INVALID_ARG", 2: "QF_ERR_SHAPE", 3: "QF_ERR_ALI
 class QfTensor(ctypes.Structure):
     """Mirror of ``qf_tensor`` (include/qf.h)."""
     _fields_ = [("x", ctypes.c_void_p), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
-                ("group", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("group", ctypes.c_int32), ("x_type", ctypes.c_int32),
                 ("y", ctypes.c_void_p), ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
 
 
@@ -97,15 +98,19 @@ def _desc(xs: Sequence[torch.Tensor], ys=None, codes=None, scales=None, groups=N
     n = len(xs)
     arr = (QfTensor * max(n, 1))()
     for i, x in enumerate(xs):
-        if x.dtype != torch.bfloat16:
-            raise TypeError("x must be bfloat16")
+        if x.dtype == torch.bfloat16:
+            xt = QF_X_BF16
+        elif x.dtype == torch.float32:
+            xt = QF_X_F32
+        else:
+            raise TypeError("x must be bfloat16 or float32")
         rows, cols = (x.shape[0], x.shape[1]) if x.dim() == 2 else (1, x.numel()) if x.dim() == 1 \
             else (x.numel() // x.shape[-1], x.shape[-1])
         d = arr[i]
         d.x = _ptr(x)
         d.rows, d.cols = rows, cols
         d.group = int(groups[i]) if groups is not None else 0
-        d.reserved = 0
+        d.x_type = xt
         d.y = _ptr(ys[i]) if ys is not None and ys[i] is not None else None
         d.codes = _ptr(codes[i]) if codes is not None and codes[i] is not None else None
         d.scales = _ptr(scales[i]) if scales is not None and scales[i] is not None else None
@@ -123,7 +128,7 @@ def output_sizes(fmt, numel: int):
 def alloc_outputs(fmt, x: torch.Tensor, want_y: bool = True):
     """Allocate (y, codes, scales) for one input tensor (torch allocations; plumbing)."""
     ncodes, nscales = output_sizes(fmt, x.numel())
-    y = torch.empty_like(x) if want_y else None
+    y = torch.empty(x.shape, dtype=torch.bfloat16, device=x.device) if want_y else None
     codes = torch.empty(ncodes, dtype=torch.uint8, device=x.device)
     scales = torch.empty(nscales, dtype=torch.uint8, device=x.device) if nscales else None
     return y, codes, scales

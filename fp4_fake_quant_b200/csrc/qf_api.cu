@@ -132,7 +132,8 @@ qf_status check_tensor(const qf_tensor& t, int i, int need_cols_multiple, int n_
     if (need_cols_multiple && t.cols % need_cols_multiple != 0)
         return fail(QF_ERR_SHAPE, "tensor %d: cols=%lld is not a multiple of %d", i,
                     (long long)t.cols, need_cols_multiple);
-    if (t.reserved != 0) return fail(QF_ERR_INVALID_ARG, "tensor %d: reserved field not 0", i);
+    if (t.x_type != QF_X_BF16 && t.x_type != QF_X_F32)
+        return fail(QF_ERR_UNSUPPORTED, "tensor %d: unknown x_type %d", i, (int)t.x_type);
     const int64_t numel = t.rows * t.cols;
     if (numel > 0 && t.x == nullptr) return fail(QF_ERR_INVALID_ARG, "tensor %d: x is NULL", i);
     if (!aligned16(t.x)) return fail(QF_ERR_ALIGN, "tensor %d: x not 16-byte aligned", i);
@@ -141,46 +142,56 @@ qf_status check_tensor(const qf_tensor& t, int i, int need_cols_multiple, int n_
     return QF_OK;
 }
 
-// The kernels of each format with their launch shapes.
-template <int MAXT, int MODE>
+// The kernels of each format with their launch shapes (XT: input element type).
+template <typename XT, int MAXT, int MODE>
 constexpr auto nv_kernel() {
-    return qf::k_fp4<true, kFp4U, MAXT, MODE, QF_NV_THREADS, QF_NV_PREFETCH>;
+    return qf::k_fp4<true, XT, kFp4U, MAXT, MODE, QF_NV_THREADS, QF_NV_PREFETCH>;
 }
-template <int MAXT>
+// FP32 input holds twice the bytes per element in registers: half the sub-tiles per unit
+template <typename XT>
+constexpr int nvb_u() { return sizeof(XT) == 2 ? QF_NVB_U : (QF_NVB_U + 1) / 2; }
+template <typename XT, int MAXT>
 constexpr auto nv_block_kernel() {
-    return qf::k_nv<QF_NVB_U, MAXT, QF_NVB_THREADS, QF_NVB_PREFETCH>;
+    return qf::k_nv<XT, nvb_u<XT>(), MAXT, QF_NVB_THREADS, QF_NVB_PREFETCH>;
 }
-template <int MAXT, int MODE>
+template <typename XT, int MAXT, int MODE>
 constexpr auto mx_kernel() {
-    return qf::k_fp4<false, kFp4U, MAXT, MODE, QF_MX_THREADS, QF_MX_PREFETCH>;
+    return qf::k_fp4<false, XT, kFp4U, MAXT, MODE, QF_MX_THREADS, QF_MX_PREFETCH>;
 }
-template <int MAXT, int MODE>
+template <typename XT, int MAXT, int MODE>
 constexpr auto q4k_kernel() {
-    return qf::k_q4k<MAXT, MODE, QF_Q4K_THREADS>;
+    return qf::k_q4k<XT, MAXT, MODE, QF_Q4K_THREADS>;
 }
 
-qf_status launch_format(qf_format f, int mode, const std::vector<DevTensor>& v, const float* am,
-                        float* so, int ng, cudaStream_t s) {
+template <typename XT>
+qf_status launch_format_t(qf_format f, int mode, const std::vector<DevTensor>& v,
+                          const float* am, float* so, int ng, cudaStream_t s) {
     if (f == QF_NVFP4) {
         if (mode == 0)
-            return launch_chunks(nv_block_kernel<kSmallT>(), nv_block_kernel<kLargeT>(),
-                                 QF_NVB_THREADS, QF_NVB_WAVES, v, 512 * QF_NVB_U, am, so, nullptr,
+            return launch_chunks(nv_block_kernel<XT, kSmallT>(), nv_block_kernel<XT, kLargeT>(),
+                                 QF_NVB_THREADS, QF_NVB_WAVES, v, 512 * nvb_u<XT>(), am, so, nullptr,
                                  ng, s);
-        return launch_chunks(nv_kernel<kSmallT, 1>(), nv_kernel<kLargeT, 1>(), QF_NV_THREADS,
+        return launch_chunks(nv_kernel<XT, kSmallT, 1>(), nv_kernel<XT, kLargeT, 1>(), QF_NV_THREADS,
                              QF_NV_WAVES, v, 256 * kFp4U, am, nullptr, nullptr, ng, s);
     }
     if (f == QF_MXFP4) {
         if (mode == 0)
-            return launch_chunks(mx_kernel<kSmallT, 0>(), mx_kernel<kLargeT, 0>(), QF_MX_THREADS,
+            return launch_chunks(mx_kernel<XT, kSmallT, 0>(), mx_kernel<XT, kLargeT, 0>(), QF_MX_THREADS,
                                  QF_MX_WAVES, v, 256 * kFp4U, nullptr, nullptr, nullptr, 0, s);
-        return launch_chunks(mx_kernel<kSmallT, 1>(), mx_kernel<kLargeT, 1>(), QF_MX_THREADS,
+        return launch_chunks(mx_kernel<XT, kSmallT, 1>(), mx_kernel<XT, kLargeT, 1>(), QF_MX_THREADS,
                              QF_MX_WAVES, v, 256 * kFp4U, nullptr, nullptr, nullptr, 0, s);
     }
     if (mode == 0)
-        return launch_chunks(q4k_kernel<kSmallT, 0>(), q4k_kernel<kLargeT, 0>(), QF_Q4K_THREADS,
+        return launch_chunks(q4k_kernel<XT, kSmallT, 0>(), q4k_kernel<XT, kLargeT, 0>(), QF_Q4K_THREADS,
                              QF_Q4K_WAVES, v, 1024, nullptr, nullptr, nullptr, 0, s);
-    return launch_chunks(q4k_kernel<kSmallT, 1>(), q4k_kernel<kLargeT, 1>(), QF_Q4K_THREADS,
+    return launch_chunks(q4k_kernel<XT, kSmallT, 1>(), q4k_kernel<XT, kLargeT, 1>(), QF_Q4K_THREADS,
                          QF_Q4K_WAVES, v, 1024, nullptr, nullptr, nullptr, 0, s);
+}
+
+qf_status launch_format(qf_format f, int mode, int x_type, const std::vector<DevTensor>& v,
+                        const float* am, float* so, int ng, cudaStream_t s) {
+    if (x_type == QF_X_F32) return launch_format_t<float>(f, mode, v, am, so, ng, s);
+    return launch_format_t<uint16_t>(f, mode, v, am, so, ng, s);
 }
 
 qf_status fakequant_impl(qf_format f, const qf_tensor* t, int n, const float* d_group_amax,
@@ -209,7 +220,9 @@ qf_status fakequant_impl(qf_format f, const qf_tensor* t, int n, const float* d_
         if (!aligned16(y) || !aligned16(t[i].codes))
             return fail(QF_ERR_ALIGN, "tensor %d: y / codes not 16-byte aligned", i);
         DevTensor d{};
-        d.x = static_cast<const uint16_t*>(t[i].x);
+        if (t[i].x_type != t[0].x_type)
+            return fail(QF_ERR_INVALID_ARG, "tensor %d: x_type differs from tensor 0's", i);
+        d.x = t[i].x;
         d.y = static_cast<uint16_t*>(y);
         d.codes = static_cast<uint8_t*>(t[i].codes);
         d.scales = static_cast<uint8_t*>(scales);
@@ -222,7 +235,7 @@ qf_status fakequant_impl(qf_format f, const qf_tensor* t, int n, const float* d_
     const float* am = nv ? d_group_amax : nullptr;
     const int ng = nv ? n_groups : 0;
     if (v.empty() && !so) return QF_OK;
-    return launch_format(f, 0, v, am, so, ng, s);
+    return launch_format(f, 0, n > 0 ? t[0].x_type : QF_X_BF16, v, am, so, ng, s);
 }
 
 }  // namespace
@@ -241,10 +254,12 @@ qf_status qf_amax_tied(const qf_tensor* t, int n, float* d_group_amax, int n_gro
     for (int i = 0; i < n; ++i) {
         qf_status st = check_tensor(t[i], i, 0, n_groups, true);
         if (st != QF_OK) return st;
+        if (t[i].x_type != t[0].x_type)
+            return fail(QF_ERR_INVALID_ARG, "tensor %d: x_type differs from tensor 0's", i);
         const int64_t numel = t[i].rows * t[i].cols;
         if (numel == 0) continue;
         DevTensor d{};
-        d.x = static_cast<const uint16_t*>(t[i].x);
+        d.x = t[i].x;
         d.numel = numel;
         d.group = t[i].group;
         ragged |= (numel & 7) != 0;
@@ -254,10 +269,17 @@ qf_status qf_amax_tied(const qf_tensor* t, int n, float* d_group_amax, int n_gro
     cudaError_t e = cudaMemsetAsync(d_group_amax, 0, sizeof(float) * (size_t)n_groups, s);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
     if (v.empty()) return QF_OK;
-    qf_status st = launch_chunks(qf::k_amax<kAmaxU, kSmallT, QF_AMAX_THREADS>,
-                                 qf::k_amax<kAmaxU, kLargeT, QF_AMAX_THREADS>, QF_AMAX_THREADS,
-                                 QF_AMAX_WAVES, v, 256 * kAmaxU, d_group_amax, nullptr, d_tracked,
-                                 n_groups, s);
+    const bool f32 = t[0].x_type == QF_X_F32;
+    // the same bytes in flight per lane: 8 vectors of BF16, or 4 sub-tiles of FP32 (8 vectors)
+    qf_status st = f32
+        ? launch_chunks(qf::k_amax<float, kAmaxU / 2, kSmallT, QF_AMAX_THREADS>,
+                        qf::k_amax<float, kAmaxU / 2, kLargeT, QF_AMAX_THREADS>, QF_AMAX_THREADS,
+                        QF_AMAX_WAVES, v, 256 * (kAmaxU / 2), d_group_amax, nullptr, d_tracked,
+                        n_groups, s)
+        : launch_chunks(qf::k_amax<uint16_t, kAmaxU, kSmallT, QF_AMAX_THREADS>,
+                        qf::k_amax<uint16_t, kAmaxU, kLargeT, QF_AMAX_THREADS>, QF_AMAX_THREADS,
+                        QF_AMAX_WAVES, v, 256 * kAmaxU, d_group_amax, nullptr, d_tracked,
+                        n_groups, s);
     if (st != QF_OK || !ragged) return st;
     // scalar tails of tensors whose size is not a multiple of 8 elements
     for (size_t b = 0; b < v.size(); b += kSmallT) {
@@ -267,7 +289,8 @@ qf_status qf_amax_tied(const qf_tensor* t, int n, float* d_group_amax, int n_gro
         P.group_amax = d_group_amax;
         P.tracked = d_tracked;
         P.n_groups = n_groups;
-        qf::k_amax_tail<kSmallT><<<(unsigned)cnt, 32, 0, s>>>(P);
+        if (f32) qf::k_amax_tail<float, kSmallT><<<(unsigned)cnt, 32, 0, s>>>(P);
+        else qf::k_amax_tail<uint16_t, kSmallT><<<(unsigned)cnt, 32, 0, s>>>(P);
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
@@ -324,13 +347,13 @@ qf_status qf_ste_backward(qf_format f, const void* grad_y, void* grad_x, int64_t
     if (numel == 0) return QF_OK;
     std::vector<DevTensor> v(1);
     v[0] = DevTensor{};
-    v[0].x = static_cast<const uint16_t*>(fwd->x);
+    v[0].x = fwd->x;
     v[0].g = static_cast<const uint16_t*>(grad_y);
     v[0].y = static_cast<uint16_t*>(grad_x);
     v[0].numel = numel;
     v[0].group = nv ? fwd->group : 0;
     const float* am = nv ? d_group_amax : nullptr;
-    return launch_format(f, 1, v, am, nullptr, n_groups, s);
+    return launch_format(f, 1, fwd->x_type, v, am, nullptr, n_groups, s);
 }
 
 const char* qf_status_string(qf_status s) {
@@ -347,6 +370,6 @@ const char* qf_status_string(qf_status s) {
 
 const char* qf_last_error(void) { return g_err; }
 
-int qf_version(void) { return (1 << 16) | 0; }
+int qf_version(void) { return (1 << 16) | 1; }
 
 }  // extern "C"

@@ -6,18 +6,23 @@
 //   * A call covers n tensors.  Their descriptors travel in a __grid_constant__
 //     kernel parameter (no device allocation, no copy), each tensor split into
 //     fixed-size "units" of elements; a unit is the work of one warp iteration.
-//   * Persistent grid: (#SMs x resident CTAs) CTAs; warp w takes units w, w+W, ...
-//   * Lane l of a warp holds 8 consecutive BF16 (one 16-byte load) of each
-//     256-element sub-tile, so every load and every BF16 store is a fully
-//     coalesced 512-byte warp transaction.  Block statistics are reduced across
-//     the 2 (NVFP4), 4 (MXFP4) or 32 (Q4_K super-block) lanes that share a block
-//     with warp shuffles.
+//     A warp binary-searches the table for its first unit and walks forward.
+//   * Inputs are BF16 or FP32 (latent master weights): every kernel is a template
+//     on the element type XT and reads whole 16-byte vectors.
+//   * MXFP4 (k_fp4): lane l holds 8 consecutive elements of each 256-element
+//     sub-tile, so BF16 loads and stores are whole 512-byte warp transactions; the
+//     4 lanes of a 32-element block reduce its max with shuffles.
+//   * NVFP4 (k_nv): one lane per 16-element block, so the E4M3 block scale is
+//     computed once per block and needs no shuffle.
+//   * Q4_K (k_q4k): one lane per 32-element sub-block, four super-blocks per warp
+//     iteration, BF16 traffic staged through padded shared-memory rows.
 //   * Blackwell's native conversions do the format rounding:
 //     cvt.rn.satfinite.e2m1x2.f32, cvt.rn.satfinite.e4m3x2.f32, cvt.rn.bf16x2.f32
 //     and the reverse cvt.rn.f16x2.{e2m1x2,e4m3x2}.
 //   * Every scale step is one IEEE binary32 operation with round-to-nearest-even
 //     (__fdiv_rn, __frcp_rn, __fmul_rn, __fadd_rn); the library is built without
-//     FMA contraction so the rounding order is the one the header documents.
+//     FMA contraction so the rounding order is the one the header documents (the
+//     one explicit FMA, in the Q4_K dequant, is exact by construction).
 #pragma once
 
 #include <cstdint>
@@ -37,7 +42,7 @@
 #define QF_MX_PREFETCH 0
 #endif
 #ifndef QF_NV_THREADS
-#define QF_NV_THREADS 256
+#define QF_NV_THREADS 256       // NVFP4 clipped STE (k_fp4)
 #endif
 #ifndef QF_NV_WAVES
 #define QF_NV_WAVES 4
@@ -46,7 +51,7 @@
 #define QF_NV_PREFETCH 1
 #endif
 #ifndef QF_NVB_THREADS
-#define QF_NVB_THREADS 256      // NVFP4 fused pass, one lane per block
+#define QF_NVB_THREADS 256      // NVFP4 fused pass, one lane per block (k_nv)
 #endif
 #ifndef QF_NVB_WAVES
 #define QF_NVB_WAVES 1000
@@ -58,7 +63,7 @@
 #define QF_NVB_U 4              // 512-element sub-tiles per warp unit
 #endif
 #ifndef QF_FP4_U
-#define QF_FP4_U 4              // 256-element sub-tiles per FP4 warp unit
+#define QF_FP4_U 4              // 256-element sub-tiles per k_fp4 warp unit
 #endif
 #ifndef QF_FP4_LD
 #define QF_FP4_LD 1             // load policy, see ld_stream
@@ -89,7 +94,7 @@ constexpr unsigned kFull = 0xFFFFFFFFu;
 
 // One tensor of a launch.
 struct DevTensor {
-    const uint16_t* x;      // BF16 input
+    const void* x;          // input: BF16 or FP32 (the launch's element type)
     uint16_t* y;            // BF16 dequant out / STE grad_x (nullable)
     uint8_t* codes;         // packed nibbles / Q4_K blocks (nullable)
     uint8_t* scales;        // E4M3 / E8M0 bytes (nullable)
@@ -157,7 +162,7 @@ __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w 
 // 16-byte streaming load on the read-only path.  LD = 0: no L1 allocation and a
 // 256-byte L2 prefetch; 1: plain non-coherent load; 2: no L1 allocation.
 template <int LD = 0>
-__device__ __forceinline__ uint4 ld_stream(const uint16_t* p) {
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
     uint4 v;
     if (LD == 0)
         asm("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -190,12 +195,63 @@ __device__ __forceinline__ uint32_t bmin2(uint32_t a, uint32_t b) {
                                *reinterpret_cast<__nv_bfloat162*>(&b));
     return *reinterpret_cast<uint32_t*>(&r);
 }
-// max |x| over the lane's 8 BF16 values, as non-negative BF16 bits
-__device__ __forceinline__ uint32_t abs_max8(uint4 v) {
-    uint32_t m = bmax2(bmax2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
-                       bmax2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
-    return max(m & 0xFFFFu, m >> 16);
-}
+
+// ------------------------------------------------------------------ element chunks
+// N consecutive input elements of type XT (uint16_t = BF16 bits, float = FP32) held
+// in registers as whole 16-byte vectors.
+template <typename XT, int N>
+struct Elems {
+    static constexpr bool kBf16 = sizeof(XT) == 2;
+    static constexpr int kVec = N * (int)sizeof(XT) / 16;
+    uint4 v[kVec];
+
+    __device__ __forceinline__ uint32_t word(int i) const {
+        const uint4& q = v[i >> 2];
+        const int k = i & 3;
+        return k == 0 ? q.x : k == 1 ? q.y : k == 2 ? q.z : q.w;
+    }
+    // element k as FP32 (exact)
+    __device__ __forceinline__ float get(int k) const {
+        if constexpr (kBf16) return (k & 1) ? bf16_hi(word(k >> 1)) : bf16_lo(word(k >> 1));
+        else return __uint_as_float(word(k));
+    }
+    // FP32 bit pattern of max |x| (non-negative floats order like their bit patterns)
+    __device__ __forceinline__ uint32_t amax_bits() const {
+        if constexpr (kBf16) {
+            uint32_t m = word(0) & 0x7FFF7FFFu;
+#pragma unroll
+            for (int i = 1; i < 4 * kVec; ++i) m = bmax2(m, word(i) & 0x7FFF7FFFu);
+            return max(m & 0xFFFFu, m >> 16) << 16;
+        } else {
+            uint32_t m = word(0) & 0x7FFFFFFFu;
+#pragma unroll
+            for (int i = 1; i < 4 * kVec; ++i) m = max(m, word(i) & 0x7FFFFFFFu);
+            return m;
+        }
+    }
+    // min and max of the elements
+    __device__ __forceinline__ void minmax(float& lo, float& hi) const {
+        if constexpr (kBf16) {
+            uint32_t mx = word(0), mn = word(0);
+#pragma unroll
+            for (int i = 1; i < 4 * kVec; ++i) { mx = bmax2(mx, word(i)); mn = bmin2(mn, word(i)); }
+            hi = fmaxf(bf16_lo(mx), bf16_hi(mx));
+            lo = fminf(bf16_lo(mn), bf16_hi(mn));
+        } else {
+            hi = get(0);
+            lo = hi;
+#pragma unroll
+            for (int k = 1; k < N; ++k) { hi = fmaxf(hi, get(k)); lo = fminf(lo, get(k)); }
+        }
+    }
+    template <int LD>
+    __device__ __forceinline__ void load(const XT* p, bool ok) {
+#pragma unroll
+        for (int i = 0; i < kVec; ++i)
+            v[i] = ok ? ld_stream<LD>(reinterpret_cast<const uint8_t*>(p) + 16 * i)
+                      : make_uint4(0, 0, 0, 0);
+    }
+};
 
 // The tensor that owns unit u, by binary search over the units' first indices
 // (for a warp's first unit).
@@ -221,7 +277,22 @@ __device__ __forceinline__ int find_tensor(const Table<MAXT>& P, int ti, int64_t
 // NVFP4 tensor scale of a tie group: s_t = amax_g / (6 * 448).
 __device__ __forceinline__ float nv_tensor_scale(float amax_g) { return __fdiv_rn(amax_g, 2688.0f); }
 
-// ------------------------------------------------------------------ NVFP4 / MXFP4
+// NVFP4 block scale from the block amax: sb = E4M3(amax_b / (6 s_t)), S = f32(sb) s_t,
+// inv = 1/S (0 when S == 0; sb = 0 when s_t == 0).
+__device__ __forceinline__ void nv_block_scale(float amax_b, float s_t, float six_st,
+                                               uint32_t& sb, float& S, float& inv) {
+    sb = 0;
+    S = 0.0f;
+    inv = 0.0f;
+    if (s_t != 0.0f) {
+        const float ratio = __fdiv_rn(amax_b, six_st);
+        sb = cvt_e4m3x2(0.0f, ratio) & 0xFFu;
+        S = __fmul_rn(f16_lo(cvt_e4m3x2_f16x2(sb)), s_t);
+        inv = (S == 0.0f) ? 0.0f : __frcp_rn(S);
+    }
+}
+
+// ------------------------------------------------------------------ k_fp4 (MXFP4; STE)
 // Per-lane result of the FP4 codec for 8 elements.
 struct Fp4Lane {
     uint32_t codes;     // 8 nibbles, element k in bits 4k..4k+3
@@ -230,46 +301,32 @@ struct Fp4Lane {
     float q[8];         // scaled values (for the clipped STE)
 };
 
-// MODE 0: codes + scales + (optionally) dequant.  Block statistics by shuffles.
-template <bool NV, bool WANT_Y>
-__device__ __forceinline__ void fp4_lane(uint4 v, float s_t, float six_st, Fp4Lane& o) {
-    uint32_t a = abs_max8(v);
+template <bool NV, bool WANT_Y, typename XT>
+__device__ __forceinline__ void fp4_lane(const Elems<XT, 8>& x, float s_t, float six_st,
+                                         Fp4Lane& o) {
+    uint32_t a = x.amax_bits();
     a = max(a, __shfl_xor_sync(kFull, a, 1));
     if (!NV) a = max(a, __shfl_xor_sync(kFull, a, 2));
     float S, inv;
     if (NV) {
-        // E4M3 block scale of the 16-element block held by this lane pair
-        uint32_t sb = 0;
-        S = 0.0f;
-        inv = 0.0f;
-        if (s_t != 0.0f) {
-            float ratio = __fdiv_rn(__uint_as_float(a << 16), six_st);
-            sb = cvt_e4m3x2(0.0f, ratio) & 0xFFu;
-            S = __fmul_rn(f16_lo(cvt_e4m3x2_f16x2(sb)), s_t);
-            inv = (S == 0.0f) ? 0.0f : __frcp_rn(S);
-        }
+        uint32_t sb;
+        nv_block_scale(__uint_as_float(a), s_t, six_st, sb, S, inv);
         o.scale = sb;
     } else {
         // E8M0: e = floor(log2 amax) - 2 clamped to >= -127; byte = e + 127 = max(E - 2, 0)
-        uint32_t E = a >> 7;
-        uint32_t c = E > 2u ? E - 2u : 0u;
+        const uint32_t E = a >> 23;
+        const uint32_t c = E > 2u ? E - 2u : 0u;
         o.scale = c;
-        inv = __uint_as_float((254u - c) << 23);                      // 2^-e
-        S = c ? __uint_as_float(c << 23) : __uint_as_float(0x00200000u);   // 2^e
+        inv = __uint_as_float((254u - c) << 23);                          // 2^-e
+        S = c ? __uint_as_float(c << 23) : __uint_as_float(0x00200000u);  // 2^e
     }
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        o.q[2 * k] = __fmul_rn(bf16_lo(w[k]), inv);
-        o.q[2 * k + 1] = __fmul_rn(bf16_hi(w[k]), inv);
-    }
+    for (int k = 0; k < 8; ++k) o.q[k] = __fmul_rn(x.get(k), inv);
     if (NV && __builtin_expect(isinf(inv), 0)) {
         // 1/S overflowed (S < 2^-128): a zero keeps its own sign instead of 0 * inf
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            if (bf16_lo(w[k]) == 0.0f) o.q[2 * k] = bf16_lo(w[k]);
-            if (bf16_hi(w[k]) == 0.0f) o.q[2 * k + 1] = bf16_hi(w[k]);
-        }
+        for (int k = 0; k < 8; ++k)
+            if (x.get(k) == 0.0f) o.q[k] = x.get(k);
     }
     uint32_t b[4];
 #pragma unroll
@@ -279,39 +336,35 @@ __device__ __forceinline__ void fp4_lane(uint4 v, float s_t, float six_st, Fp4La
         uint32_t yw[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-            uint32_t h2 = cvt_e2m1x2_f16x2(b[k]);
+            const uint32_t h2 = cvt_e2m1x2_f16x2(b[k]);
             yw[k] = cvt_bf16x2(__fmul_rn(f16_hi(h2), S), __fmul_rn(f16_lo(h2), S));
         }
         o.y = make_uint4(yw[0], yw[1], yw[2], yw[3]);
     }
 }
 
-// Loads of one warp unit (U sub-tiles of 256 elements): v = x, gv = upstream gradient
-// (STE only).  Lanes past the end of the tensor load zeros.
-template <int U, int MODE>
+template <typename XT, int U, int MODE>
 struct UnitLoad {
-    uint4 v[U];
+    Elems<XT, 8> v[U];
     uint4 gv[MODE == 1 ? U : 1];
 };
 
-template <int U, int MODE>
+template <typename XT, int U, int MODE>
 __device__ __forceinline__ void load_unit(const DevTensor& T, int64_t e0, int lane,
-                                          UnitLoad<U, MODE>& L) {
-    constexpr int LD = QF_FP4_LD;
+                                          UnitLoad<XT, U, MODE>& L) {
+    const XT* x = static_cast<const XT*>(T.x);
 #pragma unroll
     for (int s = 0; s < U; ++s) {
         const int64_t e = e0 + s * 256 + lane * 8;
         const bool ok = e < T.numel;
-        L.v[s] = ok ? ld_stream<LD>(T.x + e) : make_uint4(0, 0, 0, 0);
-        if (MODE == 1) L.gv[s] = ok ? ld_stream<LD>(T.g + e) : make_uint4(0, 0, 0, 0);
+        L.v[s].template load<QF_FP4_LD>(x + e, ok);
+        if (MODE == 1) L.gv[s] = ok ? ld_stream<QF_FP4_LD>(T.g + e) : make_uint4(0, 0, 0, 0);
     }
 }
 
-// Fused NVFP4 / MXFP4 fake-quant + pack (MODE 0) or clipped STE (MODE 1).
-// A unit is U sub-tiles of 256 elements.  The loads of a warp's next unit are
-// issued before the current one is computed, so every warp keeps a unit of
-// reads in flight while it converts.
-template <bool NV, int U, int MAXT, int MODE, int THREADS, int PREFETCH>
+// MXFP4 fused fake-quant + pack (MODE 0), or the NVFP4 / MXFP4 clipped STE (MODE 1).
+// A unit is U sub-tiles of 256 elements.
+template <bool NV, typename XT, int U, int MAXT, int MODE, int THREADS, int PREFETCH>
 __global__ void __launch_bounds__(THREADS) k_fp4(const __grid_constant__ Table<MAXT> P) {
     const int lane = threadIdx.x & 31;
     const int64_t warp = (int64_t(blockIdx.x) * THREADS + threadIdx.x) >> 5;
@@ -324,18 +377,17 @@ __global__ void __launch_bounds__(THREADS) k_fp4(const __grid_constant__ Table<M
     int64_t u = warp;
     if (u >= P.total_units) return;
     int ti = locate_tensor(P, u);
-    UnitLoad<U, MODE> cur;
-    load_unit<U, MODE>(P.t[ti], (u - P.t[ti].unit_begin) * kUnit, lane, cur);
+    UnitLoad<XT, U, MODE> cur;
+    load_unit<XT, U, MODE>(P.t[ti], (u - P.t[ti].unit_begin) * kUnit, lane, cur);
     int cur_t = -1;
     float s_t = 0.0f, six_st = 0.0f;
     while (true) {
-        // prefetch the next unit of this warp
         const int64_t un = u + nwarps;
         int tn = ti;
-        UnitLoad<U, MODE> nxt;
+        UnitLoad<XT, U, MODE> nxt;
         if (PREFETCH && un < P.total_units) {
             tn = find_tensor(P, ti, un);
-            load_unit<U, MODE>(P.t[tn], (un - P.t[tn].unit_begin) * kUnit, lane, nxt);
+            load_unit<XT, U, MODE>(P.t[tn], (un - P.t[tn].unit_begin) * kUnit, lane, nxt);
         }
         const DevTensor& T = P.t[ti];
         if (NV && ti != cur_t) {
@@ -380,20 +432,20 @@ __global__ void __launch_bounds__(THREADS) k_fp4(const __grid_constant__ Table<M
             cur = nxt;
         } else {
             ti = find_tensor(P, ti, u);
-            load_unit<U, MODE>(P.t[ti], (u - P.t[ti].unit_begin) * kUnit, lane, cur);
+            load_unit<XT, U, MODE>(P.t[ti], (u - P.t[ti].unit_begin) * kUnit, lane, cur);
         }
     }
 }
 
 // ------------------------------------------------------------------ NVFP4, lane per block
 // NVFP4 fake-quant + pack with one lane per 16-element block: a warp sub-tile is 32
-// consecutive blocks (512 elements, 1 KB of BF16) and lane l owns block l, so the
-// E4M3 block scale (one IEEE divide, one reciprocal) is computed once per block and
-// the block max needs no shuffle.  A lane reads its block's 32 bytes with two 16-byte
-// loads (together they cover whole sectors; the second is served from L1) and writes
-// 32 bytes of BF16, 8 bytes of codes and 1 scale byte: the warp's code and scale
-// stores are contiguous 256- and 32-byte runs.
-template <int U, int MAXT, int THREADS, int PREFETCH>
+// consecutive blocks (512 elements) and lane l owns block l, so the E4M3 block scale
+// (one IEEE divide, one reciprocal) is computed once per block and the block max
+// needs no shuffle.  A lane reads its block with consecutive 16-byte loads (together
+// they cover whole sectors; the later ones are served from L1) and writes 32 bytes
+// of BF16, 8 bytes of codes and 1 scale byte: the warp's code and scale stores are
+// contiguous 256- and 32-byte runs.
+template <typename XT, int U, int MAXT, int THREADS, int PREFETCH>
 __global__ void __launch_bounds__(THREADS) k_nv(const __grid_constant__ Table<MAXT> P) {
     const int lane = threadIdx.x & 31;
     const int64_t warp = (int64_t(blockIdx.x) * THREADS + threadIdx.x) >> 5;
@@ -406,14 +458,13 @@ __global__ void __launch_bounds__(THREADS) k_nv(const __grid_constant__ Table<MA
     int64_t u = warp;
     if (u >= P.total_units) return;
     int ti = locate_tensor(P, u);
-    uint4 cur[2 * U], nxt[2 * U];
-    auto load = [&](const DevTensor& T, int64_t e0, uint4 (&v)[2 * U]) {
+    Elems<XT, 16> cur[U], nxt[U];
+    auto load = [&](const DevTensor& T, int64_t e0, Elems<XT, 16> (&v)[U]) {
+        const XT* x = static_cast<const XT*>(T.x);
 #pragma unroll
         for (int s = 0; s < U; ++s) {
             const int64_t e = e0 + s * 512 + lane * 16;
-            const bool ok = e < T.numel;
-            v[2 * s] = ok ? ld_stream<QF_FP4_LD>(T.x + e) : make_uint4(0, 0, 0, 0);
-            v[2 * s + 1] = ok ? ld_stream<QF_FP4_LD>(T.x + e + 8) : make_uint4(0, 0, 0, 0);
+            v[s].template load<QF_FP4_LD>(x + e, e < T.numel);
         }
     };
     load(P.t[ti], (u - P.t[ti].unit_begin) * kUnit, cur);
@@ -436,35 +487,18 @@ __global__ void __launch_bounds__(THREADS) k_nv(const __grid_constant__ Table<MA
 #pragma unroll
         for (int s = 0; s < U; ++s) {
             const int64_t e = e0 + s * 512 + lane * 16;
-            const uint32_t w[8] = {cur[2 * s].x, cur[2 * s].y, cur[2 * s].z, cur[2 * s].w,
-                                   cur[2 * s + 1].x, cur[2 * s + 1].y, cur[2 * s + 1].z,
-                                   cur[2 * s + 1].w};
-            uint32_t m = bmax2(bmax2(bmax2(w[0] & 0x7FFF7FFFu, w[1] & 0x7FFF7FFFu),
-                                     bmax2(w[2] & 0x7FFF7FFFu, w[3] & 0x7FFF7FFFu)),
-                               bmax2(bmax2(w[4] & 0x7FFF7FFFu, w[5] & 0x7FFF7FFFu),
-                                     bmax2(w[6] & 0x7FFF7FFFu, w[7] & 0x7FFF7FFFu)));
-            const uint32_t a = max(m & 0xFFFFu, m >> 16);
-            uint32_t sb = 0;
-            float S = 0.0f, inv = 0.0f;
-            if (s_t != 0.0f) {
-                const float ratio = __fdiv_rn(__uint_as_float(a << 16), six_st);
-                sb = cvt_e4m3x2(0.0f, ratio) & 0xFFu;
-                S = __fmul_rn(f16_lo(cvt_e4m3x2_f16x2(sb)), s_t);
-                inv = (S == 0.0f) ? 0.0f : __frcp_rn(S);
-            }
+            const Elems<XT, 16>& x = cur[s];
+            uint32_t sb;
+            float S, inv;
+            nv_block_scale(__uint_as_float(x.amax_bits()), s_t, six_st, sb, S, inv);
             float q[16];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                q[2 * k] = __fmul_rn(bf16_lo(w[k]), inv);
-                q[2 * k + 1] = __fmul_rn(bf16_hi(w[k]), inv);
-            }
+            for (int k = 0; k < 16; ++k) q[k] = __fmul_rn(x.get(k), inv);
             if (__builtin_expect(isinf(inv), 0)) {
                 // 1/S overflowed (S < 2^-128): a zero keeps its own sign instead of 0 * inf
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    if (bf16_lo(w[k]) == 0.0f) q[2 * k] = bf16_lo(w[k]);
-                    if (bf16_hi(w[k]) == 0.0f) q[2 * k + 1] = bf16_hi(w[k]);
-                }
+                for (int k = 0; k < 16; ++k)
+                    if (x.get(k) == 0.0f) q[k] = x.get(k);
             }
             uint32_t b[8];
 #pragma unroll
@@ -493,7 +527,7 @@ __global__ void __launch_bounds__(THREADS) k_nv(const __grid_constant__ Table<MA
         if (PREFETCH) {
             ti = tn;
 #pragma unroll
-            for (int i = 0; i < 2 * U; ++i) cur[i] = nxt[i];
+            for (int i = 0; i < U; ++i) cur[i] = nxt[i];
         } else {
             ti = find_tensor(P, ti, u);
             load(P.t[ti], (u - P.t[ti].unit_begin) * kUnit, cur);
@@ -505,10 +539,11 @@ __global__ void __launch_bounds__(THREADS) k_nv(const __grid_constant__ Table<MA
 // One lane per 32-element sub-block: a warp iteration covers 4 super-blocks (1024
 // elements) and lane l owns sub-block j = l / 4 of super-block b = l % 4, so the
 // per-sub-block and per-super-block scalar work (divides, FP16 and integer
-// conversions) is amortised over 32 elements instead of 8.  Global loads and
-// stores stay fully coalesced: the warp stages its 2 KB through shared memory
-// (one 528-byte row per super-block, 16 bytes of padding so that the lanes'
-// 16-byte accesses hit distinct banks) and transposes there.
+// conversions) is amortised over 32 elements.  BF16 traffic stays fully coalesced:
+// the warp stages its 2 KB through shared memory (one 528-byte row per
+// super-block, 16 bytes of padding so that the lanes' 16-byte accesses hit
+// distinct banks) and transposes there.  FP32 input is read by each lane directly
+// (its 128-byte sub-block, whole lines, the later vectors served from L1).
 constexpr int kQ4kRow = 528;
 constexpr int kQ4kWarpBytes = 4 * kQ4kRow;
 constexpr float kRound = 12582912.0f;      // 1.5 * 2^23: v + kRound rounds v to an integer (RNE)
@@ -524,16 +559,14 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     return v;
 }
 
-// Per-lane fit of one sub-block (32 BF16 in w[16]); returns the super-block's FP16
-// d / dmin bits, this sub-block's 6-bit sc / m, its s = d*sc, mm = dmin*m, inv = 1/s.
+// Per-lane fit of one sub-block; returns the super-block's FP16 d / dmin bits, this
+// sub-block's 6-bit sc / m, its s = d*sc, mm = dmin*m and inv = 1/s.
 struct Q4kFit { uint32_t dbits, dminbits, sc, m; float s, mm, inv; };
 
-__device__ __forceinline__ Q4kFit q4k_fit(const uint32_t (&w)[16]) {
-    uint32_t mx = w[0], mn = w[0];
-#pragma unroll
-    for (int k = 1; k < 16; ++k) { mx = bmax2(mx, w[k]); mn = bmin2(mn, w[k]); }
-    const float hi = fmaxf(bf16_lo(mx), bf16_hi(mx));
-    const float lo = fminf(bf16_lo(mn), bf16_hi(mn));
+template <typename XT>
+__device__ __forceinline__ Q4kFit q4k_fit(const Elems<XT, 32>& x) {
+    float lo, hi;
+    x.minmax(lo, hi);
     const float min_j = lo < 0.0f ? -lo : 0.0f;
     const float scale_j = __fdiv_rn(__fadd_rn(hi, min_j), 15.0f);
     float ms = scale_j, mm = min_j;
@@ -557,39 +590,43 @@ __device__ __forceinline__ Q4kFit q4k_fit(const uint32_t (&w)[16]) {
 }
 
 // MODE 0: dequant (y) and/or 144-byte blocks (codes).  MODE 1: clipped STE, y = grad_x.
-template <int MAXT, int MODE, int THREADS>
+template <typename XT, int MAXT, int MODE, int THREADS>
 __global__ void __launch_bounds__(THREADS) k_q4k(const __grid_constant__ Table<MAXT> P) {
     __shared__ __align__(16) uint8_t stage[THREADS / 32][kQ4kWarpBytes];
+    constexpr bool kBf16 = sizeof(XT) == 2;
     const int lane = threadIdx.x & 31;
     const int b = lane & 3, j = lane >> 2;              // super-block of 4, sub-block of 8
     const uint32_t sm = (uint32_t)__cvta_generic_to_shared(stage[threadIdx.x >> 5]);
     const uint32_t sm_lane = sm + 16u * lane;           // coalesced view: row k at + k*528
-    const uint32_t sm_mine = sm + b * kQ4kRow + 64u * j; // this lane's 64-byte sub-block
+    const uint32_t sm_mine = sm + b * kQ4kRow + 64u * j; // this lane's 64 bytes of BF16
     const int64_t warp = (int64_t(blockIdx.x) * THREADS + threadIdx.x) >> 5;
     const int64_t nwarps = (int64_t(gridDim.x) * THREADS) >> 5;
     int ti = warp < P.total_units ? locate_tensor(P, warp) : 0;
     for (int64_t u = warp; u < P.total_units; u += nwarps) {
         ti = find_tensor(P, ti, u);
         const DevTensor& T = P.t[ti];
+        const XT* xp = static_cast<const XT*>(T.x);
         const int64_t e0 = (u - T.unit_begin) * 1024;
         const int64_t left = (T.numel - e0) >> 8;
         const int nsb = left < 4 ? (int)left : 4;          // super-blocks in this unit
-        uint4 v[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-            v[k] = k < nsb ? ld_stream<0>(T.x + e0 + 256 * k + 8 * lane) : make_uint4(0, 0, 0, 0);
-        __syncwarp();
-#pragma unroll
-        for (int k = 0; k < 4; ++k) sts128(sm_lane + k * kQ4kRow, v[k]);
-        __syncwarp();
-        uint32_t w[16];
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            const uint4 t = lds128(sm_mine + 16 * p);
-            w[4 * p] = t.x; w[4 * p + 1] = t.y; w[4 * p + 2] = t.z; w[4 * p + 3] = t.w;
-        }
-        const Q4kFit f = q4k_fit(w);
         const bool have = b < nsb;
+        Elems<XT, 32> x;
+        if constexpr (kBf16) {
+            uint4 v[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                v[k] = k < nsb ? ld_stream<0>(xp + e0 + 256 * k + 8 * lane) : make_uint4(0, 0, 0, 0);
+            __syncwarp();
+#pragma unroll
+            for (int k = 0; k < 4; ++k) sts128(sm_lane + k * kQ4kRow, v[k]);
+            __syncwarp();
+#pragma unroll
+            for (int p = 0; p < 4; ++p) x.v[p] = lds128(sm_mine + 16 * p);
+        } else {
+            x.template load<1>(xp + e0 + 256 * b + 32 * j, have);
+            __syncwarp();                                  // the previous unit's staging reads
+        }
+        const Q4kFit f = q4k_fit(x);
         const int64_t sb = (e0 >> 8) + b;                // this lane's super-block in the tensor
         if (MODE == 0) {
             // elements: q = clamp(RNE((x + mm) * inv), 0, 15); y = BF16(s*q - mm)
@@ -600,8 +637,7 @@ __global__ void __launch_bounds__(THREADS) k_q4k(const __grid_constant__ Table<M
                 float r[2];
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    const float x = h ? bf16_hi(w[k]) : bf16_lo(w[k]);
-                    const float t = __fmul_rn(__fadd_rn(x, f.mm), f.inv);
+                    const float t = __fmul_rn(__fadd_rn(x.get(2 * k + h), f.mm), f.inv);
                     r[h] = __fadd_rn(fminf(fmaxf(t, 0.0f), 15.0f), kRound);
                 }
                 if (k & 1) qw[k >> 1] = __byte_perm(qw[k >> 1], __byte_perm(__float_as_uint(r[0]),
@@ -658,12 +694,11 @@ __global__ void __launch_bounds__(THREADS) k_q4k(const __grid_constant__ Table<M
             // clipped STE: keep grad where 0 <= (x + mm) * inv <= 15
             uint32_t keep = 0;
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const float t0 = __fmul_rn(__fadd_rn(bf16_lo(w[k]), f.mm), f.inv);
-                const float t1 = __fmul_rn(__fadd_rn(bf16_hi(w[k]), f.mm), f.inv);
-                keep |= (uint32_t)(t0 >= 0.0f && t0 <= 15.0f) << (2 * k);
-                keep |= (uint32_t)(t1 >= 0.0f && t1 <= 15.0f) << (2 * k + 1);
+            for (int k = 0; k < 32; ++k) {
+                const float t = __fmul_rn(__fadd_rn(x.get(k), f.mm), f.inv);
+                keep |= (uint32_t)(t >= 0.0f && t <= 15.0f) << k;
             }
+            uint4 v[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k)
                 v[k] = k < nsb ? ld_stream<0>(T.g + e0 + 256 * k + 8 * lane) : make_uint4(0, 0, 0, 0);
@@ -674,14 +709,14 @@ __global__ void __launch_bounds__(THREADS) k_q4k(const __grid_constant__ Table<M
 #pragma unroll
             for (int p = 0; p < 4; ++p) {
                 uint4 g = lds128(sm_mine + 16 * p);
-                uint32_t* gw = reinterpret_cast<uint32_t*>(&g);
+                uint32_t gw[4] = {g.x, g.y, g.z, g.w};
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const int k = 4 * p + q;
-                    gw[q] = (((keep >> (2 * k)) & 1u) ? (gw[q] & 0xFFFFu) : 0u) |
-                            (((keep >> (2 * k + 1)) & 1u) ? (gw[q] & 0xFFFF0000u) : 0u);
+                    const int k = 8 * p + 2 * q;                 // elements k, k+1 of this lane
+                    gw[q] = (((keep >> k) & 1u) ? (gw[q] & 0xFFFFu) : 0u) |
+                            (((keep >> (k + 1)) & 1u) ? (gw[q] & 0xFFFF0000u) : 0u);
                 }
-                sts128(sm_mine + 16 * p, g);
+                sts128(sm_mine + 16 * p, make_uint4(gw[0], gw[1], gw[2], gw[3]));
             }
             __syncwarp();
 #pragma unroll
@@ -692,16 +727,15 @@ __global__ void __launch_bounds__(THREADS) k_q4k(const __grid_constant__ Table<M
 }
 
 // ------------------------------------------------------------------ tied amax
-// Running max|x| per lane while the warp stays in one tie group; on a group
-// change (and at the end) the warp reduces and lane 0 does one atomicMax on the
+// Each CTA reduces one contiguous range of units, so a warp stays inside one tensor
+// (one tie group) for many units; it keeps a running max |x| as FP32 bits and, on a
+// group change and at the end, reduces across the warp and does one atomicMax on the
 // group's FP32 bits (non-negative floats order like their bit patterns).
-template <int U, int MAXT, int THREADS>
+template <typename XT, int U, int MAXT, int THREADS>
 __global__ void __launch_bounds__(THREADS) k_amax(const __grid_constant__ Table<MAXT> P) {
     const int lane = threadIdx.x & 31;
     constexpr int kUnit = 256 * U;
     constexpr int kWarps = THREADS / 32;
-    // each CTA reduces one contiguous range of units, so a warp stays inside one
-    // tensor (one tie group) for many units and flushes its max rarely
     const int64_t per_cta = (P.total_units + gridDim.x - 1) / gridDim.x;
     const int64_t u_begin = int64_t(blockIdx.x) * per_cta;
     const int64_t u_end = min(u_begin + per_cta, P.total_units);
@@ -709,14 +743,14 @@ __global__ void __launch_bounds__(THREADS) k_amax(const __grid_constant__ Table<
     const int64_t u_first = u_begin + (threadIdx.x >> 5);
     int ti = u_first < u_end ? locate_tensor(P, u_first) : 0;
     int g = -1;
-    uint32_t run = 0;          // bf16x2 running max of |x|
+    uint32_t run = 0;
     auto flush = [&](int grp) {
-        uint32_t a = max(run & 0xFFFFu, run >> 16);
+        uint32_t a = run;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) a = max(a, __shfl_xor_sync(kFull, a, o));
         if (lane == 0 && grp >= 0) {
-            atomicMax(reinterpret_cast<unsigned int*>(amax) + grp, a << 16);
-            if (P.tracked) atomicMax(reinterpret_cast<unsigned int*>(P.tracked) + grp, a << 16);
+            atomicMax(reinterpret_cast<unsigned int*>(amax) + grp, a);
+            if (P.tracked) atomicMax(reinterpret_cast<unsigned int*>(P.tracked) + grp, a);
         }
         run = 0;
     };
@@ -727,25 +761,23 @@ __global__ void __launch_bounds__(THREADS) k_amax(const __grid_constant__ Table<
             if (g >= 0) flush(g);
             g = T.group;
         }
+        const XT* x = static_cast<const XT*>(T.x);
         const int64_t e0 = (u - T.unit_begin) * kUnit;
-        uint4 v[U];
+        Elems<XT, 8> v[U];
 #pragma unroll
         for (int s = 0; s < U; ++s) {
             const int64_t e = e0 + s * 256 + lane * 8;
-            v[s] = (e + 8 <= T.numel) ? ld_stream<QF_AMAX_LD>(T.x + e) : make_uint4(0, 0, 0, 0);
+            v[s].template load<QF_AMAX_LD>(x + e, e + 8 <= T.numel);
         }
 #pragma unroll
-        for (int s = 0; s < U; ++s) {
-            run = bmax2(run, bmax2(bmax2(v[s].x & 0x7FFF7FFFu, v[s].y & 0x7FFF7FFFu),
-                                   bmax2(v[s].z & 0x7FFF7FFFu, v[s].w & 0x7FFF7FFFu)));
-        }
+        for (int s = 0; s < U; ++s) run = max(run, v[s].amax_bits());
     }
     if (g >= 0) flush(g);
 }
 
 // amax of tensors whose element count is not a multiple of 8 handles the
 // scalar tail here (one thread per leftover element; at most 7 per tensor).
-template <int MAXT>
+template <typename XT, int MAXT>
 __global__ void k_amax_tail(const __grid_constant__ Table<MAXT> P) {
     const int ti = blockIdx.x;
     if (ti >= P.n) return;
@@ -753,7 +785,11 @@ __global__ void k_amax_tail(const __grid_constant__ Table<MAXT> P) {
     const int64_t start = T.numel & ~int64_t(7);
     const int64_t e = start + threadIdx.x;
     if (threadIdx.x < 8 && e < T.numel) {
-        const uint32_t a = (uint32_t)(T.x[e] & 0x7FFFu) << 16;
+        uint32_t a;
+        if constexpr (sizeof(XT) == 2)
+            a = (uint32_t)(static_cast<const uint16_t*>(T.x)[e] & 0x7FFFu) << 16;
+        else
+            a = __float_as_uint(static_cast<const float*>(T.x)[e]) & 0x7FFFFFFFu;
         atomicMax(reinterpret_cast<unsigned int*>(const_cast<float*>(P.group_amax)) + T.group, a);
         if (P.tracked) atomicMax(reinterpret_cast<unsigned int*>(P.tracked) + T.group, a);
     }

@@ -66,6 +66,10 @@ typedef enum {
     QF_ERR_CUDA = 5           /* a CUDA call failed (see qf_last_error) */
 } qf_status;
 
+/* Element type of the input x (qf_tensor.x_type). */
+#define QF_X_BF16 0             /* BF16 weights or activations */
+#define QF_X_F32 1              /* FP32 latent (master) weights */
+
 #define QF_NVFP4_BLOCK 16
 #define QF_MXFP4_BLOCK 32
 #define QF_Q4K_SUBBLOCK 32
@@ -74,14 +78,19 @@ typedef enum {
 
 /*
  * One tensor of a call.
- *   x       BF16 [rows, cols], 16-byte aligned.  May be NULL only if rows*cols == 0.
+ *   x       [rows, cols] of x_type elements, 16-byte aligned.  May be NULL only if
+ *           rows*cols == 0.
  *   rows    >= 0
  *   cols    >= 0, a multiple of the format's block size
  *   group   NVFP4 tie group in [0, n_groups): every tensor of a group shares one
  *           FP32 tensor scale (the projections an engine fuses, e.g. Q, K and V,
  *           or gate and up -- project page, Method, "Numerics").  Ignored by
  *           MXFP4 and Q4_K.
- *   reserved  must be 0
+ *   x_type  QF_X_BF16 (0) or QF_X_F32 (1): BF16 inputs, or the FP32 latent weights a
+ *           full-parameter training run keeps (the project page's memory table lists
+ *           the student's trainable weights as FP32).  Every tensor of one call has
+ *           the same x_type.  The outputs are the same for both: BF16 y, codes,
+ *           scales; an FP32 element that is a BF16 value gives the BF16 result.
  *   y       BF16 [rows, cols] dequantized output, 16-byte aligned, or NULL
  *   codes   packed output, 16-byte aligned, or NULL:
  *             NVFP4 / MXFP4: rows*cols/2 bytes; element 2i of the flat tensor in
@@ -100,7 +109,7 @@ typedef struct qf_tensor {
     int64_t rows;
     int64_t cols;
     int32_t group;
-    int32_t reserved;
+    int32_t x_type;
     void* y;
     void* codes;
     void* scales;
@@ -118,8 +127,8 @@ typedef struct qf_tensor {
  *                     max(d_tracked[g], d_group_amax[g])  (the running amax a
  *                     training loop keeps for activations; pass it as the
  *                     d_group_amax of qf_fakequant to quantize with it).
- *   Only x, rows, cols and group of each tensor are read; cols may be any value
- *   >= 0 here.  n == 0 only clears d_group_amax.
+ *   Only x, rows, cols, group and x_type of each tensor are read; cols may be any
+ *   value >= 0 here.  n == 0 only clears d_group_amax.
  * Errors: t == NULL with n > 0, n < 0, n_groups <= 0, d_group_amax == NULL,
  *   group out of range -> QF_ERR_INVALID_ARG; bad sizes -> QF_ERR_SHAPE;
  *   x not 16-byte aligned -> QF_ERR_ALIGN.
@@ -184,7 +193,7 @@ qf_status qf_pack(qf_format f, const qf_tensor* t, int n, const float* d_group_a
  *                       the element, +0 elsewhere: NVFP4/MXFP4 |x * inv| <= 6,
  *                       Q4_K 0 <= (x + mm_j) * inv_j <= 15, with the scales the
  *                       forward pass of format f derives for fwd->x.  fwd gives x,
- *                       rows, cols and (NVFP4) group; numel == rows * cols;
+ *                       x_type, rows, cols and (NVFP4) group; numel == rows * cols;
  *                       d_group_amax as for qf_fakequant (NVFP4 only).
  *   grad_y, grad_x: BF16 device arrays, 16-byte aligned.
  * Errors: mode not 0/1 or unknown format -> QF_ERR_UNSUPPORTED; the rest as above.
@@ -199,7 +208,8 @@ const char* qf_status_string(qf_status s);
 /* One-line description of the last failed call on the calling thread ("" if none). */
 const char* qf_last_error(void);
 
-/* ABI version: (major << 16) | minor. */
+/* ABI version: (major << 16) | minor.  1.1 added qf_tensor.x_type (formerly a
+ * reserved field that had to be 0, which still means BF16). */
 int qf_version(void);
 
 #ifdef __cplusplus

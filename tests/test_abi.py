@@ -58,14 +58,14 @@ def test_struct_layout_matches_header(qf):
 def test_status_strings(qf):
     for s in range(6):
         assert qf.lib.qf_status_string(s).decode().startswith("QF_")
-    assert qf.lib.qf_version() >> 16 == 1
+    assert qf.lib.qf_version() == (1 << 16) | 1
 
 
 def _tensor(qf, x=0x1000, rows=4, cols=64, group=0, y=0x2000, codes=0x3000, scales=0x4000,
-            reserved=0):
+            x_type=0):
     arr = (qf.binding.QfTensor * 1)()
     t = arr[0]
-    t.x, t.rows, t.cols, t.group, t.reserved = x, rows, cols, group, reserved
+    t.x, t.rows, t.cols, t.group, t.x_type = x, rows, cols, group, x_type
     t.y, t.codes, t.scales = y, codes, scales
     return arr
 
@@ -90,7 +90,9 @@ def test_validation_codes(qf, pack):
     assert _fq(qf, 1, _tensor(qf, x=0x1008), pack=pack) == ALIGN
     assert _fq(qf, 1, _tensor(qf, codes=0x3004), pack=pack) == ALIGN
     assert _fq(qf, 1, _tensor(qf, x=0), pack=pack) == INV
-    assert _fq(qf, 1, _tensor(qf, reserved=1), pack=pack) == INV
+    assert _fq(qf, 1, _tensor(qf, x_type=2), pack=pack) == UNSUP
+    two = (qf.binding.QfTensor * 2)(_tensor(qf)[0], _tensor(qf, x_type=1)[0])
+    assert _fq(qf, 1, two, n=2, pack=pack) == INV                    # mixed element types
     assert _fq(qf, 1, _tensor(qf, y=0, codes=0, scales=0), pack=pack) == INV
     # Q4_K ignores `scales`: a pack with no codes has no output
     assert _fq(qf, 2, _tensor(qf, cols=256, codes=0), pack=True) == INV

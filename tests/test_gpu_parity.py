@@ -306,3 +306,56 @@ def test_full_activation_tracked():
     assert res["tracked"][0] == np.float32(am)
     compare_rows("nvfp4", a, res["y"][0], res["codes"][0], res["scales"][0],
                  sample_rows(a.shape[0], 48, 400), float(am), label="act")
+
+
+# ----------------------------------------------------------------------------- FP32 latent input
+def _f32_weights(rows, cols, seed, std=0.02, outliers=1e-3):
+    rng = np.random.default_rng([seed, 7])
+    a = rng.standard_normal((rows, cols), dtype=np.float32) * np.float32(std)
+    k = int(round(outliers * a.size))
+    if k:
+        idx = rng.choice(a.size, size=k, replace=False)
+        a.reshape(-1)[idx] *= np.float32(20.0)
+    return torch.from_numpy(a)
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4", "q4k"])
+def test_f32_latent_weights(fmt):
+    """FP32 master weights (not BF16-representable) through every format, grouped."""
+    shapes = [(64, 4096), (16, 4096), (16, 4096), (48, 1024), (3, 256)]
+    ts = [_f32_weights(r, c, 60 + i) for i, (r, c) in enumerate(shapes)]
+    groups = [0, 0, 0, 1, 1]
+    res = run_fakequant(fmt, ts, groups, 2)
+    am = oracle.tied_amax(ts, groups, 2) if fmt == "nvfp4" else None
+    if fmt == "nvfp4":
+        assert_same("f32 amax", res["amax"].view(np.uint32), am.view(np.uint32))
+    compare_full(fmt, ts, res, am, groups, label=f"f32 {fmt}")
+
+
+def test_f32_equal_to_bf16_when_representable():
+    wl = workloads.nvfp4_tied(rows_scale=1 / 64, with_grads=False)
+    for fmt in ("nvfp4", "mxfp4", "q4k"):
+        a = run_fakequant(fmt, wl["tensors"], wl["groups"], 2)
+        b = run_fakequant(fmt, [t.float() for t in wl["tensors"]], wl["groups"], 2)
+        for k in ("y", "codes", "scales"):
+            for u, v in zip(a[k], b[k]):
+                if u is not None:
+                    assert_same(f"{fmt} {k}", v, u)
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4", "q4k"])
+def test_f32_clipped_ste_and_ragged_amax(fmt):
+    x = _f32_weights(8, 512, 70, std=0.05, outliers=2e-2)
+    g = workloads.normal_with_outliers(8, 512, 1e-3, 0, 1, 3, 71)
+    am = oracle.tied_amax([x], [0], 1)
+    out = torch.empty(x.shape, dtype=torch.bfloat16, device=DEV)
+    qf.qf_ste_backward(g.to(DEV), out, mode=1, fmt=fmt, x=x.to(DEV), group=0,
+                       group_amax=torch.from_numpy(am).to(DEV) if fmt == "nvfp4" else None)
+    torch.cuda.synchronize()
+    assert_same(f"f32 ste {fmt}", bits(out), oracle.ste_backward(g, 1, fmt, x, float(am[0])))
+    ts = [_f32_weights(r, c, 80 + i) for i, (r, c) in enumerate([(1, 3), (3, 5), (2, 1031)])]
+    amax = torch.empty(1, device=DEV)
+    qf.qf_amax_tied([t.to(DEV) for t in ts], [0, 0, 0], amax)
+    torch.cuda.synchronize()
+    want = oracle.tied_amax(ts, [0, 0, 0], 1)
+    assert_same("f32 ragged amax", amax.cpu().numpy().view(np.uint32), want.view(np.uint32))

@@ -35,23 +35,30 @@ def to_bf16(a: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16)
 
 
+def _out(a: np.ndarray, dtype: str) -> torch.Tensor:
+    """BF16 tensor, or the FP32 samples themselves (latent master weights)."""
+    if dtype == "f32":
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
+    return to_bf16(a)
+
+
 def normal_with_outliers(rows: int, cols: int, std: float, frac: float, factor: float,
-                         seed: int, index: int = 0) -> torch.Tensor:
+                         seed: int, index: int = 0, dtype: str = "bf16") -> torch.Tensor:
     rng = _rng(seed, index)
     a = rng.standard_normal(rows * cols, dtype=np.float32) * np.float32(std)
     k = int(round(frac * a.size))
     if k:
         idx = rng.choice(a.size, size=k, replace=False)
         a[idx] *= np.float32(factor)
-    return to_bf16(a.reshape(rows, cols))
+    return _out(a.reshape(rows, cols), dtype)
 
 
 def row_scaled_normal(rows: int, cols: int, std: float, lo: float, hi: float,
-                      seed: int, index: int = 0) -> torch.Tensor:
+                      seed: int, index: int = 0, dtype: str = "bf16") -> torch.Tensor:
     rng = _rng(seed, index)
     a = rng.standard_normal((rows, cols), dtype=np.float32) * np.float32(std)
     f = np.exp(rng.uniform(np.log(lo), np.log(hi), size=(rows, 1))).astype(np.float32)
-    return to_bf16(a * f)
+    return _out(a * f, dtype)
 
 
 def student_t_channels(rows: int, cols: int, df: float, chan_frac: float, factor: float,
@@ -89,21 +96,23 @@ def mxfp4_w4a4(rows_scale: float = 1.0, seed: int = 1):
     return {"tensors": [w, a], "names": ["w", "a"], "groups": [0, 0], "n_groups": 1}
 
 
-def q4k_weights(rows_scale: float = 1.0, seed: int = 2):
+def q4k_weights(rows_scale: float = 1.0, seed: int = 2, dtype: str = "bf16"):
     """Q4_K weight-only: down-proj 4096x14336 and up-proj 14336x4096,
     N(0, 0.015) times a per-row factor log-uniform in [0.5, 2]."""
-    down = row_scaled_normal(_rows(4096, rows_scale), 14336, 0.015, 0.5, 2.0, seed, 0)
-    up = row_scaled_normal(_rows(14336, rows_scale), 4096, 0.015, 0.5, 2.0, seed, 1)
+    down = row_scaled_normal(_rows(4096, rows_scale), 14336, 0.015, 0.5, 2.0, seed, 0, dtype)
+    up = row_scaled_normal(_rows(14336, rows_scale), 4096, 0.015, 0.5, 2.0, seed, 1, dtype)
     return {"tensors": [down, up], "names": ["down", "up"], "groups": [0, 0], "n_groups": 1}
 
 
-def nvfp4_tied(rows_scale: float = 1.0, seed: int = 3, with_grads: bool = True):
+def nvfp4_tied(rows_scale: float = 1.0, seed: int = 3, with_grads: bool = True,
+               dtype: str = "bf16"):
     """NVFP4 tied-scale fused projections: Q 4096x4096, K and V 1024x4096 (tie
     group 0), gate and up 14336x4096 (tie group 1); N(0, 0.02) with 0.1% x20
-    outliers; upstream gradients N(0, 1e-3) of the same shapes."""
+    outliers; upstream gradients N(0, 1e-3) of the same shapes.  dtype="f32" gives the FP32
+    latent master weights (the same samples, not rounded to BF16)."""
     shapes = [(4096, 4096), (1024, 4096), (1024, 4096), (14336, 4096), (14336, 4096)]
     names = ["q", "k", "v", "gate", "up"]
-    ts = [normal_with_outliers(_rows(r, rows_scale), c, 0.02, 1e-3, 20.0, seed, i)
+    ts = [normal_with_outliers(_rows(r, rows_scale), c, 0.02, 1e-3, 20.0, seed, i, dtype)
           for i, (r, c) in enumerate(shapes)]
     out = {"tensors": ts, "names": names, "groups": [0, 0, 0, 1, 1], "n_groups": 2}
     if with_grads:
