@@ -43,6 +43,8 @@ PARITY = {
     "mxfp4_quant": "on-grid round trip, idempotence, symmetry, brute-force nearest code, decoder",
     "q4k_quant": "on-grid round trip, brute-force nearest q, decoder, error bound",
     "ste_backward": "identity copy; clipped mask vs brute-force saturation",
+    "lora_merge": "exact integer-grid merges vs numpy; zero adapter / zero scale give W; "
+                  "float64 reference within one BF16 step; row/column locality",
 }
 
 
@@ -87,6 +89,7 @@ def _load():
             "qfo_ste_backward_x": (None, [P, P, I64, ctypes.c_int, ctypes.c_int, P, ctypes.c_int,
                                           I64, F]),
             "qfo_nvfp4_tensor_scale": (F, [F]),
+            "qfo_lora_merge": (None, [P, P, P, I64, I64, ctypes.c_int, F, P]),
             "qfo_nvfp4_quant": (None, [P, I64, I64, F, P, P, P, P]),
             "qfo_mxfp4_quant": (None, [P, I64, I64, P, P, P]),
             "qfo_q4k_quant": (None, [P, I64, I64, P, P]),
@@ -298,6 +301,19 @@ def q4k_decode(blocks, numel: int) -> np.ndarray:
     y = np.empty(numel, np.uint16)
     _load().qfo_q4k_decode(_ptr(np.ascontiguousarray(blocks)), numel, _ptr(y))
     return y
+
+
+def lora_merge(w, b, a, scale: float) -> np.ndarray:
+    """The BF16 merged weight M = BF16(W + scale * (B @ A)), B @ A accumulated in FP32
+    in increasing k.  w: [rows, cols], b: [rows, r], a: [r, cols], all BF16."""
+    wb, bb, ab = _bits(w), _bits(b), _bits(a)
+    rows, cols = wb.shape
+    r = bb.shape[1]
+    assert bb.shape[0] == rows and ab.shape == (r, cols)
+    m = np.empty((rows, cols), np.uint16)
+    _load().qfo_lora_merge(_ptr(wb), _ptr(np.ascontiguousarray(bb)), _ptr(np.ascontiguousarray(ab)),
+                           rows, cols, r, float(scale), _ptr(m))
+    return m
 
 
 FORMATS = {"nvfp4": 0, "mxfp4": 1, "q4k": 2}

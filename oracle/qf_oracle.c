@@ -573,6 +573,32 @@ void qfo_ste_backward_x(const uint16_t* grad_y, uint16_t* grad_x, int64_t numel,
     }
 }
 
+/* ------------------------------------------------------------------------ */
+/* LoRA merge [M-QAD]: LoRA-QAD trains low-rank adapters on a frozen BF16    */
+/* base and quantizes W + B A, not W.  Reading: the merged weight is what a  */
+/* BF16 model would hold after merging --                                    */
+/*   acc  = sum over k = 0..r-1, in increasing k, of B[i,k] * A[k,j]  (FP32; */
+/*          a BF16 x BF16 product is exact in FP32, each sum is rounded)     */
+/*   M    = BF16( W[i,j] + scale * acc )   (FP32 multiply, FP32 add, RNE)    */
+/* B is [rows, r] and A is [r, cols], both BF16 row-major; scale is FP32      */
+/* (alpha / r in the usual parameterisation).                                */
+/* ------------------------------------------------------------------------ */
+void qfo_lora_merge(const uint16_t* w, const uint16_t* b, const uint16_t* a, int64_t rows,
+                    int64_t cols, int rank, float scale, uint16_t* m)
+{
+    for (int64_t i = 0; i < rows; ++i) {
+        for (int64_t j = 0; j < cols; ++j) {
+            float acc = 0.0f;
+            for (int k = 0; k < rank; ++k) {
+                float prod = qfo_bf16_to_f32(b[i * rank + k]) * qfo_bf16_to_f32(a[(int64_t)k * cols + j]);
+                acc = acc + prod;
+            }
+            float d = scale * acc;
+            m[i * cols + j] = qfo_f32_to_bf16(qfo_bf16_to_f32(w[i * cols + j]) + d);
+        }
+    }
+}
+
 /* BF16-input entry points (the common case). */
 void qfo_nvfp4_quant(const uint16_t* x, int64_t rows, int64_t cols, float amax_g,
                      uint16_t* y, uint8_t* codes, uint8_t* scales, float* s_t_out)
