@@ -49,7 +49,7 @@ UNIT = "GB/s"
 BYTES_PER_ELEM = {"nvfp4": 2 + 2 + 0.5 + 1 / 16, "mxfp4": 2 + 2 + 0.5 + 1 / 32,
                   "q4k": 2 + 2 + 144 / 256}
 WORKLOADS = ("w4a4", "nvfp4_tied", "q4k", "nvfp4_weight", "activation", "moe_nvfp4",
-             "moe_mxfp4", "moe_q4k", "nvfp4_tied_f32", "q4k_f32")
+             "moe_mxfp4", "moe_q4k", "nvfp4_tied_f32", "q4k_f32", "lora_nvfp4")
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -186,6 +186,10 @@ def make_workload(name: str, qf, dev, seed_shift: int = 0):
         wl, fmt = _CACHE[key], name[4:]
         desc = (f"MoE 128 experts x (gate, up 768x2048, down 2048x768), {fmt.upper()}; one grouped "
                 "launch over 384 tensors" + (" after a tied amax pass" if fmt == "nvfp4" else ""))
+    elif name == "lora_nvfp4":
+        wl, fmt = workloads.nvfp4_tied(seed=3 + seed_shift, with_grads=False), "nvfp4"
+        desc = ("LoRA-QAD NVFP4: tied Q/K/V and gate/up bases with rank-16 adapters (scale 2); "
+                "amax of the merged weights + one fused merge+fake-quant+pack launch")
     elif name == "activation":
         wl, fmt = workloads.nvfp4_activation(seed=5 + seed_shift), "nvfp4"
         desc = ("NVFP4 activation 32768x4096 Student-t(3) with tracked amax: amax pass "
@@ -203,6 +207,21 @@ def make_workload(name: str, qf, dev, seed_shift: int = 0):
     W = dict(name=name, fmt=fmt, desc=desc, xs=xs, xs_h=xs_h, outs=[t for t in Y + C + S if
              t is not None], numel=numel, fq_bytes=numel * (BYTES_PER_ELEM[fmt] + in_b - 2),
              n_tensors=len(xs), in_bytes=in_b)
+    if name == "lora_nvfp4":
+        r = 16
+        ads = [(workloads.normal_with_outliers(x.shape[0], r, 0.01, 0, 1, 9 + seed_shift, 2 * i)
+                .to(dev), workloads.normal_with_outliers(r, x.shape[1], 0.02, 0, 1, 9 + seed_shift,
+                                                         2 * i + 1).to(dev), 2.0)
+               for i, x in enumerate(xs)]
+        amax = torch.zeros(ng, dtype=torch.float32, device=dev)
+        so = torch.empty(ng, dtype=torch.float32, device=dev)
+        W["pre"] = qf.prepare_amax_tied_lora(xs, ads, groups, amax)
+        W["fq"] = qf.prepare_fakequant_lora(fmt, xs, ads, Y, C, S, groups, amax, so)
+        W["step_bytes"] = W["fq_bytes"] + 2 * numel
+        W["launches"] = 2
+        W["kernel"] = "k_lora_nvfp4"
+        W["adapters"] = ads
+        return W
     if fmt == "nvfp4":
         amax = torch.zeros(ng, dtype=torch.float32, device=dev)
         cur = torch.zeros(ng, dtype=torch.float32, device=dev)

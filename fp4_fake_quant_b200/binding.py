@@ -32,6 +32,12 @@ class QfTensor(ctypes.Structure):
                 ("y", ctypes.c_void_p), ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
 
 
+class QfLora(ctypes.Structure):
+    """Mirror of ``qf_lora`` (include/qf.h)."""
+    _fields_ = [("b", ctypes.c_void_p), ("a", ctypes.c_void_p), ("rank", ctypes.c_int32),
+                ("scale", ctypes.c_float)]
+
+
 class QfError(RuntimeError):
     def __init__(self, status: int, message: str):
         super().__init__(f"{STATUS.get(status, status)}: {message}")
@@ -49,7 +55,12 @@ def _load() -> ctypes.CDLL:
     lib.qf_fakequant.argtypes = [I, T, I, P, I, P, P]
     lib.qf_pack.argtypes = [I, T, I, P, I, P, P]
     lib.qf_ste_backward.argtypes = [I, P, P, I64, I, T, P, I, P]
-    for f in (lib.qf_amax_tied, lib.qf_fakequant, lib.qf_pack, lib.qf_ste_backward):
+    L = ctypes.POINTER(QfLora)
+    lib.qf_lora_merge.argtypes = [T, L, I, P]
+    lib.qf_amax_tied_lora.argtypes = [T, L, I, P, I, P]
+    lib.qf_fakequant_lora.argtypes = [I, T, L, I, P, I, P, P]
+    for f in (lib.qf_amax_tied, lib.qf_fakequant, lib.qf_pack, lib.qf_ste_backward,
+              lib.qf_lora_merge, lib.qf_amax_tied_lora, lib.qf_fakequant_lora):
         f.restype = I
     lib.qf_status_string.argtypes = [I]
     lib.qf_status_string.restype = ctypes.c_char_p
@@ -63,8 +74,9 @@ def _load() -> ctypes.CDLL:
 lib = _load()
 
 # the entry points declared in include/qf.h
-EXPORTS = ("qf_amax_tied", "qf_fakequant", "qf_pack", "qf_ste_backward", "qf_status_string",
-           "qf_last_error", "qf_version")
+EXPORTS = ("qf_amax_tied", "qf_fakequant", "qf_pack", "qf_ste_backward", "qf_lora_merge",
+           "qf_amax_tied_lora", "qf_fakequant_lora", "qf_status_string", "qf_last_error",
+           "qf_version")
 
 
 def _check(status: int) -> None:
@@ -204,3 +216,54 @@ def prepare_amax_tied(xs, groups, group_amax, tracked=None) -> Prepared:
     keep = (arr, list(xs), group_amax, tracked)
     return Prepared(lib.qf_amax_tied, (arr, n, _ptr(group_amax), group_amax.numel(), _ptr(tracked)),
                     keep)
+
+
+def _lora(adapters):
+    """adapters: sequence of (b [rows, r] BF16, a [r, cols] BF16, scale)."""
+    arr = (QfLora * max(len(adapters), 1))()
+    for i, (b, a, scale) in enumerate(adapters):
+        if b.dtype != torch.bfloat16 or a.dtype != torch.bfloat16:
+            raise TypeError("LoRA factors must be bfloat16")
+        arr[i].b = _ptr(b)
+        arr[i].a = _ptr(a)
+        arr[i].rank = int(a.shape[0])
+        arr[i].scale = float(scale)
+    return arr
+
+
+def qf_lora_merge(xs, adapters, merged, stream=None) -> None:
+    """merged[i] <- BF16(xs[i] + scale * b @ a), b @ a accumulated in FP32 in increasing k."""
+    arr, n = _desc(xs, merged)
+    _check(lib.qf_lora_merge(arr, _lora(adapters), n, _stream(stream)))
+
+
+def qf_amax_tied_lora(xs, adapters, groups, group_amax, stream=None):
+    arr, n = _desc(xs, groups=groups)
+    _check(lib.qf_amax_tied_lora(arr, _lora(adapters), n, _ptr(group_amax), group_amax.numel(),
+                                 _stream(stream)))
+    return group_amax
+
+
+def qf_fakequant_lora(fmt, xs, adapters, ys=None, codes=None, scales=None, groups=None,
+                      group_amax=None, group_scale_out=None, stream=None) -> None:
+    arr, n = _desc(xs, ys, codes, scales, groups)
+    ng = group_amax.numel() if group_amax is not None else 0
+    _check(lib.qf_fakequant_lora(_fmt(fmt), arr, _lora(adapters), n, _ptr(group_amax), ng,
+                                 _ptr(group_scale_out), _stream(stream)))
+
+
+def prepare_fakequant_lora(fmt, xs, adapters, ys=None, codes=None, scales=None, groups=None,
+                           group_amax=None, group_scale_out=None) -> "Prepared":
+    arr, n = _desc(xs, ys, codes, scales, groups)
+    la = _lora(adapters)
+    ng = group_amax.numel() if group_amax is not None else 0
+    keep = (arr, la, list(xs), list(adapters), ys, codes, scales, group_amax, group_scale_out)
+    return Prepared(lib.qf_fakequant_lora, (_fmt(fmt), arr, la, n, _ptr(group_amax), ng,
+                                            _ptr(group_scale_out)), keep)
+
+
+def prepare_amax_tied_lora(xs, adapters, groups, group_amax) -> "Prepared":
+    arr, n = _desc(xs, groups=groups)
+    la = _lora(adapters)
+    keep = (arr, la, list(xs), list(adapters), group_amax)
+    return Prepared(lib.qf_amax_tied_lora, (arr, la, n, _ptr(group_amax), group_amax.numel()), keep)

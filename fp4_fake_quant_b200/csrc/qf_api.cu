@@ -11,6 +11,7 @@
 
 #include "qf.h"
 #include "qf_device.cuh"
+#include "qf_lora.cuh"
 
 namespace {
 
@@ -238,9 +239,165 @@ qf_status fakequant_impl(qf_format f, const qf_tensor* t, int n, const float* d_
     return launch_format(f, 0, n > 0 ? t[0].x_type : QF_X_BF16, v, am, so, ng, s);
 }
 
+// ------------------------------------------------------------------ LoRA
+constexpr int kLoraSmallT = 8;
+constexpr int kLoraLargeT = 256;
+
+template <int MODE, int R>
+qf_status lora_launch_r(const std::vector<qf::LoraTensor>& v, const float* am, float* so, int ng,
+                        cudaStream_t s) {
+    for (size_t b = 0; b < v.size(); b += kLoraLargeT) {
+        const size_t cnt = std::min<size_t>(kLoraLargeT, v.size() - b);
+        float* sout = b == 0 ? so : nullptr;
+        auto fill = [&](auto& P) {
+            memset(&P, 0, sizeof P);
+            int64_t u = 0;
+            for (size_t i = 0; i < cnt; ++i) {
+                qf::LoraTensor d = v[b + i];
+                d.unit_begin = u;
+                u += ((d.rows + qf::kLoraRows - 1) / qf::kLoraRows) * d.col_groups;
+                P.t[i] = d;
+            }
+            P.total_units = u;
+            P.n = (int)cnt;
+            P.group_amax = am;
+            P.group_scale_out = sout;
+            P.n_groups = ng;
+        };
+        if (cnt <= (size_t)kLoraSmallT) {
+            qf::LoraTable<kLoraSmallT> P;
+            fill(P);
+            qf::k_lora<MODE, R, kLoraSmallT>
+                <<<(unsigned)std::max<int64_t>(1, P.total_units), qf::kLoraThreads, 0, s>>>(P);
+        } else {
+            qf::LoraTable<kLoraLargeT> P;
+            fill(P);
+            qf::k_lora<MODE, R, kLoraLargeT>
+                <<<(unsigned)std::max<int64_t>(1, P.total_units), qf::kLoraThreads, 0, s>>>(P);
+        }
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+    }
+    return QF_OK;
+}
+
+template <int MODE>
+qf_status lora_launch(const std::vector<qf::LoraTensor>& v, int max_rank, const float* am,
+                      float* so, int ng, cudaStream_t s) {
+    if (max_rank <= 8) return lora_launch_r<MODE, 8>(v, am, so, ng, s);
+    if (max_rank <= 16) return lora_launch_r<MODE, 16>(v, am, so, ng, s);
+    return lora_launch_r<MODE, 32>(v, am, so, ng, s);
+}
+
+// Validate and describe the (tensor, adapter) pairs of a LoRA call.
+qf_status lora_tensors(const qf_tensor* t, const qf_lora* l, int n, int cols_multiple,
+                       int n_groups, bool check_group, bool need_output,
+                       std::vector<qf::LoraTensor>* out, int* max_rank) {
+    if (n < 0) return fail(QF_ERR_INVALID_ARG, "n = %d < 0", n);
+    if (n > 0 && (t == nullptr || l == nullptr))
+        return fail(QF_ERR_INVALID_ARG, "tensor or adapter array is NULL");
+    *max_rank = 1;
+    for (int i = 0; i < n; ++i) {
+        qf_status st = check_tensor(t[i], i, cols_multiple, n_groups, check_group);
+        if (st != QF_OK) return st;
+        if (t[i].x_type != QF_X_BF16)
+            return fail(QF_ERR_UNSUPPORTED, "tensor %d: LoRA bases are BF16", i);
+        if (l[i].rank < 1 || l[i].rank > QF_LORA_MAX_RANK)
+            return fail(QF_ERR_INVALID_ARG, "tensor %d: rank %d outside [1, %d]", i, l[i].rank,
+                        QF_LORA_MAX_RANK);
+        const int64_t numel = t[i].rows * t[i].cols;
+        if (numel == 0) continue;
+        if (l[i].a == nullptr || l[i].b == nullptr)
+            return fail(QF_ERR_INVALID_ARG, "tensor %d: adapter a / b is NULL", i);
+        if (!aligned16(l[i].a)) return fail(QF_ERR_ALIGN, "tensor %d: adapter a not 16-byte aligned", i);
+        if ((reinterpret_cast<uintptr_t>(l[i].b) & 1u) != 0)
+            return fail(QF_ERR_ALIGN, "tensor %d: adapter b not 2-byte aligned", i);
+        if (need_output && !t[i].y && !t[i].codes && !t[i].scales)
+            return fail(QF_ERR_INVALID_ARG, "tensor %d: no output", i);
+        if (!aligned16(t[i].y) || !aligned16(t[i].codes))
+            return fail(QF_ERR_ALIGN, "tensor %d: y / codes not 16-byte aligned", i);
+        qf::LoraTensor d{};
+        d.w = static_cast<const uint16_t*>(t[i].x);
+        d.b = static_cast<const uint16_t*>(l[i].b);
+        d.a = static_cast<const uint16_t*>(l[i].a);
+        d.y = static_cast<uint16_t*>(t[i].y);
+        d.codes = static_cast<uint8_t*>(t[i].codes);
+        d.scales = static_cast<uint8_t*>(t[i].scales);
+        d.rows = t[i].rows;
+        d.cols = t[i].cols;
+        d.col_groups = (t[i].cols + qf::kLoraCols - 1) / qf::kLoraCols;
+        d.rank = l[i].rank;
+        d.scale = l[i].scale;
+        d.group = check_group ? t[i].group : 0;
+        *max_rank = std::max(*max_rank, (int)l[i].rank);
+        out->push_back(d);
+    }
+    return QF_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+qf_status qf_lora_merge(const qf_tensor* t, const qf_lora* l, int n, void* stream) {
+    g_err[0] = 0;
+    std::vector<qf::LoraTensor> v;
+    int max_rank;
+    qf_status st = lora_tensors(t, l, n, 16, 0, false, false, &v, &max_rank);
+    if (st != QF_OK) return st;
+    for (int i = 0; i < n; ++i)
+        if (t[i].rows * t[i].cols > 0 && t[i].y == nullptr)
+            return fail(QF_ERR_INVALID_ARG, "tensor %d: y (the merged output) is NULL", i);
+    if (v.empty()) return QF_OK;
+    return lora_launch<qf::kLoraMerge>(v, max_rank, nullptr, nullptr, 0,
+                                       static_cast<cudaStream_t>(stream));
+}
+
+qf_status qf_amax_tied_lora(const qf_tensor* t, const qf_lora* l, int n, float* d_group_amax,
+                            int n_groups, void* stream) {
+    g_err[0] = 0;
+    if (n_groups <= 0) return fail(QF_ERR_INVALID_ARG, "n_groups = %d <= 0", n_groups);
+    if (d_group_amax == nullptr) return fail(QF_ERR_INVALID_ARG, "d_group_amax is NULL");
+    std::vector<qf::LoraTensor> v;
+    int max_rank;
+    qf_status st = lora_tensors(t, l, n, 16, n_groups, true, false, &v, &max_rank);
+    if (st != QF_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(d_group_amax, 0, sizeof(float) * (size_t)n_groups, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+    if (v.empty()) return QF_OK;
+    return lora_launch<qf::kLoraAmax>(v, max_rank, d_group_amax, nullptr, n_groups, s);
+}
+
+qf_status qf_fakequant_lora(qf_format f, const qf_tensor* t, const qf_lora* l, int n,
+                            const float* d_group_amax, int n_groups, float* d_group_scale_out,
+                            void* stream) {
+    g_err[0] = 0;
+    if (f != QF_NVFP4 && f != QF_MXFP4)
+        return fail(QF_ERR_UNSUPPORTED, "qf_fakequant_lora fuses NVFP4 and MXFP4 (got %d)", (int)f);
+    const bool nv = f == QF_NVFP4;
+    if (nv && (n_groups <= 0 || d_group_amax == nullptr))
+        return fail(QF_ERR_INVALID_ARG, "NVFP4 needs d_group_amax and n_groups > 0");
+    std::vector<qf::LoraTensor> v;
+    int max_rank;
+    qf_status st = lora_tensors(t, l, n, nv ? 16 : 32, n_groups, nv, true, &v, &max_rank);
+    if (st != QF_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    float* so = nv ? d_group_scale_out : nullptr;
+    if (v.empty() && !so) return QF_OK;
+    if (v.empty()) {
+        // nothing to quantize; still report the tensor scales
+        qf::LoraTensor none{};
+        none.rows = 0;
+        none.cols = 16;
+        none.col_groups = 1;
+        none.rank = 1;
+        v.push_back(none);
+    }
+    if (nv) return lora_launch<qf::kLoraNV>(v, max_rank, d_group_amax, so, n_groups, s);
+    return lora_launch<qf::kLoraMX>(v, max_rank, nullptr, nullptr, 0, s);
+}
+
 
 qf_status qf_amax_tied(const qf_tensor* t, int n, float* d_group_amax, int n_groups,
                        float* d_tracked, void* stream) {
@@ -370,6 +527,6 @@ const char* qf_status_string(qf_status s) {
 
 const char* qf_last_error(void) { return g_err; }
 
-int qf_version(void) { return (1 << 16) | 1; }
+int qf_version(void) { return (1 << 16) | 2; }
 
 }  // extern "C"

@@ -1,0 +1,237 @@
+// qf_lora.cuh -- LoRA-merged fake-quant on sm_100a (QATFactory project page, Method,
+// "QAD": LoRA-QAD trains low-rank adapters on a frozen BF16 base and quantizes
+// the merged weight W + scale * B A rather than W).
+//
+// The merged weight is formed on the fly and never written unless asked for:
+//   acc = sum over k = 0..r-1, in increasing k, of B[i,k] * A[k,j]   (FP32)
+//   M   = BF16(W[i,j] + scale * acc)
+// A BF16 x BF16 product has at most 16 significant bits, so it is exact in FP32
+// and one FMA per term rounds exactly like the separate multiply and add; the
+// fixed order makes the result reproducible bit for bit (tensor cores are not
+// used because their accumulation order is not specified).
+//
+// Layout: lane l owns 4 consecutive columns, a warp a 128-column slab, a CTA 8
+// slabs (1024 columns) by kLoraRows rows.  The warp keeps its A slab (r x 4 FP32)
+// in registers across the CTA's rows; the CTA stages its kLoraRows rows of B in
+// shared memory as FP32, so every B read is a broadcast.  W, y and codes accesses
+// are contiguous 256-, 256- and 64-byte warp runs per row.
+#pragma once
+
+#include "qf_device.cuh"
+
+namespace qf {
+
+constexpr int kLoraRows = 32;      // rows per CTA unit
+constexpr int kLoraCols = 1024;    // columns per CTA unit (8 warps x 128)
+constexpr int kLoraThreads = 256;
+
+enum LoraMode { kLoraNV = 0, kLoraMX = 1, kLoraMerge = 2, kLoraAmax = 3 };
+
+struct LoraTensor {
+    const uint16_t* w;      // BF16 base [rows, cols]
+    const uint16_t* b;      // BF16 [rows, rank]
+    const uint16_t* a;      // BF16 [rank, cols]
+    uint16_t* y;            // BF16 dequant (NV/MX) or merged weight (merge mode); nullable
+    uint8_t* codes;         // packed E2M1 nibbles (nullable)
+    uint8_t* scales;        // E4M3 / E8M0 bytes (nullable)
+    int64_t rows, cols;
+    int64_t unit_begin;     // first CTA unit of this tensor
+    int64_t col_groups;     // ceil(cols / kLoraCols)
+    int32_t rank;
+    float scale;
+    int32_t group;          // NVFP4 tie group
+    int32_t pad;
+};
+
+template <int MAXT>
+struct LoraTable {
+    LoraTensor t[MAXT];
+    int64_t total_units;
+    const float* group_amax;    // NVFP4: tie-group amax (read); amax mode: output
+    float* group_scale_out;     // NVFP4 s_t per group (nullable)
+    int32_t n;
+    int32_t n_groups;
+};
+
+template <int MAXT>
+__device__ __forceinline__ int lora_locate(const LoraTable<MAXT>& P, int64_t u) {
+    int lo = 0, hi = P.n - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (P.t[mid].unit_begin <= u) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
+__device__ __forceinline__ float bf16_round(float v) {
+    return __uint_as_float(cvt_bf16x2(0.0f, v) << 16);
+}
+
+// R: compile-time rank capacity (the runtime rank is <= R; A and B are zero-padded,
+// which adds exact zeros to an accumulator that is never -0, so results do not change).
+template <int MODE, int R, int MAXT>
+__global__ void __launch_bounds__(kLoraThreads) k_lora(const __grid_constant__ LoraTable<MAXT> P) {
+    __shared__ __align__(16) float bsm[kLoraRows][R];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int64_t cu = blockIdx.x;
+    if (MODE != kLoraAmax && cu == 0 && P.group_scale_out) {
+        for (int g = threadIdx.x; g < P.n_groups; g += kLoraThreads)
+            P.group_scale_out[g] = nv_tensor_scale(P.group_amax[g]);
+    }
+    if (cu >= P.total_units) return;
+    const LoraTensor& T = P.t[lora_locate(P, cu)];
+    const int64_t local = cu - T.unit_begin;
+    const int64_t r0 = (local / T.col_groups) * kLoraRows;
+    const int64_t c_base = (local % T.col_groups) * kLoraCols;
+    const int64_t rows_left = T.rows - r0;
+    const int nrows = rows_left < kLoraRows ? (int)rows_left : kLoraRows;
+    const int64_t col0 = c_base + wid * 128 + lane * 4;
+    const bool colok = col0 < T.cols;          // cols % 16 == 0: a lane is all in or all out
+    const int rank = T.rank;
+
+    // this CTA's rows of B as FP32, zero-padded to R
+    for (int idx = threadIdx.x; idx < kLoraRows * R; idx += kLoraThreads) {
+        const int i = idx / R, k = idx % R;
+        bsm[i][k] = (i < nrows && k < rank) ? bf16_lo(T.b[(r0 + i) * rank + k]) : 0.0f;
+    }
+    // this lane's 4 columns of A as FP32, zero-padded to R
+    float a[R][4];
+#pragma unroll
+    for (int k = 0; k < R; ++k) {
+        uint2 v = make_uint2(0, 0);
+        if (k < rank && colok) v = *reinterpret_cast<const uint2*>(T.a + k * T.cols + col0);
+        a[k][0] = bf16_lo(v.x); a[k][1] = bf16_hi(v.x);
+        a[k][2] = bf16_lo(v.y); a[k][3] = bf16_hi(v.y);
+    }
+    __syncthreads();
+
+    float s_t = 0.0f, six_st = 0.0f;
+    if (MODE == kLoraNV) {
+        s_t = nv_tensor_scale(P.group_amax[T.group]);
+        six_st = __fmul_rn(6.0f, s_t);
+    }
+    uint32_t run = 0;                          // amax mode: running max |M| (FP32 bits)
+
+    auto load_w = [&](int i0, uint2 (&wv)[4]) {
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            const bool ok = colok && i0 + h < nrows;
+            wv[h] = ok ? *reinterpret_cast<const uint2*>(T.w + (r0 + i0 + h) * T.cols + col0)
+                       : make_uint2(0, 0);
+        }
+    };
+    uint2 wcur[4], wnxt[4];
+    load_w(0, wcur);
+    for (int i0 = 0; i0 < nrows; i0 += 4) {
+        if (i0 + 4 < nrows) load_w(i0 + 4, wnxt);          // the next 4 rows, in flight meanwhile
+        // merged values of 4 rows x this lane's 4 columns
+        float x[4][4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            const int i = min(i0 + h, nrows - 1);            // rows past the end are not stored
+            float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+            for (int k = 0; k < R; k += 4) {
+                const float4 bk = *reinterpret_cast<const float4*>(&bsm[i][k]);
+                const float bb[4] = {bk.x, bk.y, bk.z, bk.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) acc[c] = __fmaf_rn(bb[q], a[k + q][c], acc[c]);
+            }
+            const float wf[4] = {bf16_lo(wcur[h].x), bf16_hi(wcur[h].x), bf16_lo(wcur[h].y),
+                                 bf16_hi(wcur[h].y)};
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                x[h][c] = bf16_round(__fadd_rn(wf[c], __fmul_rn(T.scale, acc[c])));
+        }
+        if (MODE == kLoraMerge) {
+#pragma unroll
+            for (int h = 0; h < 4; ++h)
+                if (colok && i0 + h < nrows && T.y)
+                    *reinterpret_cast<uint2*>(T.y + (r0 + i0 + h) * T.cols + col0) =
+                        make_uint2(cvt_bf16x2(x[h][1], x[h][0]), cvt_bf16x2(x[h][3], x[h][2]));
+        } else {
+            uint32_t m[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                m[h] = 0;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) m[h] = max(m[h], __float_as_uint(x[h][c]) & 0x7FFFFFFFu);
+            }
+            if (MODE == kLoraAmax) {
+#pragma unroll
+                for (int h = 0; h < 4; ++h)
+                    if (i0 + h < nrows) run = max(run, m[h]);
+            } else {
+                // block max over the 4 (NVFP4, 16 elements) or 8 (MXFP4, 32) lanes of the block
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    m[h] = max(m[h], __shfl_xor_sync(kFull, m[h], 1));
+                    m[h] = max(m[h], __shfl_xor_sync(kFull, m[h], 2));
+                    if (MODE == kLoraMX) m[h] = max(m[h], __shfl_xor_sync(kFull, m[h], 4));
+                }
+                float S[4], inv[4];
+                uint32_t sbyte[4];
+                if (MODE == kLoraNV) {
+                    // the 4 lanes of a block each derive one of the 4 rows' scales, then share
+                    const int t = lane & 3;
+                    const uint32_t mt = t == 0 ? m[0] : t == 1 ? m[1] : t == 2 ? m[2] : m[3];
+                    uint32_t sb_t;
+                    float S_t, inv_t;
+                    nv_block_scale(__uint_as_float(mt), s_t, six_st, sb_t, S_t, inv_t);
+                    const int base = lane & ~3;
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        sbyte[h] = __shfl_sync(kFull, sb_t, base + h);
+                        S[h] = __shfl_sync(kFull, S_t, base + h);
+                        inv[h] = __shfl_sync(kFull, inv_t, base + h);
+                    }
+                } else {
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        const uint32_t E = m[h] >> 23;
+                        sbyte[h] = E > 2u ? E - 2u : 0u;
+                        inv[h] = __uint_as_float((254u - sbyte[h]) << 23);
+                        S[h] = sbyte[h] ? __uint_as_float(sbyte[h] << 23) : __uint_as_float(0x00200000u);
+                    }
+                }
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    float q[4];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) q[c] = __fmul_rn(x[h][c], inv[h]);
+                    if (MODE == kLoraNV && __builtin_expect(isinf(inv[h]), 0)) {
+#pragma unroll
+                        for (int c = 0; c < 4; ++c)
+                            if (x[h][c] == 0.0f) q[c] = x[h][c];
+                    }
+                    const uint32_t b0 = cvt_e2m1x2(q[1], q[0]), b1 = cvt_e2m1x2(q[3], q[2]);
+                    if (!colok || i0 + h >= nrows) continue;
+                    const int64_t e = (r0 + i0 + h) * T.cols + col0;   // flat element index
+                    if (T.y) {
+                        const uint32_t h0 = cvt_e2m1x2_f16x2(b0), h1 = cvt_e2m1x2_f16x2(b1);
+                        *reinterpret_cast<uint2*>(T.y + e) = make_uint2(
+                            cvt_bf16x2(__fmul_rn(f16_hi(h0), S[h]), __fmul_rn(f16_lo(h0), S[h])),
+                            cvt_bf16x2(__fmul_rn(f16_hi(h1), S[h]), __fmul_rn(f16_lo(h1), S[h])));
+                    }
+                    if (T.codes)
+                        *reinterpret_cast<uint16_t*>(T.codes + (e >> 1)) = (uint16_t)(b0 | (b1 << 8));
+                    if (T.scales && (lane & (MODE == kLoraNV ? 3 : 7)) == 0)
+                        T.scales[e >> (MODE == kLoraNV ? 4 : 5)] = (uint8_t)sbyte[h];
+                }
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < 4; ++h) wcur[h] = wnxt[h];
+    }
+    if (MODE == kLoraAmax) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) run = max(run, __shfl_xor_sync(kFull, run, o));
+        if (lane == 0 && run != 0)
+            atomicMax(reinterpret_cast<unsigned int*>(const_cast<float*>(P.group_amax)) + T.group, run);
+    }
+}
+
+}  // namespace qf

@@ -202,6 +202,48 @@ qf_status qf_ste_backward(qf_format f, const void* grad_y, void* grad_x, int64_t
                           int mode, const qf_tensor* fwd, const float* d_group_amax,
                           int n_groups, void* stream);
 
+/*
+ * LoRA adapters (project page, Method, "QAD": LoRA-QAD trains low-rank adapters
+ * on a frozen BF16 base and quantizes the merged weight, not the base).
+ * For tensor t with base W = t.x (BF16 [rows, cols]):
+ *   acc = sum over k = 0..rank-1, in increasing k, of b[i,k] * a[k,j]   (FP32; each
+ *         BF16 x BF16 product is exact in FP32, each sum is rounded)
+ *   M   = BF16( W[i,j] + scale * acc )      (an FP32 multiply, an FP32 add, RNE)
+ * M is the merged weight a BF16 model holds after merging the adapter.
+ *   b       BF16 [rows, rank] row-major (device)
+ *   a       BF16 [rank, cols] row-major (device), 16-byte aligned
+ *   rank    1 .. QF_LORA_MAX_RANK
+ *   scale   FP32 multiplier of B A (alpha / rank in the usual parameterisation)
+ */
+#define QF_LORA_MAX_RANK 32
+typedef struct qf_lora {
+    const void* b;
+    const void* a;
+    int32_t rank;
+    float scale;
+} qf_lora;
+
+/*
+ * qf_lora_merge -- writes the merged weight M of each tensor to t[i].y (BF16
+ * [rows, cols]); codes and scales are ignored.  Use it to feed qf_fakequant with
+ * formats qf_fakequant_lora does not fuse (Q4_K).
+ * qf_amax_tied_lora -- qf_amax_tied of the merged weights (NVFP4 tie groups).
+ * qf_fakequant_lora -- qf_fakequant of the merged weights, NVFP4 or MXFP4, with the
+ *   merge formed on the fly (M is never written): bitwise the same outputs as
+ *   qf_lora_merge followed by qf_fakequant.
+ * All three: t[i].x_type must be QF_X_BF16; cols a multiple of 16 (MXFP4: 32);
+ * l[i] is the adapter of t[i].  Errors as for the calls without LoRA, plus
+ * QF_ERR_INVALID_ARG for a NULL adapter pointer or a rank outside
+ * [1, QF_LORA_MAX_RANK], QF_ERR_UNSUPPORTED for FP32 bases or (qf_fakequant_lora)
+ * the Q4_K format.
+ */
+qf_status qf_lora_merge(const qf_tensor* t, const qf_lora* l, int n, void* stream);
+qf_status qf_amax_tied_lora(const qf_tensor* t, const qf_lora* l, int n, float* d_group_amax,
+                            int n_groups, void* stream);
+qf_status qf_fakequant_lora(qf_format f, const qf_tensor* t, const qf_lora* l, int n,
+                            const float* d_group_amax, int n_groups, float* d_group_scale_out,
+                            void* stream);
+
 /* Static description of a status code. */
 const char* qf_status_string(qf_status s);
 
@@ -209,7 +251,7 @@ const char* qf_status_string(qf_status s);
 const char* qf_last_error(void);
 
 /* ABI version: (major << 16) | minor.  1.1 added qf_tensor.x_type (formerly a
- * reserved field that had to be 0, which still means BF16). */
+ * reserved field that had to be 0, which still means BF16); 1.2 the LoRA calls. */
 int qf_version(void);
 
 #ifdef __cplusplus

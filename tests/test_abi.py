@@ -58,7 +58,7 @@ def test_struct_layout_matches_header(qf):
 def test_status_strings(qf):
     for s in range(6):
         assert qf.lib.qf_status_string(s).decode().startswith("QF_")
-    assert qf.lib.qf_version() == (1 << 16) | 1
+    assert qf.lib.qf_version() == (1 << 16) | 2
 
 
 def _tensor(qf, x=0x1000, rows=4, cols=64, group=0, y=0x2000, codes=0x3000, scales=0x4000,
@@ -145,3 +145,28 @@ def test_product_path_has_no_oracle_dependency():
     out = subprocess.run(["ldd", os.path.join(pkg, "libqf.so")], capture_output=True,
                          text=True).stdout
     assert "oracle" not in out
+
+
+def test_lora_validation(qf):
+    INV, SHAPE, ALIGN, UNSUP = 1, 2, 3, 4
+    lib = qf.lib
+    L = qf.binding.QfLora
+    def lora(b=0x5000, a=0x6000, rank=16, scale=1.0):
+        arr = (L * 1)()
+        arr[0].b, arr[0].a, arr[0].rank, arr[0].scale = b, a, rank, scale
+        return arr
+    t = _tensor(qf, cols=64)
+    assert lib.qf_fakequant_lora(2, t, lora(), 1, None, 0, None, None) == UNSUP     # Q4_K not fused
+    assert lib.qf_fakequant_lora(1, t, lora(rank=0), 1, None, 0, None, None) == INV
+    assert lib.qf_fakequant_lora(1, t, lora(rank=33), 1, None, 0, None, None) == INV
+    assert lib.qf_fakequant_lora(1, t, lora(a=0), 1, None, 0, None, None) == INV
+    assert lib.qf_fakequant_lora(1, t, lora(a=0x6008), 1, None, 0, None, None) == ALIGN
+    assert lib.qf_fakequant_lora(1, t, lora(b=0x5001), 1, None, 0, None, None) == ALIGN
+    assert lib.qf_fakequant_lora(1, _tensor(qf, cols=48), lora(), 1, None, 0, None, None) == SHAPE
+    assert lib.qf_fakequant_lora(1, _tensor(qf, x_type=1), lora(), 1, None, 0, None, None) == UNSUP
+    assert lib.qf_fakequant_lora(0, t, lora(), 1, None, 1, None, None) == INV           # no amax
+    assert lib.qf_fakequant_lora(1, t, None, 1, None, 0, None, None) == INV
+    assert lib.qf_lora_merge(_tensor(qf, y=0), lora(), 1, None) == INV                   # no output
+    assert lib.qf_amax_tied_lora(t, lora(), 1, None, 1, None) == INV
+    assert lib.qf_amax_tied_lora(_tensor(qf, group=3), lora(), 1, 0x7000, 2, None) == INV
+    assert lib.qf_lora_merge(_tensor(qf, rows=0), lora(), 1, None) == 0                 # empty

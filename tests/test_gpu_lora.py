@@ -1,0 +1,107 @@
+"""GPU parity of the LoRA-merged fake-quant (bit for bit against the oracle).
+
+LoRA-QAD (QATFactory project page, Method, "QAD") quantizes W + scale * B A.  The
+fused calls form the BF16 merged weight on the fly; they must equal the oracle's
+merge followed by its quantizer, and the library's own merge followed by
+qf_fakequant."""
+import numpy as np
+import pytest
+import torch
+
+import fp4_fake_quant_b200 as qf
+import oracle
+import workloads
+from gpu_helpers import DEV, assert_same, bits, u8
+
+pytestmark = pytest.mark.gpu
+
+
+def _case(rows, cols, rank, seed):
+    w = workloads.normal_with_outliers(rows, cols, 0.02, 1e-3, 20.0, seed, 0)
+    b = workloads.normal_with_outliers(rows, rank, 0.01, 0.0, 1.0, seed, 1)
+    a = workloads.normal_with_outliers(rank, cols, 0.02, 0.0, 1.0, seed, 2)
+    return w, b, a
+
+
+SHAPES = [(37, 1040, 3), (64, 2048, 8), (33, 768, 16), (40, 4096, 32), (1, 32, 1)]
+
+
+@pytest.mark.parametrize("rows,cols,rank", SHAPES)
+def test_lora_merge_and_amax(rows, cols, rank):
+    w, b, a = _case(rows, cols, rank, rows + rank)
+    scale = 32.0 / rank
+    want = oracle.lora_merge(w, b, a, scale)
+    m = torch.empty(rows, cols, dtype=torch.bfloat16, device=DEV)
+    adapters = [(b.to(DEV), a.to(DEV), scale)]
+    qf.qf_lora_merge([w.to(DEV)], adapters, [m])
+    amax = torch.empty(1, device=DEV)
+    qf.qf_amax_tied_lora([w.to(DEV)], adapters, [0], amax)
+    torch.cuda.synchronize()
+    assert_same("merged", bits(m), want)
+    assert_same("merged amax", amax.cpu().numpy().view(np.uint32),
+                np.float32([oracle.amax(want)]).view(np.uint32))
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4"])
+@pytest.mark.parametrize("rows,cols,rank", SHAPES)
+def test_lora_fakequant_equals_merge_then_quantize(fmt, rows, cols, rank):
+    if fmt == "mxfp4" and cols % 32:
+        pytest.skip("MXFP4 needs 32 | cols")
+    w, b, a = _case(rows, cols, rank, 3 * rows + rank)
+    scale = 16.0 / rank
+    merged = oracle.lora_merge(w, b, a, scale)
+    am = oracle.amax(merged)
+    if fmt == "nvfp4":
+        y, c, s, _ = oracle.nvfp4(merged, am)
+    else:
+        y, c, s = oracle.mxfp4(merged)
+    wd = w.to(DEV)
+    adapters = [(b.to(DEV), a.to(DEV), scale)]
+    yo, co, so = qf.alloc_outputs(fmt, wd)
+    amax = torch.empty(1, device=DEV)
+    kw = {}
+    if fmt == "nvfp4":
+        qf.qf_amax_tied_lora([wd], adapters, [0], amax)
+        kw = {"groups": [0], "group_amax": amax}
+    qf.qf_fakequant_lora(fmt, [wd], adapters, [yo], [co], [so], **kw)
+    torch.cuda.synchronize()
+    assert_same("lora y", bits(yo), y)
+    assert_same("lora codes", u8(co), c)
+    assert_same("lora scales", u8(so), s)
+    # the library's own merge followed by qf_fakequant gives the same bytes
+    m = torch.empty_like(wd)
+    qf.qf_lora_merge([wd], adapters, [m])
+    y2, c2, s2 = qf.alloc_outputs(fmt, wd)
+    qf.qf_fakequant(fmt, [m], [y2], [c2], [s2], **kw)
+    torch.cuda.synchronize()
+    assert torch.equal(y2, yo) and torch.equal(c2, co) and torch.equal(s2, so)
+
+
+def test_lora_grouped_experts_with_tied_groups():
+    """Several adapted tensors in one launch (gate/up tied, down its own group)."""
+    ts, ads, groups, merged = [], [], [], []
+    for e in range(3):
+        for j, (r, c) in enumerate([(96, 2048), (96, 2048), (256, 768)]):
+            w, b, a = _case(r, c, 16, 100 + 3 * e + j)
+            ts.append(w)
+            ads.append((b, a, 2.0))
+            groups.append(2 * e + (j == 2))
+            merged.append(oracle.lora_merge(w, b, a, 2.0))
+    am = np.zeros(6, np.float32)
+    for m, g in zip(merged, groups):
+        am[g] = max(am[g], np.float32(oracle.amax(m)))
+    xs = [t.to(DEV) for t in ts]
+    adapters = [(b.to(DEV), a.to(DEV), s) for b, a, s in ads]
+    amax = torch.empty(6, device=DEV)
+    qf.qf_amax_tied_lora(xs, adapters, groups, amax)
+    outs = [qf.alloc_outputs("nvfp4", x) for x in xs]
+    so = torch.empty(6, device=DEV)
+    qf.qf_fakequant_lora("nvfp4", xs, adapters, [o[0] for o in outs], [o[1] for o in outs],
+                         [o[2] for o in outs], groups, amax, so)
+    torch.cuda.synchronize()
+    assert_same("grouped lora amax", amax.cpu().numpy().view(np.uint32), am.view(np.uint32))
+    for i, m in enumerate(merged):
+        y, c, s, _ = oracle.nvfp4(m, am[groups[i]])
+        assert_same(f"grouped lora y {i}", bits(outs[i][0]), y)
+        assert_same(f"grouped lora codes {i}", u8(outs[i][1]), c)
+        assert_same(f"grouped lora scales {i}", u8(outs[i][2]), s)
