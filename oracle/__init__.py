@@ -42,6 +42,8 @@ PARITY = {
     "nvfp4_quant": "on-grid round trip, symmetry, block locality, brute-force nearest code, decoder",
     "mxfp4_quant": "on-grid round trip, idempotence, symmetry, brute-force nearest code, decoder",
     "q4k_quant": "on-grid round trip, brute-force nearest q, decoder, error bound",
+    "q4k_quant (mse fit)": "grid membership + float64 least error over the grid, never worse than "
+                           "min/max, on-grid equal to min/max, decoder, lower total error",
     "ste_backward": "identity copy; clipped mask vs brute-force saturation",
     "lora_merge": "exact integer-grid merges vs numpy; zero adapter / zero scale give W; "
                   "float64 reference within one BF16 step; row/column locality",
@@ -86,6 +88,9 @@ def _load():
             "qfo_mxfp4_quant_x": (None, [P, ctypes.c_int, I64, I64, P, P, P]),
             "qfo_q4k_quant_x": (None, [P, ctypes.c_int, I64, I64, P, P]),
             "qfo_q4k_fit_one_x": (None, [P, ctypes.c_int, P, P, P, P, P]),
+            "qfo_q4k_quant_fit": (None, [P, ctypes.c_int, ctypes.c_int, I64, I64, P, P]),
+            "qfo_q4k_fit_one_fit": (None, [P, ctypes.c_int, ctypes.c_int, P, P, P, P, P]),
+            "qfo_q4k_search_scale_one": (F, [P, F, F]),
             "qfo_ste_backward_x": (None, [P, P, I64, ctypes.c_int, ctypes.c_int, P, ctypes.c_int,
                                           I64, F]),
             "qfo_nvfp4_tensor_scale": (F, [F]),
@@ -256,19 +261,20 @@ def mxfp4(x, rows: int | None = None, cols: int | None = None):
     return y, codes, scales
 
 
-def q4k(x, rows: int | None = None, cols: int | None = None):
-    """Q4_K quantize-dequantize + pack.  Returns (y_bits, blocks[n/256, 144])."""
+def q4k(x, rows: int | None = None, cols: int | None = None, mse: bool = False):
+    """Q4_K quantize-dequantize + pack (min/max fit, or the MSE-searched fit).
+    Returns (y_bits, blocks[n/256, 144])."""
     xb, xt = _xin(x)
     if rows is None:
         rows, cols = xb.shape
     n = rows * cols
     y = np.empty(n, np.uint16)
     blocks = np.empty((n // 256) * 144, np.uint8)
-    _load().qfo_q4k_quant_x(_ptr(xb), xt, rows, cols, _ptr(y), _ptr(blocks))
+    _load().qfo_q4k_quant_fit(_ptr(xb), xt, int(mse), rows, cols, _ptr(y), _ptr(blocks))
     return y, blocks
 
 
-def q4k_fit_one(x256: np.ndarray):
+def q4k_fit_one(x256: np.ndarray, mse: bool = False):
     """Unpacked fit of one super-block: (d_bits, dmin_bits, sc[8], m[8], q[256])."""
     xb, xt = _xin(x256)
     xb = xb.reshape(-1)
@@ -278,9 +284,16 @@ def q4k_fit_one(x256: np.ndarray):
     sc = np.empty(8, np.uint8)
     m = np.empty(8, np.uint8)
     q = np.empty(256, np.uint8)
-    _load().qfo_q4k_fit_one_x(_ptr(xb), xt, ctypes.byref(d), ctypes.byref(dm), _ptr(sc), _ptr(m),
-                              _ptr(q))
+    _load().qfo_q4k_fit_one_fit(_ptr(xb), xt, int(mse), ctypes.byref(d), ctypes.byref(dm),
+                                _ptr(sc), _ptr(m), _ptr(q))
     return int(d.value), int(dm.value), sc, m, q
+
+
+def q4k_search_scale(v32: np.ndarray, hi: float, min_j: float) -> float:
+    """The MSE-searched scale of one 32-element sub-block (values as FP32)."""
+    v = np.ascontiguousarray(v32, dtype=np.float32)
+    assert v.size == 32
+    return float(_load().qfo_q4k_search_scale_one(_ptr(v), float(hi), float(min_j)))
 
 
 def nvfp4_decode(codes, scales, s_t: float, numel: int) -> np.ndarray:
@@ -316,7 +329,7 @@ def lora_merge(w, b, a, scale: float) -> np.ndarray:
     return m
 
 
-FORMATS = {"nvfp4": 0, "mxfp4": 1, "q4k": 2}
+FORMATS = {"nvfp4": 0, "mxfp4": 1, "q4k": 2, "q4k_mse": 3}
 
 
 def ste_backward(grad_y, mode: int = 0, fmt: str = "nvfp4", x=None, amax_g: float = 0.0):

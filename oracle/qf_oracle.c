@@ -367,7 +367,56 @@ typedef struct {
     uint8_t q[256];              /* 4-bit values */
 } q4k_super;
 
-static void q4k_fit(const void* x, int xt, q4k_super* o, uint16_t* y)
+/* ------------------------------------------------------------------------ */
+/* MSE-searched sub-block scale (the project page's "Key findings" name an   */
+/* MSE-optimal quantizer as the Q4_K PTQ baseline without giving its steps;  */
+/* this is a plain reading of "search the scale for least squared error").   */
+/* With the sub-block's offset min_j fixed, the scale is searched over the   */
+/* step counts n of the grid below -- 15 first (the min/max fit), then the   */
+/* others in the listed order -- as scale = (hi + min_j) / n, and the one     */
+/* with the smallest squared dequantization error                            */
+/*   err = sum over i, in order, of (x_i - (scale*q_i - min_j))^2,           */
+/*   q_i = clamp(RNE((x_i + min_j) * (1/scale)), 0, 15)                      */
+/* is kept (a later candidate must be strictly smaller).  Everything is       */
+/* binary32 with one rounding per operation.                                 */
+/* ------------------------------------------------------------------------ */
+static const float kQ4kSearch[9] = {15.0f, 14.0f, 14.5f, 15.5f, 16.0f, 16.5f, 17.0f, 17.5f, 18.0f};
+
+static float q4k_sub_err(const float* v, float scale, float min_j)
+{
+    float inv = 1.0f / scale;
+    float err = 0.0f;
+    for (int i = 0; i < 32; ++i) {
+        float q = nearbyintf((v[i] + min_j) * inv);
+        if (q < 0.0f) q = 0.0f;
+        if (q > 15.0f) q = 15.0f;
+        float deq = scale * q - min_j;
+        float r = v[i] - deq;
+        err = err + r * r;
+    }
+    return err;
+}
+
+static float q4k_search_scale(const float* v, float hi, float min_j)
+{
+    float range = hi + min_j;
+    float best = range / kQ4kSearch[0];
+    if (best == 0.0f) return best;
+    float best_err = q4k_sub_err(v, best, min_j);
+    for (int t = 1; t < 9; ++t) {
+        float scale = range / kQ4kSearch[t];
+        float err = q4k_sub_err(v, scale, min_j);
+        if (err < best_err) { best_err = err; best = scale; }
+    }
+    return best;
+}
+
+float qfo_q4k_search_scale_one(const float* v, float hi, float min_j)
+{
+    return q4k_search_scale(v, hi, min_j);
+}
+
+static void q4k_fit(const void* x, int xt, int mse, q4k_super* o, uint16_t* y)
 {
     float scale[8], minv[8];
     for (int j = 0; j < 8; ++j) {
@@ -378,7 +427,13 @@ static void q4k_fit(const void* x, int xt, q4k_super* o, uint16_t* y)
             if (v > hi) hi = v;
         }
         minv[j] = (mn < 0.0f) ? -mn : 0.0f;
-        scale[j] = (hi + minv[j]) / 15.0f;
+        if (mse) {
+            float vals[32];
+            for (int i = 0; i < 32; ++i) vals[i] = xval(x, xt, 32 * j + i);
+            scale[j] = q4k_search_scale(vals, hi, minv[j]);
+        } else {
+            scale[j] = (hi + minv[j]) / 15.0f;
+        }
     }
     float max_scale = 0.0f, max_min = 0.0f;
     for (int j = 0; j < 8; ++j) {
@@ -446,25 +501,38 @@ static void q4k_pack(const q4k_super* o, uint8_t* blk)
 
 /* Q4_K quantize-dequantize + pack of one [rows, cols] matrix, cols % 256 == 0.
  * y: [rows*cols] BF16 (may be NULL); blocks: [rows*cols/256] x 144 bytes (may be NULL). */
-void qfo_q4k_quant_x(const void* x, int xt, int64_t rows, int64_t cols,
-                     uint16_t* y, uint8_t* blocks)
+void qfo_q4k_quant_fit(const void* x, int xt, int mse, int64_t rows, int64_t cols,
+                       uint16_t* y, uint8_t* blocks)
 {
     q4k_super o;
     for (int64_t r = 0; r < rows; ++r) {
         for (int64_t b = 0; b < cols / 256; ++b) {
             const int64_t base = r * cols + b * 256;
-            q4k_fit(xoff(x, xt, base), xt, &o, y ? y + base : NULL);
+            q4k_fit(xoff(x, xt, base), xt, mse, &o, y ? y + base : NULL);
             if (blocks) q4k_pack(&o, blocks + (base / 256) * 144);
         }
     }
 }
 
 /* Q4_K scale/min fit of one 256-element super-block, unpacked (for pins). */
+void qfo_q4k_quant_x(const void* x, int xt, int64_t rows, int64_t cols,
+                     uint16_t* y, uint8_t* blocks)
+{ qfo_q4k_quant_fit(x, xt, 0, rows, cols, y, blocks); }
+
+void qfo_q4k_fit_one_fit(const void* x, int xt, int mse, uint16_t* d, uint16_t* dmin,
+                         uint8_t* sc, uint8_t* m, uint8_t* q)
+{
+    q4k_super o;
+    q4k_fit(x, xt, mse, &o, NULL);
+    *d = o.d; *dmin = o.dmin;
+    memcpy(sc, o.sc, 8); memcpy(m, o.m, 8); memcpy(q, o.q, 256);
+}
+
 void qfo_q4k_fit_one_x(const void* x, int xt, uint16_t* d, uint16_t* dmin, uint8_t* sc,
                        uint8_t* m, uint8_t* q)
 {
     q4k_super o;
-    q4k_fit(x, xt, &o, NULL);
+    q4k_fit(x, xt, 0, &o, NULL);
     *d = o.d; *dmin = o.dmin;
     memcpy(sc, o.sc, 8); memcpy(m, o.m, 8); memcpy(q, o.q, 256);
 }
@@ -535,6 +603,7 @@ void qfo_q4k_decode(const uint8_t* blocks, int64_t numel, uint16_t* y)
 void qfo_ste_backward_x(const uint16_t* grad_y, uint16_t* grad_x, int64_t numel, int mode,
                         int fmt, const void* x, int xt, int64_t cols, float amax_g)
 {
+    /* fmt: 0 NVFP4, 1 MXFP4, 2 Q4_K (min/max fit), 3 Q4_K (MSE-searched fit) */
     if (mode == 0) { for (int64_t i = 0; i < numel; ++i) grad_x[i] = grad_y[i]; return; }
     int64_t rows = cols ? numel / cols : 0;
     if (fmt == 0) {
@@ -558,7 +627,7 @@ void qfo_ste_backward_x(const uint16_t* grad_y, uint16_t* grad_x, int64_t numel,
     } else {
         q4k_super o;
         for (int64_t base = 0; base < rows * cols; base += 256) {
-            q4k_fit(xoff(x, xt, base), xt, &o, NULL);
+            q4k_fit(xoff(x, xt, base), xt, fmt == 3, &o, NULL);
             float d = qfo_f16_to_f32(o.d), dmin = qfo_f16_to_f32(o.dmin);
             for (int j = 0; j < 8; ++j) {
                 float s = d * (float)o.sc[j], mm = dmin * (float)o.m[j];
