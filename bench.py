@@ -47,9 +47,9 @@ import workloads  # noqa: E402
 METRIC = "fake-quant+pack GB/s and Gelem/s per format; % of B200 HBM roofline"
 UNIT = "GB/s"
 BYTES_PER_ELEM = {"nvfp4": 2 + 2 + 0.5 + 1 / 16, "mxfp4": 2 + 2 + 0.5 + 1 / 32,
-                  "q4k": 2 + 2 + 144 / 256}
+                  "q4k": 2 + 2 + 144 / 256, "q4k_mse": 2 + 2 + 144 / 256}
 WORKLOADS = ("w4a4", "nvfp4_tied", "q4k", "nvfp4_weight", "activation", "moe_nvfp4",
-             "moe_mxfp4", "moe_q4k", "nvfp4_tied_f32", "q4k_f32", "lora_nvfp4")
+             "moe_mxfp4", "moe_q4k", "nvfp4_tied_f32", "q4k_f32", "lora_nvfp4", "q4k_mse")
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -167,6 +167,10 @@ def make_workload(name: str, qf, dev, seed_shift: int = 0):
         wl, fmt = workloads.q4k_weights(seed=2 + seed_shift), "q4k"
         desc = ("Q4_K weight-only: down 4096x14336 + up 14336x4096, N(0,0.015) x per-row "
                 "log-uniform[0.5,2]; one grouped fake-quant+pack launch (144-byte blocks)")
+    elif name == "q4k_mse":
+        wl, fmt = workloads.q4k_weights(seed=2 + seed_shift), "q4k_mse"
+        desc = ("Q4_K with the MSE-searched scale fit (9 trial scales per sub-block): down "
+                "4096x14336 + up 14336x4096; one grouped launch (the PTQ-baseline quantizer)")
     elif name == "q4k_f32":
         wl, fmt = workloads.q4k_weights(seed=2 + seed_shift, dtype="f32"), "q4k"
         desc = ("Q4_K from FP32 latent weights: down 4096x14336 + up 14336x4096; one grouped "
@@ -240,7 +244,7 @@ def make_workload(name: str, qf, dev, seed_shift: int = 0):
         W["fq"] = qf.prepare_fakequant(fmt, xs, Y, C, S)
         W["step_bytes"] = W["fq_bytes"]
         W["launches"] = chunks
-        W["kernel"] = "k_fp4_mxfp4" if fmt == "mxfp4" else "k_q4k"
+        W["kernel"] = {"mxfp4": "k_fp4_mxfp4", "q4k": "k_q4k", "q4k_mse": "k_q4k_mse"}[fmt]
     return W
 
 

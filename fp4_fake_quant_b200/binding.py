@@ -17,10 +17,10 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libqf.so")
 
-QF_NVFP4, QF_MXFP4, QF_Q4K = 0, 1, 2
+QF_NVFP4, QF_MXFP4, QF_Q4K, QF_Q4K_MSE = 0, 1, 2, 3
 QF_X_BF16, QF_X_F32 = 0, 1
-FORMATS = {"nvfp4": QF_NVFP4, "mxfp4": QF_MXFP4, "q4k": QF_Q4K}
-BLOCK = {QF_NVFP4: 16, QF_MXFP4: 32, QF_Q4K: 256}
+FORMATS = {"nvfp4": QF_NVFP4, "mxfp4": QF_MXFP4, "q4k": QF_Q4K, "q4k_mse": QF_Q4K_MSE}
+BLOCK = {QF_NVFP4: 16, QF_MXFP4: 32, QF_Q4K: 256, QF_Q4K_MSE: 256}
 STATUS = {0: "QF_OK", 1: "QF_ERR_INVALID_ARG", 2: "QF_ERR_SHAPE", 3: "QF_ERR_ALIGN",
           4: "QF_ERR_UNSUPPORTED", 5: "QF_ERR_CUDA"}
 
@@ -132,7 +132,7 @@ def _desc(xs: Sequence[torch.Tensor], ys=None, codes=None, scales=None, groups=N
 def output_sizes(fmt, numel: int):
     """Bytes of (codes, scales) for one tensor of ``numel`` elements."""
     f = _fmt(fmt)
-    if f == QF_Q4K:
+    if f in (QF_Q4K, QF_Q4K_MSE):
         return (numel // 256) * 144, 0
     return numel // 2, numel // BLOCK[f]
 

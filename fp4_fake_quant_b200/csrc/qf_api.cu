@@ -41,6 +41,9 @@ qf_status cuda_fail(cudaError_t e, const char* what) {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int block_of(qf_format f) { return f == QF_NVFP4 ? 16 : f == QF_MXFP4 ? 32 : 256; }
+bool known_format(qf_format f) {
+    return f == QF_NVFP4 || f == QF_MXFP4 || f == QF_Q4K || f == QF_Q4K_MSE;
+}
 
 // Launch shape of one kernel: SM count, resident CTAs per SM, CTA size, waves.
 struct Launch { int sms; int per_sm; int threads; int waves; };
@@ -159,9 +162,9 @@ template <typename XT, int MAXT, int MODE>
 constexpr auto mx_kernel() {
     return qf::k_fp4<false, XT, kFp4U, MAXT, MODE, QF_MX_THREADS, QF_MX_PREFETCH>;
 }
-template <typename XT, int MAXT, int MODE>
+template <typename XT, int MAXT, int MODE, bool MSE>
 constexpr auto q4k_kernel() {
-    return qf::k_q4k<XT, MAXT, MODE, QF_Q4K_THREADS>;
+    return qf::k_q4k<XT, MAXT, MODE, QF_Q4K_THREADS, MSE>;
 }
 
 template <typename XT>
@@ -182,11 +185,21 @@ qf_status launch_format_t(qf_format f, int mode, const std::vector<DevTensor>& v
         return launch_chunks(mx_kernel<XT, kSmallT, 1>(), mx_kernel<XT, kLargeT, 1>(), QF_MX_THREADS,
                              QF_MX_WAVES, v, 256 * kFp4U, nullptr, nullptr, nullptr, 0, s);
     }
+    if (f == QF_Q4K_MSE) {
+        if (mode == 0)
+            return launch_chunks(q4k_kernel<XT, kSmallT, 0, true>(),
+                                 q4k_kernel<XT, kLargeT, 0, true>(), QF_Q4K_THREADS,
+                                 QF_Q4K_WAVES, v, 1024, nullptr, nullptr, nullptr, 0, s);
+        return launch_chunks(q4k_kernel<XT, kSmallT, 1, true>(), q4k_kernel<XT, kLargeT, 1, true>(),
+                             QF_Q4K_THREADS, QF_Q4K_WAVES, v, 1024, nullptr, nullptr, nullptr, 0,
+                             s);
+    }
     if (mode == 0)
-        return launch_chunks(q4k_kernel<XT, kSmallT, 0>(), q4k_kernel<XT, kLargeT, 0>(), QF_Q4K_THREADS,
-                             QF_Q4K_WAVES, v, 1024, nullptr, nullptr, nullptr, 0, s);
-    return launch_chunks(q4k_kernel<XT, kSmallT, 1>(), q4k_kernel<XT, kLargeT, 1>(), QF_Q4K_THREADS,
-                         QF_Q4K_WAVES, v, 1024, nullptr, nullptr, nullptr, 0, s);
+        return launch_chunks(q4k_kernel<XT, kSmallT, 0, false>(),
+                             q4k_kernel<XT, kLargeT, 0, false>(), QF_Q4K_THREADS, QF_Q4K_WAVES, v,
+                             1024, nullptr, nullptr, nullptr, 0, s);
+    return launch_chunks(q4k_kernel<XT, kSmallT, 1, false>(), q4k_kernel<XT, kLargeT, 1, false>(),
+                         QF_Q4K_THREADS, QF_Q4K_WAVES, v, 1024, nullptr, nullptr, nullptr, 0, s);
 }
 
 qf_status launch_format(qf_format f, int mode, int x_type, const std::vector<DevTensor>& v,
@@ -198,8 +211,7 @@ qf_status launch_format(qf_format f, int mode, int x_type, const std::vector<Dev
 qf_status fakequant_impl(qf_format f, const qf_tensor* t, int n, const float* d_group_amax,
                          int n_groups, float* d_group_scale_out, void* stream, bool pack_only) {
     g_err[0] = 0;
-    if (f != QF_NVFP4 && f != QF_MXFP4 && f != QF_Q4K)
-        return fail(QF_ERR_UNSUPPORTED, "unknown format %d", (int)f);
+    if (!known_format(f)) return fail(QF_ERR_UNSUPPORTED, "unknown format %d", (int)f);
     if (n < 0) return fail(QF_ERR_INVALID_ARG, "n = %d < 0", n);
     if (n > 0 && t == nullptr) return fail(QF_ERR_INVALID_ARG, "tensor array is NULL");
     const bool nv = f == QF_NVFP4;
@@ -215,7 +227,7 @@ qf_status fakequant_impl(qf_format f, const qf_tensor* t, int n, const float* d_
         const int64_t numel = t[i].rows * t[i].cols;
         if (numel == 0) continue;
         void* y = pack_only ? nullptr : t[i].y;
-        void* scales = f == QF_Q4K ? nullptr : t[i].scales;
+        void* scales = (f == QF_Q4K || f == QF_Q4K_MSE) ? nullptr : t[i].scales;
         if (!y && !t[i].codes && !scales)
             return fail(QF_ERR_INVALID_ARG, "tensor %d: no output (y, codes, scales all NULL)", i);
         if (!aligned16(y) || !aligned16(t[i].codes))
@@ -489,8 +501,7 @@ qf_status qf_ste_backward(qf_format f, const void* grad_y, void* grad_x, int64_t
         if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
         return QF_OK;
     }
-    if (f != QF_NVFP4 && f != QF_MXFP4 && f != QF_Q4K)
-        return fail(QF_ERR_UNSUPPORTED, "unknown format %d", (int)f);
+    if (!known_format(f)) return fail(QF_ERR_UNSUPPORTED, "unknown format %d", (int)f);
     if (fwd == nullptr) return fail(QF_ERR_INVALID_ARG, "clipped STE needs the forward tensor");
     const bool nv = f == QF_NVFP4;
     if (nv && (n_groups <= 0 || d_group_amax == nullptr))
@@ -527,6 +538,6 @@ const char* qf_status_string(qf_status s) {
 
 const char* qf_last_error(void) { return g_err; }
 
-int qf_version(void) { return (1 << 16) | 2; }
+int qf_version(void) { return (1 << 16) | 3; }
 
 }  // extern "C"

@@ -559,16 +559,57 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     return v;
 }
 
+// Squared dequantization error of one sub-block at a trial scale (offset min_j),
+// summed in element order: q = clamp(RNE((x + min_j) / scale), 0, 15),
+// err = sum (x - (scale*q - min_j))^2, one rounding per operation.
+template <typename XT>
+__device__ __forceinline__ float q4k_sub_err(const Elems<XT, 32>& x, float scale, float min_j) {
+    const float inv = __frcp_rn(scale);
+    float err = 0.0f;
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+        const float t = __fmul_rn(__fadd_rn(x.get(k), min_j), inv);
+        const float q = __fsub_rn(__fadd_rn(fminf(fmaxf(t, 0.0f), 15.0f), kRound), kRound);
+        const float r = __fsub_rn(x.get(k), __fsub_rn(__fmul_rn(scale, q), min_j));
+        err = __fadd_rn(err, __fmul_rn(r, r));
+    }
+    return err;
+}
+
+// MSE-searched sub-block scale: with the offset fixed, try scale = (hi + min_j) / n
+// for n = 15 (the min/max fit) and then 14, 14.5, 15.5, 16, 16.5, 17, 17.5, 18; keep
+// the least squared error (a later trial must be strictly smaller).
+template <typename XT>
+__device__ __forceinline__ float q4k_search_scale(const Elems<XT, 32>& x, float hi, float min_j) {
+    const float range = __fadd_rn(hi, min_j);
+    float best = __fdiv_rn(range, 15.0f);
+    if (best == 0.0f) return best;
+    float best_err = q4k_sub_err(x, best, min_j);
+    const float steps[8] = {14.0f, 14.5f, 15.5f, 16.0f, 16.5f, 17.0f, 17.5f, 18.0f};
+#pragma unroll 1
+    for (int t = 0; t < 8; ++t) {
+        const float scale = __fdiv_rn(range, steps[t]);
+        const float err = q4k_sub_err(x, scale, min_j);
+        if (err < best_err) {
+            best_err = err;
+            best = scale;
+        }
+    }
+    return best;
+}
+
 // Per-lane fit of one sub-block; returns the super-block's FP16 d / dmin bits, this
-// sub-block's 6-bit sc / m, its s = d*sc, mm = dmin*m and inv = 1/s.
+// sub-block's 6-bit sc / m, its s = d*sc, mm = dmin*m and inv = 1/s.  MSE selects
+// the searched sub-block scale instead of the min/max one.
 struct Q4kFit { uint32_t dbits, dminbits, sc, m; float s, mm, inv; };
 
-template <typename XT>
+template <typename XT, bool MSE>
 __device__ __forceinline__ Q4kFit q4k_fit(const Elems<XT, 32>& x) {
     float lo, hi;
     x.minmax(lo, hi);
     const float min_j = lo < 0.0f ? -lo : 0.0f;
-    const float scale_j = __fdiv_rn(__fadd_rn(hi, min_j), 15.0f);
+    const float scale_j = MSE ? q4k_search_scale(x, hi, min_j)
+                              : __fdiv_rn(__fadd_rn(hi, min_j), 15.0f);
     float ms = scale_j, mm = min_j;
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {               // the 8 lanes of this super-block
@@ -590,7 +631,7 @@ __device__ __forceinline__ Q4kFit q4k_fit(const Elems<XT, 32>& x) {
 }
 
 // MODE 0: dequant (y) and/or 144-byte blocks (codes).  MODE 1: clipped STE, y = grad_x.
-template <typename XT, int MAXT, int MODE, int THREADS>
+template <typename XT, int MAXT, int MODE, int THREADS, bool MSE>
 __global__ void __launch_bounds__(THREADS) k_q4k(const __grid_constant__ Table<MAXT> P) {
     __shared__ __align__(16) uint8_t stage[THREADS / 32][kQ4kWarpBytes];
     constexpr bool kBf16 = sizeof(XT) == 2;
@@ -626,7 +667,7 @@ __global__ void __launch_bounds__(THREADS) k_q4k(const __grid_constant__ Table<M
             x.template load<1>(xp + e0 + 256 * b + 32 * j, have);
             __syncwarp();                                  // the previous unit's staging reads
         }
-        const Q4kFit f = q4k_fit(x);
+        const Q4kFit f = q4k_fit<XT, MSE>(x);
         const int64_t sb = (e0 >> 8) + b;                // this lane's super-block in the tensor
         if (MODE == 0) {
             // elements: q = clamp(RNE((x + mm) * inv), 0, 15); y = BF16(s*q - mm)

@@ -54,7 +54,8 @@ extern "C" {
 typedef enum {
     QF_NVFP4 = 0,
     QF_MXFP4 = 1,
-    QF_Q4K = 2
+    QF_Q4K = 2,
+    QF_Q4K_MSE = 3      /* Q4_K with the MSE-searched sub-block scales (same layout) */
 } qf_format;
 
 typedef enum {
@@ -244,6 +245,20 @@ qf_status qf_fakequant_lora(qf_format f, const qf_tensor* t, const qf_lora* l, i
                             const float* d_group_amax, int n_groups, float* d_group_scale_out,
                             void* stream);
 
+/*
+ * QF_Q4K_MSE -- the Q4_K format (identical 144-byte blocks and dequantization) with
+ * an MSE-searched fit, the kind of post-training quantizer the project page uses as
+ * its Q4_K PTQ baseline ("Key findings"; the pages do not give its steps).  Per
+ * 32-element sub-block, with min_j as in the min/max fit, the scale is chosen among
+ * (max x + min_j) / n for n = 15 (tried first), 14, 14.5, 15.5, 16, 16.5, 17, 17.5, 18
+ * as the one with the least
+ *   err = sum over i, in order, of (x_i - (scale*q_i - min_j))^2,
+ *   q_i = clamp(RNE((x_i + min_j) * (1/scale)), 0, 15)
+ * (binary32, one rounding per operation; a later n must be strictly better); then
+ * d, dmin, sc, m and the codes follow exactly as for QF_Q4K.  Accepted by
+ * qf_fakequant, qf_pack and qf_ste_backward.
+ */
+
 /* Static description of a status code. */
 const char* qf_status_string(qf_status s);
 
@@ -251,7 +266,8 @@ const char* qf_status_string(qf_status s);
 const char* qf_last_error(void);
 
 /* ABI version: (major << 16) | minor.  1.1 added qf_tensor.x_type (formerly a
- * reserved field that had to be 0, which still means BF16); 1.2 the LoRA calls. */
+ * reserved field that had to be 0, which still means BF16); 1.2 the LoRA calls;
+ * 1.3 QF_Q4K_MSE. */
 int qf_version(void);
 
 #ifdef __cplusplus

@@ -107,7 +107,7 @@ def oracle_outputs(fmt: str, x_cpu, amax_g: float = 0.0):
         return y, c, s
     if fmt == "mxfp4":
         return oracle.mxfp4(x_cpu)
-    y, b = oracle.q4k(x_cpu)
+    y, b = oracle.q4k(x_cpu, mse=fmt == "q4k_mse")
     return y, b, None
 
 
@@ -127,8 +127,9 @@ def compare_rows(fmt: str, x_cpu, y_bits, codes, scales, rows, amax_g: float = 0
     """Compare the CUDA outputs of selected rows with the oracle run on those rows alone
     (rows are independent given the tie-group amax)."""
     R, K = x_cpu.shape
-    cpr = K // 2 if fmt != "q4k" else (K // 256) * 144
-    spr = K // (16 if fmt == "nvfp4" else 32) if fmt != "q4k" else 0
+    q4 = fmt in ("q4k", "q4k_mse")
+    cpr = K // 2 if not q4 else (K // 256) * 144
+    spr = K // (16 if fmt == "nvfp4" else 32) if not q4 else 0
     for r in rows:
         xr = x_cpu[r:r + 1]
         y, c, s = oracle_outputs(fmt, xr, amax_g)

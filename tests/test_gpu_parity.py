@@ -359,3 +359,36 @@ def test_f32_clipped_ste_and_ragged_amax(fmt):
     torch.cuda.synchronize()
     want = oracle.tied_amax(ts, [0, 0, 0], 1)
     assert_same("f32 ragged amax", amax.cpu().numpy().view(np.uint32), want.view(np.uint32))
+
+
+# ----------------------------------------------------------------------------- Q4_K, MSE-searched fit
+def test_q4k_mse_small_and_ragged():
+    wl = workloads.q4k_weights(rows_scale=1 / 64)
+    ts = wl["tensors"] + [workloads.normal_with_outliers(3, 768, 0.02, 1e-2, 20.0, 7, 0),
+                          _f32_weights(5, 256, 90)[:, :256].contiguous()]
+    res = run_fakequant("q4k_mse", ts[:3])
+    compare_full("q4k_mse", ts[:3], res, label="q4k mse")
+    for i, t in enumerate(ts[3:]):                 # one element type per call
+        res = run_fakequant("q4k_mse", [t])
+        compare_full("q4k_mse", [t], res, label=f"q4k mse extra {i}")
+
+
+def test_q4k_mse_pack_and_clipped_ste():
+    x = workloads.q4k_weights(rows_scale=1 / 256)["tensors"][1]
+    full = run_fakequant("q4k_mse", [x])
+    pk = run_fakequant("q4k_mse", [x], pack_only=True)
+    assert_same("q4k mse pack", pk["codes"][0], full["codes"][0])
+    g = workloads.normal_with_outliers(x.shape[0], x.shape[1], 1e-3, 0, 1, 3, 91)
+    out = torch.empty(x.shape, dtype=torch.bfloat16, device=DEV)
+    qf.qf_ste_backward(g.to(DEV), out, mode=1, fmt="q4k_mse", x=x.to(DEV))
+    torch.cuda.synchronize()
+    assert_same("q4k mse ste", bits(out), oracle.ste_backward(g, 1, "q4k_mse", x))
+
+
+@pytest.mark.slow
+def test_full_q4k_mse_sampled_rows():
+    wl = workloads.q4k_weights()
+    res = run_fakequant("q4k_mse", wl["tensors"])
+    for i, x in enumerate(wl["tensors"]):
+        compare_rows("q4k_mse", x, res["y"][i], res["codes"][i], None,
+                     sample_rows(x.shape[0], 24, 500 + i), label=f"q4k mse[{i}]")
