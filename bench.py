@@ -6,8 +6,9 @@ N(0, 0.02) and activations 8 x 4096 tokens by 4096 hidden, Student-t(3) with 1%
 of channels x50 -- quantized in ONE grouped qf_fakequant launch that writes
 dequantized BF16, packed E2M1 nibbles and E8M0 block scales.  A step is that
 launch.  Other workloads (`--workload`): nvfp4_tied, q4k, nvfp4_weight,
-activation, moe_nvfp4, moe_mxfp4, moe_q4k; an NVFP4 step is the tied-amax pass
-followed by the fused pass.
+activation, moe_nvfp4, moe_mxfp4, moe_q4k, nvfp4_tied_f32, q4k_f32 (FP32 master
+weights), lora_nvfp4 (LoRA-merged weights), q4k_mse (MSE-searched Q4_K fit); an
+NVFP4 step is the tied-amax pass followed by the fused pass.
 
   value      GB/s of algorithmic bytes per step (read BF16 + write BF16 + codes +
              scales = 4.5625 / 4.53125 / 4.5625 B per element for NVFP4 / MXFP4 /
@@ -15,12 +16,13 @@ followed by the fused pass.
              max over ranks, summed over ranks (weak scaling).
   e2e        the same metric through the public API with pinned host buffers:
              host->device copy of the inputs, the step, device->host copy of every
-             output, per step.
+             output, per step, pipelined in row chunks (host.HostPipeline).
   roofline   the fused-pass kernel's achieved GB/s (its algorithmic bytes / its
              mean CUDA-event duration in the timed region) against the measured
              HBM copy bandwidth.
   cpu_baseline  the oracle (scalar C, one thread) on a bounded sample of the rows.
-  per_format the other workloads, each timed per call with the L2 flushed.
+  per_format the other workloads, each timed per call with the L2 flushed
+             (L2Flush: L2 left holding only clean lines).
 
 `--impl reference` times the oracle on the host cores for the same metric (the
 reference arm).  Launch with torchrun for N > 1 GPUs (one process per GPU).
@@ -265,7 +267,7 @@ def run_ours(args, rank, world, local_rank):
     W = make_workload(args.workload, qf, dev, seed_shift=1000 * rank)
     numel, step_bytes = W["numel"], W["step_bytes"]
     in_bytes = W["in_bytes"] * numel
-    flush_buf = torch.empty(2 * l2, dtype=torch.uint8, device=dev) if in_bytes < 2 * l2 else None
+    flush_buf = L2Flush(dev, l2) if in_bytes < 2 * l2 else None
     torch.cuda.synchronize()
 
     for _ in range(args.warmup):
@@ -279,7 +281,7 @@ def run_ours(args, rank, world, local_rank):
     with ClockSampler(torch.cuda.current_device()) as clk:
         for i in range(args.steps):
             if flush_buf is not None:
-                flush_buf.add_(1)            # L2 flush, outside the timed event pairs
+                flush_buf()                  # L2 flush, outside the timed event pairs
             ev[i][0].record(stream)
             if W["pre"] is not None:
                 W["pre"]()
@@ -338,7 +340,8 @@ def run_ours(args, rank, world, local_rank):
                    "elements_per_step": numel, "bytes_per_step": step_bytes,
                    "input": "fp32" if W["in_bytes"] == 4 else "bf16",
                    "l2": (f"L2 flushed before every step ({in_bytes / 1e6:.0f} MB of input "
-                          f"< 2x the {l2 / 1e6:.0f} MB L2)") if flush_buf is not None else
+                          f"< 2x the {l2 / 1e6:.0f} MB L2): write a 2xL2 buffer, then read "
+                          f"another, so L2 holds only clean lines") if flush_buf is not None else
                          (f"inputs larger than L2 ({in_bytes / 1e6:.0f} MB of input vs "
                           f"{l2 / 1e6:.0f} MB); no flush between steps"),
                    "parallelism": f"replicas x{world} (weak scaling, no collective)"},
@@ -355,6 +358,24 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0 and world == 1 and not args.no_cpu:
         result["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_rows_frac)
     return result
+
+
+class L2Flush:
+    """Evicts the timed kernel's data from L2 between timed calls.
+
+    It writes a buffer of twice the L2 size, then reads a second one of that size.
+    The read writes back the dirty lines the write left, so L2 holds only clean
+    lines when the timed region starts.  Otherwise the timed kernel would pay for
+    writing back up to a whole L2 of the flush's own data.  That costs a kernel of
+    tens of MB nearly as much as its own traffic."""
+
+    def __init__(self, dev, l2: int):
+        self.w = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+        self.r = torch.zeros(2 * l2 // 8, dtype=torch.int64, device=dev)
+
+    def __call__(self):
+        self.w.add_(1)
+        self.r.max()
 
 
 def timed_calls(fn, iters, warm, flush):
@@ -375,23 +396,26 @@ def timed_calls(fn, iters, warm, flush):
 
 def per_format(qf, dev, args, l2):
     peak, _ = peaks()
-    scratch = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
-    flush = lambda: scratch.add_(1)  # noqa: E731
+    flush = L2Flush(dev, l2)
     out = {}
     for name in WORKLOADS:
         if name == args.workload:
             continue
         W = make_workload(name, qf, dev)
-        it = args.pf_iters
-        t_fq = timed_calls(W["fq"], it, 3, flush)
+        it, warm = args.pf_iters, args.pf_warmup
+        t_fq = timed_calls(W["fq"], it, warm, flush)
+        t_hot = timed_calls(W["fq"], it, warm, lambda: None)
         gbs = W["fq_bytes"] / (t_fq * 1e-3) / 1e9
         d = {"format": W["fmt"], "input": "fp32" if W["in_bytes"] == 4 else "bf16",
              "tensors": W["n_tensors"], "elements": W["numel"],
              "fused_us": t_fq * 1e3, "fused_GB/s": gbs, "fused_Gelem/s": W["numel"] / t_fq / 1e6,
-             "fused_frac_of_hbm_peak": gbs / peak}
+             "fused_frac_of_hbm_peak": gbs / peak,
+             # back-to-back calls without a flush: a tensor that fits in L2 is read from it
+             "fused_hot_l2_us": t_hot * 1e3,
+             "fused_hot_l2_GB/s": W["fq_bytes"] / (t_hot * 1e-3) / 1e9}
         if W["pre"] is not None:
-            t_pre = timed_calls(W["pre"], it, 3, flush)
-            t_step = timed_calls(lambda: run_step(W), it, 3, flush)
+            t_pre = timed_calls(W["pre"], it, warm, flush)
+            t_step = timed_calls(lambda: run_step(W), it, warm, flush)
             d.update({"amax_us": t_pre * 1e3,
                       "amax_GB/s": W["in_bytes"] * W["numel"] / t_pre / 1e6,
                       "step_us": t_step * 1e3,
@@ -499,7 +523,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="w4a4", choices=WORKLOADS)
     ap.add_argument("--e2e-steps", type=int, default=5)
-    ap.add_argument("--pf-iters", type=int, default=20)
+    ap.add_argument("--pf-iters", type=int, default=100)
+    ap.add_argument("--pf-warmup", type=int, default=20)
     ap.add_argument("--cpu-rows-frac", type=float, default=0.5)
     ap.add_argument("--no-per-format", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")

@@ -156,6 +156,35 @@ __device__ __forceinline__ float f16_lo(uint32_t h2) {
 __device__ __forceinline__ float f16_hi(uint32_t h2) {
     return __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
 }
+// Paired FP32 arithmetic of sm_100 (two independent lanes per instruction); each
+// half rounds exactly as the scalar mul.rn / add.rn / fma.rn.f32 of the same
+// operands.  One rule on their use: a paired product must not feed an add.  The
+// code generator was seen to fuse a paired multiply and a following paired add
+// into one rounding despite the explicit .rn (and also when the product was
+// written as fma(a, b, -0)); a parity test caught it.  So paired products here
+// feed only conversions, comparisons and selects, paired adds take no product,
+// and every product that is added to something is a scalar __fmul_rn.
+__device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 add2_rn(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 fma2_rn(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mov.b64 rc, {%6, %7};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
@@ -559,40 +588,66 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     return v;
 }
 
-// Squared dequantization error of one sub-block at a trial scale (offset min_j),
+// Squared dequantization error of one sub-block at two trial scales (offset min_j),
 // summed in element order: q = clamp(RNE((x + min_j) / scale), 0, 15),
-// err = sum (x - (scale*q - min_j))^2, one rounding per operation.
+// err = sum (x - (scale*q - min_j))^2, one rounding per operation.  The two trials
+// share sm_100's paired FP32 pipe where no product feeds an add (the scaled value
+// and the rounding to an integer); the products scale*q and r*r, which are added
+// to, stay scalar.  The error is accumulated as (dq - x)^2, whose square equals
+// that of x - dq bit for bit (round-to-nearest is symmetric, so dq - x is exactly
+// -(x - dq)).
 template <typename XT>
-__device__ __forceinline__ float q4k_sub_err(const Elems<XT, 32>& x, float scale, float min_j) {
-    const float inv = __frcp_rn(scale);
-    float err = 0.0f;
+__device__ __forceinline__ float2 q4k_sub_err2(const Elems<XT, 32>& x, float2 scale, float min_j) {
+    const float2 inv = make_float2(__frcp_rn(scale.x), __frcp_rn(scale.y));
+    const float2 rnd = make_float2(kRound, kRound), nrnd = make_float2(-kRound, -kRound);
+    float2 err = make_float2(0.0f, 0.0f);
 #pragma unroll
     for (int k = 0; k < 32; ++k) {
-        const float t = __fmul_rn(__fadd_rn(x.get(k), min_j), inv);
-        const float q = __fsub_rn(__fadd_rn(fminf(fmaxf(t, 0.0f), 15.0f), kRound), kRound);
-        const float r = __fsub_rn(x.get(k), __fsub_rn(__fmul_rn(scale, q), min_j));
-        err = __fadd_rn(err, __fmul_rn(r, r));
+        const float xk = x.get(k);
+        const float xm = __fadd_rn(xk, min_j);
+        const float2 t = mul2_rn(make_float2(xm, xm), inv);
+        const float2 c = make_float2(fminf(fmaxf(t.x, 0.0f), 15.0f), fminf(fmaxf(t.y, 0.0f), 15.0f));
+        const float2 q = add2_rn(add2_rn(c, rnd), nrnd);
+        const float2 dq = make_float2(__fsub_rn(__fmul_rn(scale.x, q.x), min_j),
+                                      __fsub_rn(__fmul_rn(scale.y, q.y), min_j));
+        const float2 r = add2_rn(dq, make_float2(-xk, -xk));
+        err = make_float2(__fadd_rn(err.x, __fmul_rn(r.x, r.x)),
+                          __fadd_rn(err.y, __fmul_rn(r.y, r.y)));
     }
     return err;
 }
 
 // MSE-searched sub-block scale: with the offset fixed, try scale = (hi + min_j) / n
 // for n = 15 (the min/max fit) and then 14, 14.5, 15.5, 16, 16.5, 17, 17.5, 18; keep
-// the least squared error (a later trial must be strictly smaller).
+// the least squared error (a later trial must be strictly smaller).  The errors are
+// computed two trials at a time and then compared in trial order.
 template <typename XT>
 __device__ __forceinline__ float q4k_search_scale(const Elems<XT, 32>& x, float hi, float min_j) {
     const float range = __fadd_rn(hi, min_j);
     float best = __fdiv_rn(range, 15.0f);
     if (best == 0.0f) return best;
-    float best_err = q4k_sub_err(x, best, min_j);
-    const float steps[8] = {14.0f, 14.5f, 15.5f, 16.0f, 16.5f, 17.0f, 17.5f, 18.0f};
+    const float s14 = __fdiv_rn(range, 14.0f);
+    const float2 e0 = q4k_sub_err2(x, make_float2(best, s14), min_j);
+    float best_err = e0.x;
+    if (e0.y < best_err) {
+        best_err = e0.y;
+        best = s14;
+    }
+    // the remaining trials in pairs (14.5, 15.5), (16, 16.5), (17, 17.5) and 18 alone
+    // (its pair's second half repeats it and is ignored)
 #pragma unroll 1
-    for (int t = 0; t < 8; ++t) {
-        const float scale = __fdiv_rn(range, steps[t]);
-        const float err = q4k_sub_err(x, scale, min_j);
-        if (err < best_err) {
-            best_err = err;
-            best = scale;
+    for (int p = 0; p < 4; ++p) {
+        const float na = p == 0 ? 14.5f : p == 1 ? 16.0f : p == 2 ? 17.0f : 18.0f;
+        const float nb = p == 0 ? 15.5f : p == 1 ? 16.5f : p == 2 ? 17.5f : 18.0f;
+        const float2 sc = make_float2(__fdiv_rn(range, na), __fdiv_rn(range, nb));
+        const float2 err = q4k_sub_err2(x, sc, min_j);
+        if (err.x < best_err) {
+            best_err = err.x;
+            best = sc.x;
+        }
+        if (p < 3 && err.y < best_err) {
+            best_err = err.y;
+            best = sc.y;
         }
     }
     return best;

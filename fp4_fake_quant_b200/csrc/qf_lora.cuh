@@ -15,6 +15,12 @@
 // in registers across the CTA's rows; the CTA stages its kLoraRows rows of B in
 // shared memory as FP32, so every B read is a broadcast.  W, y and codes accesses
 // are contiguous 256-, 256- and 64-byte warp runs per row.
+//
+// The products run on sm_100's paired FP32 pipe: one fma.rn.f32x2 updates the
+// accumulators of two adjacent columns, each rounded exactly as a scalar
+// fma.rn.f32 would be (and, the products being exact, as a separate multiply and
+// add would be).  B is stored in shared memory with every value twice, so one
+// 16-byte load yields the (b, b) operand pairs of two consecutive k.
 #pragma once
 
 #include "qf_device.cuh"
@@ -64,15 +70,11 @@ __device__ __forceinline__ int lora_locate(const LoraTable<MAXT>& P, int64_t u) 
     return lo;
 }
 
-__device__ __forceinline__ float bf16_round(float v) {
-    return __uint_as_float(cvt_bf16x2(0.0f, v) << 16);
-}
-
 // R: compile-time rank capacity (the runtime rank is <= R; A and B are zero-padded,
 // which adds exact zeros to an accumulator that is never -0, so results do not change).
 template <int MODE, int R, int MAXT>
 __global__ void __launch_bounds__(kLoraThreads) k_lora(const __grid_constant__ LoraTable<MAXT> P) {
-    __shared__ __align__(16) float bsm[kLoraRows][R];
+    __shared__ __align__(16) float2 bsm[kLoraRows][R];      // (b, b) pairs
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int64_t cu = blockIdx.x;
     if (MODE != kLoraAmax && cu == 0 && P.group_scale_out) {
@@ -93,16 +95,17 @@ __global__ void __launch_bounds__(kLoraThreads) k_lora(const __grid_constant__ L
     // this CTA's rows of B as FP32, zero-padded to R
     for (int idx = threadIdx.x; idx < kLoraRows * R; idx += kLoraThreads) {
         const int i = idx / R, k = idx % R;
-        bsm[i][k] = (i < nrows && k < rank) ? bf16_lo(T.b[(r0 + i) * rank + k]) : 0.0f;
+        const float b = (i < nrows && k < rank) ? bf16_lo(T.b[(r0 + i) * rank + k]) : 0.0f;
+        bsm[i][k] = make_float2(b, b);
     }
-    // this lane's 4 columns of A as FP32, zero-padded to R
-    float a[R][4];
+    // this lane's 4 columns of A as FP32 pairs (columns 0,1 and 2,3), zero-padded to R
+    float2 a[R][2];
 #pragma unroll
     for (int k = 0; k < R; ++k) {
         uint2 v = make_uint2(0, 0);
         if (k < rank && colok) v = *reinterpret_cast<const uint2*>(T.a + k * T.cols + col0);
-        a[k][0] = bf16_lo(v.x); a[k][1] = bf16_hi(v.x);
-        a[k][2] = bf16_lo(v.y); a[k][3] = bf16_hi(v.y);
+        a[k][0] = make_float2(bf16_lo(v.x), bf16_hi(v.x));
+        a[k][1] = make_float2(bf16_lo(v.y), bf16_hi(v.y));
     }
     __syncthreads();
 
@@ -127,31 +130,34 @@ __global__ void __launch_bounds__(kLoraThreads) k_lora(const __grid_constant__ L
         if (i0 + 4 < nrows) load_w(i0 + 4, wnxt);          // the next 4 rows, in flight meanwhile
         // merged values of 4 rows x this lane's 4 columns
         float x[4][4];
+        uint32_t xw[4][2];                                   // the same, as packed BF16 pairs
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
             const int i = min(i0 + h, nrows - 1);            // rows past the end are not stored
-            float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            float2 acc01 = make_float2(0.0f, 0.0f), acc23 = make_float2(0.0f, 0.0f);
 #pragma unroll
-            for (int k = 0; k < R; k += 4) {
+            for (int k = 0; k < R; k += 2) {
                 const float4 bk = *reinterpret_cast<const float4*>(&bsm[i][k]);
-                const float bb[4] = {bk.x, bk.y, bk.z, bk.w};
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) acc[c] = __fmaf_rn(bb[q], a[k + q][c], acc[c]);
+                const float2 b0 = make_float2(bk.x, bk.y), b1 = make_float2(bk.z, bk.w);
+                acc01 = fma2_rn(b0, a[k][0], acc01);
+                acc23 = fma2_rn(b0, a[k][1], acc23);
+                acc01 = fma2_rn(b1, a[k + 1][0], acc01);
+                acc23 = fma2_rn(b1, a[k + 1][1], acc23);
             }
-            const float wf[4] = {bf16_lo(wcur[h].x), bf16_hi(wcur[h].x), bf16_lo(wcur[h].y),
-                                 bf16_hi(wcur[h].y)};
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-                x[h][c] = bf16_round(__fadd_rn(wf[c], __fmul_rn(T.scale, acc[c])));
+            // scalar: a paired product must not feed an add (see mul2_rn)
+            xw[h][0] = cvt_bf16x2(__fadd_rn(bf16_hi(wcur[h].x), __fmul_rn(T.scale, acc01.y)),
+                                  __fadd_rn(bf16_lo(wcur[h].x), __fmul_rn(T.scale, acc01.x)));
+            xw[h][1] = cvt_bf16x2(__fadd_rn(bf16_hi(wcur[h].y), __fmul_rn(T.scale, acc23.y)),
+                                  __fadd_rn(bf16_lo(wcur[h].y), __fmul_rn(T.scale, acc23.x)));
+            x[h][0] = bf16_lo(xw[h][0]); x[h][1] = bf16_hi(xw[h][0]);
+            x[h][2] = bf16_lo(xw[h][1]); x[h][3] = bf16_hi(xw[h][1]);
         }
         if (MODE == kLoraMerge) {
 #pragma unroll
             for (int h = 0; h < 4; ++h)
                 if (colok && i0 + h < nrows && T.y)
                     *reinterpret_cast<uint2*>(T.y + (r0 + i0 + h) * T.cols + col0) =
-                        make_uint2(cvt_bf16x2(x[h][1], x[h][0]), cvt_bf16x2(x[h][3], x[h][2]));
+                        make_uint2(xw[h][0], xw[h][1]);
         } else {
             uint32_t m[4];
 #pragma unroll
@@ -199,9 +205,10 @@ __global__ void __launch_bounds__(kLoraThreads) k_lora(const __grid_constant__ L
                 }
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
-                    float q[4];
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) q[c] = __fmul_rn(x[h][c], inv[h]);
+                    const float2 inv2 = make_float2(inv[h], inv[h]);
+                    const float2 q01 = mul2_rn(make_float2(x[h][0], x[h][1]), inv2);
+                    const float2 q23 = mul2_rn(make_float2(x[h][2], x[h][3]), inv2);
+                    float q[4] = {q01.x, q01.y, q23.x, q23.y};
                     if (MODE == kLoraNV && __builtin_expect(isinf(inv[h]), 0)) {
 #pragma unroll
                         for (int c = 0; c < 4; ++c)
@@ -212,9 +219,11 @@ __global__ void __launch_bounds__(kLoraThreads) k_lora(const __grid_constant__ L
                     const int64_t e = (r0 + i0 + h) * T.cols + col0;   // flat element index
                     if (T.y) {
                         const uint32_t h0 = cvt_e2m1x2_f16x2(b0), h1 = cvt_e2m1x2_f16x2(b1);
-                        *reinterpret_cast<uint2*>(T.y + e) = make_uint2(
-                            cvt_bf16x2(__fmul_rn(f16_hi(h0), S[h]), __fmul_rn(f16_lo(h0), S[h])),
-                            cvt_bf16x2(__fmul_rn(f16_hi(h1), S[h]), __fmul_rn(f16_lo(h1), S[h])));
+                        const float2 S2 = make_float2(S[h], S[h]);
+                        const float2 d01 = mul2_rn(make_float2(f16_lo(h0), f16_hi(h0)), S2);
+                        const float2 d23 = mul2_rn(make_float2(f16_lo(h1), f16_hi(h1)), S2);
+                        *reinterpret_cast<uint2*>(T.y + e) =
+                            make_uint2(cvt_bf16x2(d01.y, d01.x), cvt_bf16x2(d23.y, d23.x));
                     }
                     if (T.codes)
                         *reinterpret_cast<uint16_t*>(T.codes + (e >> 1)) = (uint16_t)(b0 | (b1 << 8));
