@@ -183,7 +183,9 @@ def make_workload(name: str, qf, dev, seed_shift: int = 0):
                 "pass + one grouped fake-quant+pack launch (FP32 in, BF16 + codes out)")
     elif name == "nvfp4_weight":
         wl, fmt = workloads.nvfp4_weight(seed=0 + seed_shift), "nvfp4"
-        desc = "NVFP4 weight 4096x4096 N(0,0.02), 0.1% x20 outliers; amax pass + fake-quant+pack"
+        desc = ("NVFP4 weight 4096x4096 N(0,0.02), 0.1% x20 outliers; qf_amax_fakequant: amax, "
+                "grid barrier and fake-quant+pack in one cooperative launch (input L2-resident "
+                "for the second pass)")
     elif name in ("moe_nvfp4", "moe_mxfp4", "moe_q4k"):
         key = ("moe", seed_shift)                    # the three formats share one input set
         if key not in _CACHE:
@@ -227,6 +229,21 @@ def make_workload(name: str, qf, dev, seed_shift: int = 0):
         W["launches"] = 2
         W["kernel"] = "k_lora_nvfp4"
         W["adapters"] = ads
+        return W
+    if name == "nvfp4_weight":
+        amax = torch.zeros(ng, dtype=torch.float32, device=dev)
+        so = torch.empty(ng, dtype=torch.float32, device=dev)
+        W["workspace"] = qf.alloc_workspace(ng, dev)
+        W["pre"] = None
+        W["fq"] = qf.prepare_amax_fakequant(xs, Y, C, S, groups, amax, group_scale_out=so,
+                                            workspace=W["workspace"])
+        W["fq_bytes"] = W["step_bytes"] = W["fq_bytes"] + in_b * numel
+        W["launches"] = 1
+        W["kernel"] = "k_nv_oneshot"
+        # the same step as two launches (qf_amax_tied, then qf_fakequant), for comparison
+        pre2 = qf.prepare_amax_tied(xs, groups, amax)
+        fq2 = qf.prepare_fakequant(fmt, xs, Y, C, S, groups, amax, so)
+        W["two_call"] = lambda: (pre2(), fq2())
         return W
     if fmt == "nvfp4":
         amax = torch.zeros(ng, dtype=torch.float32, device=dev)
@@ -420,6 +437,11 @@ def per_format(qf, dev, args, l2):
                       "amax_GB/s": W["in_bytes"] * W["numel"] / t_pre / 1e6,
                       "step_us": t_step * 1e3,
                       "step_GB/s": W["step_bytes"] / t_step / 1e6})
+        if "two_call" in W:
+            t2 = timed_calls(W["two_call"], it, warm, flush)
+            d.update({"fused_is": "the whole one-launch step (amax + fake-quant + pack)",
+                      "two_launch_step_us": t2 * 1e3,
+                      "two_launch_step_GB/s": W["step_bytes"] / t2 / 1e6})
         if name.startswith("moe_"):
             xs, fmt = W["xs"], W["fmt"]
             n = len(xs)

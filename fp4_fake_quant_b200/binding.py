@@ -22,7 +22,7 @@ QF_X_BF16, QF_X_F32 = 0, 1
 FORMATS = {"nvfp4": QF_NVFP4, "mxfp4": QF_MXFP4, "q4k": QF_Q4K, "q4k_mse": QF_Q4K_MSE}
 BLOCK = {QF_NVFP4: 16, QF_MXFP4: 32, QF_Q4K: 256, QF_Q4K_MSE: 256}
 STATUS = {0: "QF_OK", 1: "QF_ERR_INVALID_ARG", 2: "QF_ERR_SHAPE", 3: "QF_ERR_ALIGN",
-          4: "QF_ERR_UNSUPPORTED", 5: "QF_ERR_CUDA"}
+          4: "QF_ERR_UNSUPPORTED", 5: "QF_ERR_CUDA", 6: "QF_ERR_TIMEOUT"}
 
 
 class QfTensor(ctypes.Structure):
@@ -59,8 +59,13 @@ def _load() -> ctypes.CDLL:
     lib.qf_lora_merge.argtypes = [T, L, I, P]
     lib.qf_amax_tied_lora.argtypes = [T, L, I, P, I, P]
     lib.qf_fakequant_lora.argtypes = [I, T, L, I, P, I, P, P]
+    lib.qf_amax_fakequant.argtypes = [T, I, P, I, P, P, P, ctypes.c_size_t, P]
+    lib.qf_amax_fakequant_workspace_bytes.argtypes = [I]
+    lib.qf_amax_fakequant_workspace_bytes.restype = ctypes.c_size_t
+    lib.qf_workspace_check.argtypes = [P, P]
     for f in (lib.qf_amax_tied, lib.qf_fakequant, lib.qf_pack, lib.qf_ste_backward,
-              lib.qf_lora_merge, lib.qf_amax_tied_lora, lib.qf_fakequant_lora):
+              lib.qf_lora_merge, lib.qf_amax_tied_lora, lib.qf_fakequant_lora,
+              lib.qf_amax_fakequant, lib.qf_workspace_check):
         f.restype = I
     lib.qf_status_string.argtypes = [I]
     lib.qf_status_string.restype = ctypes.c_char_p
@@ -75,8 +80,9 @@ lib = _load()
 
 # the entry points declared in include/qf.h
 EXPORTS = ("qf_amax_tied", "qf_fakequant", "qf_pack", "qf_ste_backward", "qf_lora_merge",
-           "qf_amax_tied_lora", "qf_fakequant_lora", "qf_status_string", "qf_last_error",
-           "qf_version")
+           "qf_amax_tied_lora", "qf_fakequant_lora", "qf_amax_fakequant",
+           "qf_amax_fakequant_workspace_bytes", "qf_workspace_check", "qf_status_string",
+           "qf_last_error", "qf_version")
 
 
 def _check(status: int) -> None:
@@ -216,6 +222,42 @@ def prepare_amax_tied(xs, groups, group_amax, tracked=None) -> Prepared:
     keep = (arr, list(xs), group_amax, tracked)
     return Prepared(lib.qf_amax_tied, (arr, n, _ptr(group_amax), group_amax.numel(), _ptr(tracked)),
                     keep)
+
+
+def workspace_bytes(n_groups: int) -> int:
+    """Bytes of device workspace qf_amax_fakequant needs for ``n_groups`` tie groups."""
+    return int(lib.qf_amax_fakequant_workspace_bytes(int(n_groups)))
+
+
+def alloc_workspace(n_groups: int, device=None) -> torch.Tensor:
+    """A zeroed qf_amax_fakequant workspace (a torch allocation; plumbing)."""
+    dev = torch.device(device) if device is not None else torch.device("cuda")
+    return torch.zeros(workspace_bytes(n_groups), dtype=torch.uint8, device=dev)
+
+
+def qf_amax_fakequant(xs, ys=None, codes=None, scales=None, groups=None, group_amax=None,
+                      tracked=None, group_scale_out=None, workspace=None, stream=None) -> None:
+    """NVFP4 tie-group amax and fused fake-quant + pack in one call (one launch when
+    the inputs fit in L2 and a workspace is given)."""
+    arr, n = _desc(xs, ys, codes, scales, groups)
+    wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib.qf_amax_fakequant(arr, n, _ptr(group_amax), group_amax.numel(), _ptr(tracked),
+                                 _ptr(group_scale_out), _ptr(workspace), wsb, _stream(stream)))
+
+
+def prepare_amax_fakequant(xs, ys=None, codes=None, scales=None, groups=None, group_amax=None,
+                           tracked=None, group_scale_out=None, workspace=None) -> "Prepared":
+    arr, n = _desc(xs, ys, codes, scales, groups)
+    wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    keep = (arr, list(xs), ys, codes, scales, group_amax, tracked, group_scale_out, workspace)
+    return Prepared(lib.qf_amax_fakequant,
+                    (arr, n, _ptr(group_amax), group_amax.numel(), _ptr(tracked),
+                     _ptr(group_scale_out), _ptr(workspace), wsb), keep)
+
+
+def qf_workspace_check(workspace: torch.Tensor, stream=None) -> None:
+    """Synchronize and raise QfError(QF_ERR_TIMEOUT) if a grid barrier gave up."""
+    _check(lib.qf_workspace_check(_ptr(workspace), _stream(stream)))
 
 
 def _lora(adapters):

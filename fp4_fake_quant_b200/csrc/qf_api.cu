@@ -12,6 +12,7 @@
 #include "qf.h"
 #include "qf_device.cuh"
 #include "qf_lora.cuh"
+#include "qf_oneshot.cuh"
 
 namespace {
 
@@ -22,7 +23,10 @@ using qf::kThreads;
 constexpr int kSmallT = 8;      // descriptor table sizes (kernel-parameter bytes: ~0.6 KB / ~27 KB)
 constexpr int kLargeT = 384;
 constexpr int kFp4U = QF_FP4_U;  // 256-element sub-tiles per warp unit
-constexpr int kAmaxU = 8;
+#ifndef QF_AMAX_U
+#define QF_AMAX_U 4
+#endif
+constexpr int kAmaxU = QF_AMAX_U;
 
 thread_local char g_err[512] = "";
 
@@ -47,18 +51,32 @@ bool known_format(qf_format f) {
 
 // Launch shape of one kernel: SM count, resident CTAs per SM, CTA size, waves.
 struct Launch { int sms; int per_sm; int threads; int waves; };
+// The SM count and occupancy of a (kernel, CTA size, device) are queried once per
+// host thread and kept: the queries cost microseconds of host time per call.
+struct ShapeEntry { const void* kernel; int threads; int dev; int sms; int per_sm; };
+
 template <typename K>
 qf_status launch_shape(K kernel, int threads, int waves, Launch* L) {
+    thread_local std::vector<ShapeEntry> cache;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    const void* key = reinterpret_cast<const void*>(kernel);
+    L->threads = threads;
+    L->waves = waves;
+    for (const ShapeEntry& c : cache) {
+        if (c.kernel == key && c.threads == threads && c.dev == dev) {
+            L->sms = c.sms;
+            L->per_sm = c.per_sm;
+            return QF_OK;
+        }
+    }
     e = cudaDeviceGetAttribute(&L->sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&L->per_sm, kernel, threads, 0);
     if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
     if (L->per_sm < 1) L->per_sm = 1;
-    L->threads = threads;
-    L->waves = waves;
+    cache.push_back({key, threads, dev, L->sms, L->per_sm});
     return QF_OK;
 }
 
@@ -347,6 +365,97 @@ qf_status lora_tensors(const qf_tensor* t, const qf_lora* l, int n, int cols_mul
     return QF_OK;
 }
 
+// Zero the group amax, then fold max |x| of every tensor into its group (and into
+// the running amax when d_tracked is given).
+qf_status amax_launch(const std::vector<DevTensor>& v, int x_type, float* d_group_amax,
+                      int n_groups, float* d_tracked, cudaStream_t s) {
+    bool ragged = false;
+    for (const DevTensor& d : v) ragged |= (d.numel & 7) != 0;
+    cudaError_t e = cudaMemsetAsync(d_group_amax, 0, sizeof(float) * (size_t)n_groups, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+    if (v.empty()) return QF_OK;
+    const bool f32 = x_type == QF_X_F32;
+    // the same bytes in flight per lane: 8 vectors of BF16, or 4 sub-tiles of FP32 (8 vectors)
+    qf_status st = f32
+        ? launch_chunks(qf::k_amax<float, kAmaxU / 2, kSmallT, QF_AMAX_THREADS>,
+                        qf::k_amax<float, kAmaxU / 2, kLargeT, QF_AMAX_THREADS>, QF_AMAX_THREADS,
+                        QF_AMAX_WAVES, v, 256 * (kAmaxU / 2), d_group_amax, nullptr, d_tracked,
+                        n_groups, s)
+        : launch_chunks(qf::k_amax<uint16_t, kAmaxU, kSmallT, QF_AMAX_THREADS>,
+                        qf::k_amax<uint16_t, kAmaxU, kLargeT, QF_AMAX_THREADS>, QF_AMAX_THREADS,
+                        QF_AMAX_WAVES, v, 256 * kAmaxU, d_group_amax, nullptr, d_tracked,
+                        n_groups, s);
+    if (st != QF_OK || !ragged) return st;
+    // scalar tails of tensors whose size is not a multiple of 8 elements
+    for (size_t b = 0; b < v.size(); b += kSmallT) {
+        const size_t cnt = std::min<size_t>(kSmallT, v.size() - b);
+        Table<kSmallT> P;
+        fill_table(P, v, b, cnt, 256 * kAmaxU);
+        P.group_amax = d_group_amax;
+        P.tracked = d_tracked;
+        P.n_groups = n_groups;
+        if (f32) qf::k_amax_tail<float, kSmallT><<<(unsigned)cnt, 32, 0, s>>>(P);
+        else qf::k_amax_tail<uint16_t, kSmallT><<<(unsigned)cnt, 32, 0, s>>>(P);
+    }
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+    return QF_OK;
+}
+
+// ------------------------------------------------------------------ one-shot NVFP4
+size_t oneshot_ws_bytes(int n_groups) {
+    const size_t b = sizeof(uint32_t) * ((size_t)qf::kOneshotHeaderWords + (size_t)n_groups);
+    return (b + 255) / 256 * 256;
+}
+
+// L2 size and cooperative-launch support of the current device, queried once per
+// host thread and device.
+struct DevProps { int dev; int l2; int coop; };
+qf_status dev_props(DevProps* D) {
+    thread_local std::vector<DevProps> cache;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    for (const DevProps& c : cache) {
+        if (c.dev == dev) {
+            *D = c;
+            return QF_OK;
+        }
+    }
+    DevProps d{dev, 0, 0};
+    e = cudaDeviceGetAttribute(&d.l2, cudaDevAttrL2CacheSize, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    e = cudaDeviceGetAttribute(&d.coop, cudaDevAttrCooperativeLaunch, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    cache.push_back(d);
+    *D = d;
+    return QF_OK;
+}
+
+template <typename XT, int MAXT>
+qf_status oneshot_launch(const std::vector<DevTensor>& v, float* am, float* tracked, float* so,
+                         int ng, uint32_t* ws, cudaStream_t s) {
+    constexpr int U = nvb_u<XT>();
+    auto kernel = qf::k_nv_oneshot<XT, U, MAXT, QF_ONESHOT_THREADS>;
+    Launch L;
+    qf_status st = launch_shape(kernel, QF_ONESHOT_THREADS, 1, &L);
+    if (st != QF_OK) return st;
+    Table<MAXT> P;
+    fill_table(P, v, 0, v.size(), 512 * U);
+    P.group_amax = am;
+    P.tracked = tracked;
+    P.group_scale_out = so;
+    P.n_groups = ng;
+    // at most one CTA per resident slot: every CTA must be resident for the barrier,
+    // which the cooperative launch guarantees (or refuses to launch)
+    const int grid = grid_for(L, P.total_units);
+    void* args[] = {&P, &ws};
+    cudaError_t e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kernel), dim3(grid),
+                                                dim3(QF_ONESHOT_THREADS), args, 0, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchCooperativeKernel");
+    return QF_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -419,7 +528,6 @@ qf_status qf_amax_tied(const qf_tensor* t, int n, float* d_group_amax, int n_gro
     if (n_groups <= 0) return fail(QF_ERR_INVALID_ARG, "n_groups = %d <= 0", n_groups);
     if (d_group_amax == nullptr) return fail(QF_ERR_INVALID_ARG, "d_group_amax is NULL");
     std::vector<DevTensor> v;
-    bool ragged = false;
     for (int i = 0; i < n; ++i) {
         qf_status st = check_tensor(t[i], i, 0, n_groups, true);
         if (st != QF_OK) return st;
@@ -431,38 +539,95 @@ qf_status qf_amax_tied(const qf_tensor* t, int n, float* d_group_amax, int n_gro
         d.x = t[i].x;
         d.numel = numel;
         d.group = t[i].group;
-        ragged |= (numel & 7) != 0;
         v.push_back(d);
     }
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaMemsetAsync(d_group_amax, 0, sizeof(float) * (size_t)n_groups, s);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
-    if (v.empty()) return QF_OK;
-    const bool f32 = t[0].x_type == QF_X_F32;
-    // the same bytes in flight per lane: 8 vectors of BF16, or 4 sub-tiles of FP32 (8 vectors)
-    qf_status st = f32
-        ? launch_chunks(qf::k_amax<float, kAmaxU / 2, kSmallT, QF_AMAX_THREADS>,
-                        qf::k_amax<float, kAmaxU / 2, kLargeT, QF_AMAX_THREADS>, QF_AMAX_THREADS,
-                        QF_AMAX_WAVES, v, 256 * (kAmaxU / 2), d_group_amax, nullptr, d_tracked,
-                        n_groups, s)
-        : launch_chunks(qf::k_amax<uint16_t, kAmaxU, kSmallT, QF_AMAX_THREADS>,
-                        qf::k_amax<uint16_t, kAmaxU, kLargeT, QF_AMAX_THREADS>, QF_AMAX_THREADS,
-                        QF_AMAX_WAVES, v, 256 * kAmaxU, d_group_amax, nullptr, d_tracked,
-                        n_groups, s);
-    if (st != QF_OK || !ragged) return st;
-    // scalar tails of tensors whose size is not a multiple of 8 elements
-    for (size_t b = 0; b < v.size(); b += kSmallT) {
-        const size_t cnt = std::min<size_t>(kSmallT, v.size() - b);
-        Table<kSmallT> P;
-        fill_table(P, v, b, cnt, 256 * kAmaxU);
-        P.group_amax = d_group_amax;
-        P.tracked = d_tracked;
-        P.n_groups = n_groups;
-        if (f32) qf::k_amax_tail<float, kSmallT><<<(unsigned)cnt, 32, 0, s>>>(P);
-        else qf::k_amax_tail<uint16_t, kSmallT><<<(unsigned)cnt, 32, 0, s>>>(P);
+    return amax_launch(v, n > 0 ? t[0].x_type : QF_X_BF16, d_group_amax, n_groups, d_tracked,
+                       static_cast<cudaStream_t>(stream));
+}
+
+size_t qf_amax_fakequant_workspace_bytes(int n_groups) {
+    return n_groups > 0 ? oneshot_ws_bytes(n_groups) : 0;
+}
+
+qf_status qf_amax_fakequant(const qf_tensor* t, int n, float* d_group_amax, int n_groups,
+                            float* d_tracked, float* d_group_scale_out, void* d_workspace,
+                            size_t workspace_bytes, void* stream) {
+    g_err[0] = 0;
+    if (n < 0) return fail(QF_ERR_INVALID_ARG, "n = %d < 0", n);
+    if (n > 0 && t == nullptr) return fail(QF_ERR_INVALID_ARG, "tensor array is NULL");
+    if (n_groups <= 0) return fail(QF_ERR_INVALID_ARG, "n_groups = %d <= 0", n_groups);
+    if (d_group_amax == nullptr) return fail(QF_ERR_INVALID_ARG, "d_group_amax is NULL");
+    if (d_workspace != nullptr) {
+        if (workspace_bytes < oneshot_ws_bytes(n_groups))
+            return fail(QF_ERR_INVALID_ARG, "workspace of %zu bytes < %zu needed for %d groups",
+                        workspace_bytes, oneshot_ws_bytes(n_groups), n_groups);
+        if (!aligned16(d_workspace)) return fail(QF_ERR_ALIGN, "workspace not 16-byte aligned");
     }
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+    // every check of qf_amax_tied and of qf_fakequant(QF_NVFP4) before anything launches
+    std::vector<DevTensor> v;
+    v.reserve(n);
+    int64_t in_bytes = 0;
+    for (int i = 0; i < n; ++i) {
+        qf_status st = check_tensor(t[i], i, 16, n_groups, true);
+        if (st != QF_OK) return st;
+        if (t[i].x_type != t[0].x_type)
+            return fail(QF_ERR_INVALID_ARG, "tensor %d: x_type differs from tensor 0's", i);
+        const int64_t numel = t[i].rows * t[i].cols;
+        if (numel == 0) continue;
+        if (!t[i].y && !t[i].codes && !t[i].scales)
+            return fail(QF_ERR_INVALID_ARG, "tensor %d: no output (y, codes, scales all NULL)", i);
+        if (!aligned16(t[i].y) || !aligned16(t[i].codes))
+            return fail(QF_ERR_ALIGN, "tensor %d: y / codes not 16-byte aligned", i);
+        DevTensor d{};
+        d.x = t[i].x;
+        d.y = static_cast<uint16_t*>(t[i].y);
+        d.codes = static_cast<uint8_t*>(t[i].codes);
+        d.scales = static_cast<uint8_t*>(t[i].scales);
+        d.numel = numel;
+        d.group = t[i].group;
+        v.push_back(d);
+        in_bytes += numel * (t[i].x_type == QF_X_F32 ? 4 : 2);
+    }
+    const int x_type = n > 0 ? t[0].x_type : QF_X_BF16;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    DevProps D;
+    qf_status st = dev_props(&D);
+    if (st != QF_OK) return st;
+    const bool one = d_workspace != nullptr && !v.empty() && v.size() <= (size_t)kLargeT &&
+                     D.coop && in_bytes * 3 <= (int64_t)D.l2;
+    if (one) {
+        uint32_t* ws = static_cast<uint32_t*>(d_workspace);
+        if (v.size() <= (size_t)kSmallT)
+            return x_type == QF_X_F32
+                ? oneshot_launch<float, kSmallT>(v, d_group_amax, d_tracked, d_group_scale_out,
+                                                 n_groups, ws, s)
+                : oneshot_launch<uint16_t, kSmallT>(v, d_group_amax, d_tracked, d_group_scale_out,
+                                                    n_groups, ws, s);
+        return x_type == QF_X_F32
+            ? oneshot_launch<float, kLargeT>(v, d_group_amax, d_tracked, d_group_scale_out, n_groups,
+                                             ws, s)
+            : oneshot_launch<uint16_t, kLargeT>(v, d_group_amax, d_tracked, d_group_scale_out,
+                                                n_groups, ws, s);
+    }
+    // two launches: the tie-group amax, then the fused pass on the scale it gives
+    st = amax_launch(v, x_type, d_group_amax, n_groups, d_tracked, s);
+    if (st != QF_OK) return st;
+    if (v.empty() && !d_group_scale_out) return QF_OK;
+    return launch_format(QF_NVFP4, 0, x_type, v, d_tracked ? d_tracked : d_group_amax,
+                         d_group_scale_out, n_groups, s);
+}
+
+qf_status qf_workspace_check(const void* d_workspace, void* stream) {
+    g_err[0] = 0;
+    if (d_workspace == nullptr) return fail(QF_ERR_INVALID_ARG, "workspace is NULL");
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    uint32_t err = 0;
+    e = cudaMemcpy(&err, static_cast<const uint32_t*>(d_workspace) + 2, sizeof err,
+                   cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy");
+    if (err & qf::kOneshotErrTimeout)
+        return fail(QF_ERR_TIMEOUT, "a grid barrier gave up waiting; clear the workspace before reuse");
     return QF_OK;
 }
 
@@ -532,12 +697,13 @@ const char* qf_status_string(qf_status s) {
         case QF_ERR_ALIGN: return "QF_ERR_ALIGN: pointer not 16-byte aligned";
         case QF_ERR_UNSUPPORTED: return "QF_ERR_UNSUPPORTED: unknown format or mode";
         case QF_ERR_CUDA: return "QF_ERR_CUDA: a CUDA call failed";
+        case QF_ERR_TIMEOUT: return "QF_ERR_TIMEOUT: a bounded device wait gave up";
     }
     return "unknown qf_status";
 }
 
 const char* qf_last_error(void) { return g_err; }
 
-int qf_version(void) { return (1 << 16) | 3; }
+int qf_version(void) { return (1 << 16) | 4; }
 
 }  // extern "C"

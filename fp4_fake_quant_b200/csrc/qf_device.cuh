@@ -51,7 +51,7 @@
 #define QF_NV_PREFETCH 1
 #endif
 #ifndef QF_NVB_THREADS
-#define QF_NVB_THREADS 256      // NVFP4 fused pass, one lane per block (k_nv)
+#define QF_NVB_THREADS 128      // NVFP4 fused pass, one lane per block (k_nv)
 #endif
 #ifndef QF_NVB_WAVES
 #define QF_NVB_WAVES 1000
@@ -78,10 +78,13 @@
 #define QF_AMAX_THREADS 256
 #endif
 #ifndef QF_AMAX_WAVES
-#define QF_AMAX_WAVES 1
+#define QF_AMAX_WAVES 1000
 #endif
 #ifndef QF_AMAX_LD
 #define QF_AMAX_LD 0
+#endif
+#ifndef QF_AMAX_ORDER
+#define QF_AMAX_ORDER 0         // 0: one contiguous unit range per CTA, 1: grid-stride sweep
 #endif
 #ifndef QF_ST_POLICY
 #define QF_ST_POLICY 0          // 0: default write-back stores, 1: streaming (.cs) stores
@@ -474,6 +477,62 @@ __global__ void __launch_bounds__(THREADS) k_fp4(const __grid_constant__ Table<M
 // they cover whole sectors; the later ones are served from L1) and writes 32 bytes
 // of BF16, 8 bytes of codes and 1 scale byte: the warp's code and scale stores are
 // contiguous 256- and 32-byte runs.
+template <typename XT, int U, int LD>
+__device__ __forceinline__ void nv_load_unit(const DevTensor& T, int64_t e0, int lane,
+                                             Elems<XT, 16> (&v)[U]) {
+    const XT* x = static_cast<const XT*>(T.x);
+#pragma unroll
+    for (int s = 0; s < U; ++s) {
+        const int64_t e = e0 + s * 512 + lane * 16;
+        v[s].template load<LD>(x + e, e < T.numel);
+    }
+}
+
+// Encode one warp unit (U sub-tiles of 512 elements starting at element e0).
+template <typename XT, int U>
+__device__ __forceinline__ void nv_encode_unit(const DevTensor& T, int64_t e0, int lane,
+                                               const Elems<XT, 16> (&cur)[U], float s_t,
+                                               float six_st) {
+#pragma unroll
+    for (int s = 0; s < U; ++s) {
+        const int64_t e = e0 + s * 512 + lane * 16;
+        const Elems<XT, 16>& x = cur[s];
+        uint32_t sb;
+        float S, inv;
+        nv_block_scale(__uint_as_float(x.amax_bits()), s_t, six_st, sb, S, inv);
+        float q[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) q[k] = __fmul_rn(x.get(k), inv);
+        if (__builtin_expect(isinf(inv), 0)) {
+            // 1/S overflowed (S < 2^-128): a zero keeps its own sign instead of 0 * inf
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+                if (x.get(k) == 0.0f) q[k] = x.get(k);
+        }
+        uint32_t b[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) b[k] = cvt_e2m1x2(q[2 * k + 1], q[2 * k]);
+        if (e < T.numel) {
+            if (T.y) {
+                uint32_t yw[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t h2 = cvt_e2m1x2_f16x2(b[k]);
+                    yw[k] = cvt_bf16x2(__fmul_rn(f16_hi(h2), S), __fmul_rn(f16_lo(h2), S));
+                }
+                st_v4(T.y + e, make_uint4(yw[0], yw[1], yw[2], yw[3]));
+                st_v4(T.y + e + 8, make_uint4(yw[4], yw[5], yw[6], yw[7]));
+            }
+            if (T.codes) {
+                const uint32_t lo = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
+                const uint32_t hi = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
+                *reinterpret_cast<uint2*>(T.codes + (e >> 1)) = make_uint2(lo, hi);
+            }
+            if (T.scales) T.scales[e >> 4] = (uint8_t)sb;
+        }
+    }
+}
+
 template <typename XT, int U, int MAXT, int THREADS, int PREFETCH>
 __global__ void __launch_bounds__(THREADS) k_nv(const __grid_constant__ Table<MAXT> P) {
     const int lane = threadIdx.x & 31;
@@ -488,15 +547,7 @@ __global__ void __launch_bounds__(THREADS) k_nv(const __grid_constant__ Table<MA
     if (u >= P.total_units) return;
     int ti = locate_tensor(P, u);
     Elems<XT, 16> cur[U], nxt[U];
-    auto load = [&](const DevTensor& T, int64_t e0, Elems<XT, 16> (&v)[U]) {
-        const XT* x = static_cast<const XT*>(T.x);
-#pragma unroll
-        for (int s = 0; s < U; ++s) {
-            const int64_t e = e0 + s * 512 + lane * 16;
-            v[s].template load<QF_FP4_LD>(x + e, e < T.numel);
-        }
-    };
-    load(P.t[ti], (u - P.t[ti].unit_begin) * kUnit, cur);
+    nv_load_unit<XT, U, QF_FP4_LD>(P.t[ti], (u - P.t[ti].unit_begin) * kUnit, lane, cur);
     int cur_t = -1;
     float s_t = 0.0f, six_st = 0.0f;
     while (true) {
@@ -504,7 +555,7 @@ __global__ void __launch_bounds__(THREADS) k_nv(const __grid_constant__ Table<MA
         int tn = ti;
         if (PREFETCH && un < P.total_units) {
             tn = find_tensor(P, ti, un);
-            load(P.t[tn], (un - P.t[tn].unit_begin) * kUnit, nxt);
+            nv_load_unit<XT, U, QF_FP4_LD>(P.t[tn], (un - P.t[tn].unit_begin) * kUnit, lane, nxt);
         }
         const DevTensor& T = P.t[ti];
         if (ti != cur_t) {
@@ -512,45 +563,7 @@ __global__ void __launch_bounds__(THREADS) k_nv(const __grid_constant__ Table<MA
             six_st = __fmul_rn(6.0f, s_t);
             cur_t = ti;
         }
-        const int64_t e0 = (u - T.unit_begin) * kUnit;
-#pragma unroll
-        for (int s = 0; s < U; ++s) {
-            const int64_t e = e0 + s * 512 + lane * 16;
-            const Elems<XT, 16>& x = cur[s];
-            uint32_t sb;
-            float S, inv;
-            nv_block_scale(__uint_as_float(x.amax_bits()), s_t, six_st, sb, S, inv);
-            float q[16];
-#pragma unroll
-            for (int k = 0; k < 16; ++k) q[k] = __fmul_rn(x.get(k), inv);
-            if (__builtin_expect(isinf(inv), 0)) {
-                // 1/S overflowed (S < 2^-128): a zero keeps its own sign instead of 0 * inf
-#pragma unroll
-                for (int k = 0; k < 16; ++k)
-                    if (x.get(k) == 0.0f) q[k] = x.get(k);
-            }
-            uint32_t b[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) b[k] = cvt_e2m1x2(q[2 * k + 1], q[2 * k]);
-            if (e < T.numel) {
-                if (T.y) {
-                    uint32_t yw[8];
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const uint32_t h2 = cvt_e2m1x2_f16x2(b[k]);
-                        yw[k] = cvt_bf16x2(__fmul_rn(f16_hi(h2), S), __fmul_rn(f16_lo(h2), S));
-                    }
-                    st_v4(T.y + e, make_uint4(yw[0], yw[1], yw[2], yw[3]));
-                    st_v4(T.y + e + 8, make_uint4(yw[4], yw[5], yw[6], yw[7]));
-                }
-                if (T.codes) {
-                    const uint32_t lo = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
-                    const uint32_t hi = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
-                    *reinterpret_cast<uint2*>(T.codes + (e >> 1)) = make_uint2(lo, hi);
-                }
-                if (T.scales) T.scales[e >> 4] = (uint8_t)sb;
-            }
-        }
+        nv_encode_unit<XT, U>(T, (u - T.unit_begin) * kUnit, lane, cur, s_t, six_st);
         if (un >= P.total_units) break;
         u = un;
         if (PREFETCH) {
@@ -559,7 +572,7 @@ __global__ void __launch_bounds__(THREADS) k_nv(const __grid_constant__ Table<MA
             for (int i = 0; i < U; ++i) cur[i] = nxt[i];
         } else {
             ti = find_tensor(P, ti, u);
-            load(P.t[ti], (u - P.t[ti].unit_begin) * kUnit, cur);
+            nv_load_unit<XT, U, QF_FP4_LD>(P.t[ti], (u - P.t[ti].unit_begin) * kUnit, lane, cur);
         }
     }
 }
@@ -832,25 +845,38 @@ __global__ void __launch_bounds__(THREADS) k_amax(const __grid_constant__ Table<
     const int lane = threadIdx.x & 31;
     constexpr int kUnit = 256 * U;
     constexpr int kWarps = THREADS / 32;
+#if QF_AMAX_ORDER == 0
     const int64_t per_cta = (P.total_units + gridDim.x - 1) / gridDim.x;
     const int64_t u_begin = int64_t(blockIdx.x) * per_cta;
     const int64_t u_end = min(u_begin + per_cta, P.total_units);
-    float* amax = const_cast<float*>(P.group_amax);
     const int64_t u_first = u_begin + (threadIdx.x >> 5);
+    constexpr int64_t u_step = kWarps;
+#else
+    const int64_t u_end = P.total_units;
+    const int64_t u_first = int64_t(blockIdx.x) * kWarps + (threadIdx.x >> 5);
+    const int64_t u_step = int64_t(gridDim.x) * kWarps;
+#endif
+    float* amax = const_cast<float*>(P.group_amax);
     int ti = u_first < u_end ? locate_tensor(P, u_first) : 0;
     int g = -1;
     uint32_t run = 0;
-    auto flush = [&](int grp) {
+    auto warp_max = [&]() {
         uint32_t a = run;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) a = max(a, __shfl_xor_sync(kFull, a, o));
-        if (lane == 0 && grp >= 0) {
-            atomicMax(reinterpret_cast<unsigned int*>(amax) + grp, a);
-            if (P.tracked) atomicMax(reinterpret_cast<unsigned int*>(P.tracked) + grp, a);
-        }
+        return a;
+    };
+    auto publish = [&](int grp, uint32_t a) {
+        atomicMax(reinterpret_cast<unsigned int*>(amax) + grp, a);
+        if (P.tracked) atomicMax(reinterpret_cast<unsigned int*>(P.tracked) + grp, a);
+    };
+    // a warp that moves on to another tie group publishes the finished one at once
+    auto flush = [&](int grp) {
+        const uint32_t a = warp_max();
+        if (lane == 0 && grp >= 0) publish(grp, a);
         run = 0;
     };
-    for (int64_t u = u_first; u < u_end; u += kWarps) {
+    for (int64_t u = u_first; u < u_end; u += u_step) {
         ti = find_tensor(P, ti, u);
         const DevTensor& T = P.t[ti];
         if (T.group != g) {
@@ -868,7 +894,28 @@ __global__ void __launch_bounds__(THREADS) k_amax(const __grid_constant__ Table<
 #pragma unroll
         for (int s = 0; s < U; ++s) run = max(run, v[s].amax_bits());
     }
-    if (g >= 0) flush(g);
+    // The warps' last groups are combined in the CTA first: when every CTA ends at
+    // about the same time, thousands of same-address atomics would otherwise queue
+    // at the end of the kernel (one per CTA and group remains).
+    __shared__ int wgrp[kWarps];
+    __shared__ uint32_t wmax[kWarps];
+    const uint32_t a = warp_max();
+    if (lane == 0) {
+        wgrp[threadIdx.x >> 5] = g;
+        wmax[threadIdx.x >> 5] = a;
+    }
+    __syncthreads();
+    if (threadIdx.x < kWarps) {
+        const int w = threadIdx.x, gw = wgrp[w];
+        bool first = gw >= 0;                       // first warp of the CTA with this group
+        uint32_t m = wmax[w];
+        for (int o = 0; o < kWarps; ++o) {
+            if (wgrp[o] != gw) continue;
+            if (o < w) first = false;
+            m = max(m, wmax[o]);
+        }
+        if (first) publish(gw, m);
+    }
 }
 
 // amax of tensors whose element count is not a multiple of 8 handles the

@@ -236,10 +236,18 @@ __global__ void __launch_bounds__(kLoraThreads) k_lora(const __grid_constant__ L
         for (int h = 0; h < 4; ++h) wcur[h] = wnxt[h];
     }
     if (MODE == kLoraAmax) {
+        // one atomic per CTA (its unit lies in one tensor), not one per warp
+        __shared__ uint32_t wmax[kLoraThreads / 32];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) run = max(run, __shfl_xor_sync(kFull, run, o));
-        if (lane == 0 && run != 0)
-            atomicMax(reinterpret_cast<unsigned int*>(const_cast<float*>(P.group_amax)) + T.group, run);
+        if (lane == 0) wmax[wid] = run;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            for (int w = 1; w < kLoraThreads / 32; ++w) run = max(run, wmax[w]);
+            if (run != 0)
+                atomicMax(reinterpret_cast<unsigned int*>(const_cast<float*>(P.group_amax)) + T.group,
+                          run);
+        }
     }
 }
 

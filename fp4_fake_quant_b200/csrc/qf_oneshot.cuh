@@ -1,0 +1,194 @@
+// qf_oneshot.cuh -- NVFP4 tie-group amax and fake-quant + pack in ONE launch, for calls
+// whose inputs fit in L2 (sm_100a: 126 MB).
+//
+// NVFP4 needs the FP32 tensor scale s_t = amax_g / 2688 of a whole tie group before
+// any block can be encoded (QATFactory project page, Method, "Numerics": one
+// tensor-level scale shared by the fused projections), so the plain path is two
+// launches that both read the input from HBM.  For an input that fits in L2 this
+// kernel runs both phases in one cooperative launch:
+//   phase 1  every CTA reads its units from HBM and folds max |x| into per-group
+//            slots of a device workspace (atomicMax on the FP32 bits, after a
+//            CTA-level combine);
+//   barrier  a grid-wide arrive counter; all CTAs are co-resident (cooperative launch),
+//            and the wait is bounded: after kOneshotSpinLimit polls the CTA sets the
+//            workspace's error word and returns without writing its outputs;
+//   phase 2  every CTA re-reads the same units -- now L2 hits -- and encodes them
+//            exactly as k_nv does.
+// The last CTA to finish resets the workspace (slots and counters) to zero, so a
+// zeroed workspace stays valid for the next call on the same stream.
+//
+// Workspace layout (32-bit words): [0] arrive count, [1] depart count, [2] error
+// flags, [3] unused, [4 + g] group g's running max |x| as FP32 bits.
+#pragma once
+
+#include "qf_device.cuh"
+
+namespace qf {
+
+constexpr int kOneshotHeaderWords = 4;
+constexpr uint32_t kOneshotSpinLimit = 1u << 22;    // polls, ~256 ns apart: about a second
+constexpr uint32_t kOneshotErrTimeout = 1u;
+#ifndef QF_ONESHOT_THREADS
+#define QF_ONESHOT_THREADS 256
+#endif
+#ifndef QF_ONESHOT_MINB
+#define QF_ONESHOT_MINB 1       // minimum resident CTAs per SM asked of the register allocator
+#endif
+#ifndef QF_ONESHOT_PF
+#define QF_ONESHOT_PF 0         // 1: the encode pass loads the next unit while encoding this one
+#endif
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ uint32_t ld_relaxed_gpu(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// P.group_amax: output, this call's tie-group amax.  P.tracked (nullable): running
+// amax, max-accumulated in place; when given, s_t comes from the updated running
+// value (the activation reading), otherwise from this call's amax.
+// P.group_scale_out (nullable): s_t per group.
+template <typename XT, int U, int MAXT, int THREADS>
+__global__ void __launch_bounds__(THREADS, QF_ONESHOT_MINB)
+    k_nv_oneshot(const __grid_constant__ Table<MAXT> P, uint32_t* __restrict__ ws) {
+    constexpr int kWarps = THREADS / 32;
+    constexpr int kUnit = 512 * U;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int64_t warp = int64_t(blockIdx.x) * kWarps + wid;
+    const int64_t nwarps = int64_t(gridDim.x) * kWarps;
+    uint32_t* slot = ws + kOneshotHeaderWords;
+
+    // ---- phase 1: max |x| per tie group over this warp's units
+    int ti = warp < P.total_units ? locate_tensor(P, warp) : 0;
+    int g = -1;
+    uint32_t run = 0;
+    auto warp_max = [&]() {
+        uint32_t a = run;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) a = max(a, __shfl_xor_sync(kFull, a, o));
+        return a;
+    };
+    for (int64_t u = warp; u < P.total_units; u += nwarps) {
+        ti = find_tensor(P, ti, u);
+        const DevTensor& T = P.t[ti];
+        if (T.group != g) {
+            const uint32_t a = warp_max();
+            if (lane == 0 && g >= 0) atomicMax(slot + g, a);
+            run = 0;
+            g = T.group;
+        }
+        Elems<XT, 16> v[U];
+        nv_load_unit<XT, U, 1>(T, (u - T.unit_begin) * kUnit, lane, v);
+#pragma unroll
+        for (int s = 0; s < U; ++s) run = max(run, v[s].amax_bits());
+    }
+    __shared__ int wgrp[kWarps];
+    __shared__ uint32_t wmax[kWarps];
+    __shared__ int s_flag;
+    {
+        const uint32_t a = warp_max();
+        if (lane == 0) {
+            wgrp[wid] = g;
+            wmax[wid] = a;
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x < kWarps) {
+        const int w = threadIdx.x, gw = wgrp[w];
+        bool first = gw >= 0;
+        uint32_t m = wmax[w];
+        for (int o = 0; o < kWarps; ++o) {
+            if (wgrp[o] != gw) continue;
+            if (o < w) first = false;
+            m = max(m, wmax[o]);
+        }
+        if (first) atomicMax(slot + gw, m);
+    }
+    __syncthreads();
+
+    // ---- grid barrier (bounded)
+    if (threadIdx.x == 0) {
+        __threadfence();                                    // this CTA's slot updates first
+        atomicAdd(ws + 0, 1u);
+        uint32_t polls = 0;
+        bool done = ld_acquire_gpu(ws + 0) >= gridDim.x;
+        while (!done && ++polls < kOneshotSpinLimit) {
+            __nanosleep(256);
+            done = ld_acquire_gpu(ws + 0) >= gridDim.x;
+        }
+        if (!done) atomicOr(ws + 2, kOneshotErrTimeout);
+        s_flag = done;
+    }
+    __syncthreads();
+    if (!s_flag) return;                                    // outputs left unwritten
+
+    // ---- group statistics out (CTA 0)
+    auto eff_amax = [&](int grp) {
+        float a = __uint_as_float(ld_relaxed_gpu(slot + grp));
+        if (P.tracked) a = fmaxf(a, P.tracked[grp]);
+        return a;
+    };
+    if (blockIdx.x == 0) {
+        for (int q = threadIdx.x; q < P.n_groups; q += THREADS) {
+            const float cur = __uint_as_float(ld_relaxed_gpu(slot + q));
+            const float e = eff_amax(q);
+            const_cast<float*>(P.group_amax)[q] = cur;
+            if (P.tracked) P.tracked[q] = e;
+            if (P.group_scale_out) P.group_scale_out[q] = nv_tensor_scale(e);
+        }
+    }
+
+    // ---- phase 2: encode the same units (their lines are in L2 now)
+    if (warp < P.total_units) {
+        ti = locate_tensor(P, warp);
+        int cur_t = -1;
+        float s_t = 0.0f, six_st = 0.0f;
+        Elems<XT, 16> v[U], nx[U];
+        if (QF_ONESHOT_PF) nv_load_unit<XT, U, 1>(P.t[ti], (warp - P.t[ti].unit_begin) * kUnit, lane, v);
+        for (int64_t u = warp; u < P.total_units; u += nwarps) {
+            ti = find_tensor(P, ti, u);
+            const DevTensor& T = P.t[ti];
+            if (ti != cur_t) {
+                s_t = nv_tensor_scale(eff_amax(T.group));
+                six_st = __fmul_rn(6.0f, s_t);
+                cur_t = ti;
+            }
+            const int64_t e0 = (u - T.unit_begin) * kUnit;
+            if (QF_ONESHOT_PF) {
+                const int64_t un = u + nwarps;
+                if (un < P.total_units) {
+                    const int tn = find_tensor(P, ti, un);
+                    nv_load_unit<XT, U, 1>(P.t[tn], (un - P.t[tn].unit_begin) * kUnit, lane, nx);
+                }
+                nv_encode_unit<XT, U>(T, e0, lane, v, s_t, six_st);
+#pragma unroll
+                for (int i = 0; i < U; ++i) v[i] = nx[i];
+            } else {
+                nv_load_unit<XT, U, 1>(T, e0, lane, v);
+                nv_encode_unit<XT, U>(T, e0, lane, v, s_t, six_st);
+            }
+        }
+    }
+
+    // ---- depart; the last CTA out leaves the workspace zeroed for the next call
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        s_flag = atomicAdd(ws + 1, 1u) == gridDim.x - 1;
+    }
+    __syncthreads();
+    if (s_flag) {
+        for (int q = threadIdx.x; q < P.n_groups; q += THREADS) slot[q] = 0u;
+        if (threadIdx.x == 0) {
+            ws[0] = 0u;
+            ws[1] = 0u;
+        }
+    }
+}
+
+}  // namespace qf

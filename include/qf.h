@@ -34,7 +34,9 @@
  *     is asynchronous on that stream.
  *   - Arguments are validated on the host before anything is launched; an
  *     invalid call returns an error status and launches nothing.  A CUDA launch
- *     failure returns QF_ERR_CUDA.  Kernels never trap and contain no waits.
+ *     failure returns QF_ERR_CUDA.  Kernels never trap.  The one wait in the
+ *     library is the grid barrier of qf_amax_fakequant's single-launch path,
+ *     which is bounded (see there).
  *     qf_last_error() gives a one-line description of the last failure on the
  *     calling thread.
  *   - Calls on the same stream are ordered; calls whose outputs overlap and that
@@ -45,6 +47,7 @@
 #ifndef QF_H
 #define QF_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -64,7 +67,8 @@ typedef enum {
     QF_ERR_SHAPE = 2,         /* negative or overflowing size, cols not a block multiple */
     QF_ERR_ALIGN = 3,         /* x / y / codes not 16-byte aligned */
     QF_ERR_UNSUPPORTED = 4,   /* unknown format or mode */
-    QF_ERR_CUDA = 5           /* a CUDA call failed (see qf_last_error) */
+    QF_ERR_CUDA = 5,          /* a CUDA call failed (see qf_last_error) */
+    QF_ERR_TIMEOUT = 6        /* a bounded device wait gave up (qf_workspace_check) */
 } qf_status;
 
 /* Element type of the input x (qf_tensor.x_type). */
@@ -173,6 +177,56 @@ qf_status qf_fakequant(qf_format f, const qf_tensor* t, int n, const float* d_gr
                        int n_groups, float* d_group_scale_out, void* stream);
 
 /*
+ * qf_amax_fakequant -- NVFP4 tie-group amax and fused fake-quant + pack in one call:
+ * the results of qf_amax_tied followed by qf_fakequant(QF_NVFP4, ...) on the
+ * scale it gives, bit for bit.  The tensor scale needs the amax of the whole tie
+ * group before any block is encoded (project page, Method, "Numerics": one FP32
+ * tensor scale per fused projection group), which costs a second pass over x.
+ *
+ * When every input fits comfortably in L2 (all x bytes <= L2 size / 3: up to
+ * about 44 MB on a B200), a workspace is given, n <= 384 and the device supports
+ * cooperative launches, both passes run in ONE cooperative launch.  The first
+ * pass reads x from HBM and folds max |x| into the workspace.  A grid-wide
+ * barrier follows.  The second pass re-reads x from L2 and encodes it.
+ * Otherwise, or with d_workspace == NULL, the call makes the two launches of
+ * qf_amax_tied and qf_fakequant.
+ *
+ *   t, n, n_groups     as for qf_fakequant with QF_NVFP4 (every check of
+ *                      qf_amax_tied and qf_fakequant is made before any launch).
+ *   d_group_amax       FP32[n_groups], overwritten with this call's group amax.
+ *   d_tracked          NULL, or FP32[n_groups] running amax, updated in place to
+ *                      max(d_tracked[g], amax_g); when given, s_t is taken from
+ *                      the updated running value (activations), otherwise from
+ *                      amax_g (weights).
+ *   d_group_scale_out  NULL, or FP32[n_groups] receiving each s_t.
+ *   d_workspace        NULL, or device memory of at least
+ *                      qf_amax_fakequant_workspace_bytes(n_groups) bytes,
+ *                      16-byte aligned, ALL ZERO before its first use (e.g.
+ *                      cudaMemset once).  Every call that completes leaves it zero
+ *                      again, so it can be reused by later calls on the same stream.
+ *                      Calls that may overlap (different streams) need their own
+ *                      workspaces.
+ *   workspace_bytes    its size.
+ * The barrier wait is bounded (about a second of polling).  A CTA that gives up
+ * sets an error flag in the workspace and writes none of its outputs.
+ * qf_workspace_check then reports QF_ERR_TIMEOUT, and the workspace must be
+ * zeroed again before reuse.  A cooperative launch guarantees that every CTA is
+ * resident, so the wait completes unless a CTA faults.
+ * Errors: as qf_fakequant; a workspace smaller than needed -> QF_ERR_INVALID_ARG,
+ *   not 16-byte aligned -> QF_ERR_ALIGN.
+ */
+qf_status qf_amax_fakequant(const qf_tensor* t, int n, float* d_group_amax, int n_groups,
+                            float* d_tracked, float* d_group_scale_out, void* d_workspace,
+                            size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace qf_amax_fakequant needs for n_groups tie groups (0 if n_groups <= 0). */
+size_t qf_amax_fakequant_workspace_bytes(int n_groups);
+
+/* Synchronizes `stream`, then reads the error flags of a qf_amax_fakequant
+ * workspace: QF_OK, or QF_ERR_TIMEOUT if a grid barrier gave up. */
+qf_status qf_workspace_check(const void* d_workspace, void* stream);
+
+/*
  * qf_pack -- the engine-layout export and weight sync (project page, Method,
  * "QARL": after every optimizer step the trainer writes its weights in the
  * engine's byte layout and hands them over; "Export").  Identical to qf_fakequant except that y is never
@@ -267,7 +321,7 @@ const char* qf_last_error(void);
 
 /* ABI version: (major << 16) | minor.  1.1 added qf_tensor.x_type (formerly a
  * reserved field that had to be 0, which still means BF16); 1.2 the LoRA calls;
- * 1.3 QF_Q4K_MSE. */
+ * 1.3 QF_Q4K_MSE; 1.4 qf_amax_fakequant, its workspace calls and QF_ERR_TIMEOUT. */
 int qf_version(void);
 
 #ifdef __cplusplus

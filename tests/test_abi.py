@@ -56,9 +56,9 @@ def test_struct_layout_matches_header(qf):
 
 
 def test_status_strings(qf):
-    for s in range(6):
+    for s in range(7):
         assert qf.lib.qf_status_string(s).decode().startswith("QF_")
-    assert qf.lib.qf_version() == (1 << 16) | 3
+    assert qf.lib.qf_version() == (1 << 16) | 4
 
 
 def _tensor(qf, x=0x1000, rows=4, cols=64, group=0, y=0x2000, codes=0x3000, scales=0x4000,
@@ -132,6 +132,36 @@ def test_amax_and_ste_validation(qf):
     assert lib.qf_ste_backward(1, 0x1000, 0x2000, 256, 1, None, None, 0, None) == INV
     assert lib.qf_ste_backward(1, 0x1000, 0x2000, 255, 1, _tensor(qf), None, 0, None) == SHAPE
     assert lib.qf_ste_backward(0, 0x1000, 0x2000, 256, 1, _tensor(qf), None, 1, None) == INV
+
+
+def test_amax_fakequant_validation(qf):
+    """qf_amax_fakequant makes every check of qf_amax_tied and qf_fakequant(NVFP4),
+    plus its workspace checks, before anything launches."""
+    INV, SHAPE, ALIGN = 1, 2, 3
+    lib = qf.lib
+    wb = lib.qf_amax_fakequant_workspace_bytes
+    assert wb(0) == 0 and wb(-3) == 0
+    assert wb(1) == 256 and wb(60) == 256 and wb(61) == 512      # 4 header words + 1 per group
+    assert qf.workspace_bytes(256) == 1280
+
+    def call(arr, n=1, amax=0x5000, ng=1, ws=0x9000, wsb=256):
+        return lib.qf_amax_fakequant(arr, n, amax, ng, None, None, ws, wsb, None)
+
+    assert call(_tensor(qf), n=-1) == INV
+    assert call(None) == INV
+    assert call(_tensor(qf), ng=0) == INV
+    assert call(_tensor(qf), amax=None) == INV
+    assert call(_tensor(qf), wsb=255) == INV                       # workspace too small
+    assert call(_tensor(qf), ng=61, wsb=256) == INV
+    assert call(_tensor(qf), ws=0x9008) == ALIGN
+    assert call(_tensor(qf, cols=24)) == SHAPE                     # NVFP4 needs 16 | cols
+    assert call(_tensor(qf, group=1)) == INV
+    assert call(_tensor(qf, y=0, codes=0, scales=0)) == INV
+    assert call(_tensor(qf, codes=0x3004)) == ALIGN
+    assert call(_tensor(qf, x=0x1008)) == ALIGN
+    two = (qf.binding.QfTensor * 2)(_tensor(qf)[0], _tensor(qf, x_type=1)[0])
+    assert call(two, n=2) == INV
+    assert lib.qf_workspace_check(None, None) == INV
 
 
 def test_product_path_has_no_oracle_dependency():
