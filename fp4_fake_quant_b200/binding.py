@@ -63,9 +63,10 @@ def _load() -> ctypes.CDLL:
     lib.qf_amax_fakequant_workspace_bytes.argtypes = [I]
     lib.qf_amax_fakequant_workspace_bytes.restype = ctypes.c_size_t
     lib.qf_workspace_check.argtypes = [P, P]
+    lib.qf_amax_fakequant_noalloc.argtypes = [T, I, P, I, P, P, P]
     for f in (lib.qf_amax_tied, lib.qf_fakequant, lib.qf_pack, lib.qf_ste_backward,
               lib.qf_lora_merge, lib.qf_amax_tied_lora, lib.qf_fakequant_lora,
-              lib.qf_amax_fakequant, lib.qf_workspace_check):
+              lib.qf_amax_fakequant, lib.qf_workspace_check, lib.qf_amax_fakequant_noalloc):
         f.restype = I
     lib.qf_status_string.argtypes = [I]
     lib.qf_status_string.restype = ctypes.c_char_p
@@ -81,7 +82,8 @@ lib = _load()
 # the entry points declared in include/qf.h
 EXPORTS = ("qf_amax_tied", "qf_fakequant", "qf_pack", "qf_ste_backward", "qf_lora_merge",
            "qf_amax_tied_lora", "qf_fakequant_lora", "qf_amax_fakequant",
-           "qf_amax_fakequant_workspace_bytes", "qf_workspace_check", "qf_status_string",
+           "qf_amax_fakequant_workspace_bytes", "qf_workspace_check",
+           "qf_amax_fakequant_noalloc", "qf_status_string",
            "qf_last_error", "qf_version")
 
 
@@ -253,6 +255,15 @@ def prepare_amax_fakequant(xs, ys=None, codes=None, scales=None, groups=None, gr
     return Prepared(lib.qf_amax_fakequant,
                     (arr, n, _ptr(group_amax), group_amax.numel(), _ptr(tracked),
                      _ptr(group_scale_out), _ptr(workspace), wsb), keep)
+
+
+def qf_amax_fakequant_noalloc(xs, ys=None, codes=None, scales=None, groups=None,
+                              group_amax=None, tracked=None, group_scale_out=None,
+                              stream=None) -> None:
+    """qf_amax_fakequant on the library's static device workspace (nothing allocated)."""
+    arr, n = _desc(xs, ys, codes, scales, groups)
+    _check(lib.qf_amax_fakequant_noalloc(arr, n, _ptr(group_amax), group_amax.numel(),
+                                         _ptr(tracked), _ptr(group_scale_out), _stream(stream)))
 
 
 def qf_workspace_check(workspace: torch.Tensor, stream=None) -> None:

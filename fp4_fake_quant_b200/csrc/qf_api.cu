@@ -7,6 +7,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 #include "qf.h"
@@ -27,6 +28,9 @@ constexpr int kFp4U = QF_FP4_U;  // 256-element sub-tiles per warp unit
 #define QF_AMAX_U 4
 #endif
 constexpr int kAmaxU = QF_AMAX_U;
+#ifndef QF_NOALLOC_MAX_GROUPS
+#define QF_NOALLOC_MAX_GROUPS 4092     // 4 header words + 4092 slots = 16 KB of static scratch
+#endif
 
 thread_local char g_err[512] = "";
 
@@ -456,6 +460,36 @@ qf_status oneshot_launch(const std::vector<DevTensor>& v, float* am, float* trac
     return QF_OK;
 }
 
+// ------------------------------------------------------------------ static scratch
+// The workspace of qf_amax_fakequant_noalloc: module-level device memory, one copy per
+// device, never allocated at run time.  Capacity: the header words plus one word per
+// tie group, for up to QF_NOALLOC_MAX_GROUPS groups.
+constexpr int kNoallocWords = qf::kOneshotHeaderWords + QF_NOALLOC_MAX_GROUPS;
+__device__ __align__(256) uint32_t g_noalloc_ws[kNoallocWords];
+
+// Its address on the current device, looked up once per device (with that device
+// current, as cudaGetSymbolAddress requires) and kept.
+qf_status noalloc_ws(void** out) {
+    static std::mutex mu;
+    static std::vector<std::pair<int, void*>> addr;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    std::lock_guard<std::mutex> lock(mu);
+    for (const auto& a : addr) {
+        if (a.first == dev) {
+            *out = a.second;
+            return QF_OK;
+        }
+    }
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_ws);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+    addr.emplace_back(dev, p);
+    *out = p;
+    return QF_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -617,6 +651,42 @@ qf_status qf_amax_fakequant(const qf_tensor* t, int n, float* d_group_amax, int 
                          d_group_scale_out, n_groups, s);
 }
 
+qf_status qf_amax_fakequant_noalloc(const qf_tensor* t, int n, float* d_group_amax,
+                                    int n_groups, float* d_tracked, float* d_group_scale_out,
+                                    void* stream) {
+    g_err[0] = 0;
+    if (n_groups > QF_NOALLOC_MAX_GROUPS)
+        return fail(QF_ERR_INVALID_ARG, "n_groups = %d exceeds the static workspace (%d groups)",
+                    n_groups, QF_NOALLOC_MAX_GROUPS);
+    if (n_groups <= 0) return fail(QF_ERR_INVALID_ARG, "n_groups = %d <= 0", n_groups);
+    // the argument checks of qf_amax_fakequant, made here too so that an invalid call
+    // enqueues nothing (not even the clearing of the workspace)
+    if (n < 0) return fail(QF_ERR_INVALID_ARG, "n = %d < 0", n);
+    if (n > 0 && t == nullptr) return fail(QF_ERR_INVALID_ARG, "tensor array is NULL");
+    if (d_group_amax == nullptr) return fail(QF_ERR_INVALID_ARG, "d_group_amax is NULL");
+    for (int i = 0; i < n; ++i) {
+        qf_status st = check_tensor(t[i], i, 16, n_groups, true);
+        if (st != QF_OK) return st;
+        if (t[i].x_type != t[0].x_type)
+            return fail(QF_ERR_INVALID_ARG, "tensor %d: x_type differs from tensor 0's", i);
+        if (t[i].rows * t[i].cols == 0) continue;
+        if (!t[i].y && !t[i].codes && !t[i].scales)
+            return fail(QF_ERR_INVALID_ARG, "tensor %d: no output (y, codes, scales all NULL)", i);
+        if (!aligned16(t[i].y) || !aligned16(t[i].codes))
+            return fail(QF_ERR_ALIGN, "tensor %d: y / codes not 16-byte aligned", i);
+    }
+    void* ws = nullptr;
+    qf_status st = noalloc_ws(&ws);
+    if (st != QF_OK) return st;
+    // the part of the workspace this call uses must start at zero: clear it on the
+    // call's stream, whatever an earlier call (or a timed-out one) left there
+    const size_t bytes = oneshot_ws_bytes(n_groups);
+    cudaError_t e = cudaMemsetAsync(ws, 0, bytes, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+    return qf_amax_fakequant(t, n, d_group_amax, n_groups, d_tracked, d_group_scale_out, ws, bytes,
+                             stream);
+}
+
 qf_status qf_workspace_check(const void* d_workspace, void* stream) {
     g_err[0] = 0;
     if (d_workspace == nullptr) return fail(QF_ERR_INVALID_ARG, "workspace is NULL");
@@ -704,6 +774,6 @@ const char* qf_status_string(qf_status s) {
 
 const char* qf_last_error(void) { return g_err; }
 
-int qf_version(void) { return (1 << 16) | 4; }
+int qf_version(void) { return (1 << 16) | 5; }
 
 }  // extern "C"

@@ -222,6 +222,27 @@ qf_status qf_amax_fakequant(const qf_tensor* t, int n, float* d_group_amax, int 
 /* Bytes of workspace qf_amax_fakequant needs for n_groups tie groups (0 if n_groups <= 0). */
 size_t qf_amax_fakequant_workspace_bytes(int n_groups);
 
+/*
+ * qf_amax_fakequant_noalloc -- qf_amax_fakequant with a workspace the library owns:
+ * a static device array of 16 KB per device, compiled into libqf.so.  No memory is
+ * allocated, neither by this call nor by the caller.  The project page has no
+ * counterpart: this is an interface convenience, not part of the method.
+ *
+ * The results are bit for bit those of qf_amax_fakequant with a caller workspace.
+ * The call first clears the part of the static workspace it uses (one
+ * cudaMemsetAsync on `stream`), then runs qf_amax_fakequant on it.
+ * Limit: n_groups <= 4092; larger counts return QF_ERR_INVALID_ARG (use
+ * qf_amax_fakequant with a workspace of your own).
+ * The static workspace is shared by every call on the device.  Two calls that may
+ * run at the same time (different streams, or different host threads with no
+ * ordering between them) race on it: serialize them, or give each its own
+ * workspace through qf_amax_fakequant.
+ * Errors: as qf_amax_fakequant.
+ */
+qf_status qf_amax_fakequant_noalloc(const qf_tensor* t, int n, float* d_group_amax,
+                                    int n_groups, float* d_tracked, float* d_group_scale_out,
+                                    void* stream);
+
 /* Synchronizes `stream`, then reads the error flags of a qf_amax_fakequant
  * workspace: QF_OK, or QF_ERR_TIMEOUT if a grid barrier gave up. */
 qf_status qf_workspace_check(const void* d_workspace, void* stream);
@@ -321,7 +342,8 @@ const char* qf_last_error(void);
 
 /* ABI version: (major << 16) | minor.  1.1 added qf_tensor.x_type (formerly a
  * reserved field that had to be 0, which still means BF16); 1.2 the LoRA calls;
- * 1.3 QF_Q4K_MSE; 1.4 qf_amax_fakequant, its workspace calls and QF_ERR_TIMEOUT. */
+ * 1.3 QF_Q4K_MSE; 1.4 qf_amax_fakequant, its workspace calls and QF_ERR_TIMEOUT;
+ * 1.5 qf_amax_fakequant_noalloc. */
 int qf_version(void);
 
 #ifdef __cplusplus

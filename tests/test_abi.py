@@ -58,7 +58,7 @@ def test_struct_layout_matches_header(qf):
 def test_status_strings(qf):
     for s in range(7):
         assert qf.lib.qf_status_string(s).decode().startswith("QF_")
-    assert qf.lib.qf_version() == (1 << 16) | 4
+    assert qf.lib.qf_version() == (1 << 16) | 5
 
 
 def _tensor(qf, x=0x1000, rows=4, cols=64, group=0, y=0x2000, codes=0x3000, scales=0x4000,
