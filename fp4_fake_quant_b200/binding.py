@@ -59,6 +59,7 @@ def _load() -> ctypes.CDLL:
     lib.qf_lora_merge.argtypes = [T, L, I, P]
     lib.qf_amax_tied_lora.argtypes = [T, L, I, P, I, P]
     lib.qf_fakequant_lora.argtypes = [I, T, L, I, P, I, P, P]
+    lib.qf_amax_fakequant_lora.argtypes = [T, L, I, P, I, P, P]
     lib.qf_amax_fakequant.argtypes = [T, I, P, I, P, P, P, ctypes.c_size_t, P]
     lib.qf_amax_fakequant_workspace_bytes.argtypes = [I]
     lib.qf_amax_fakequant_workspace_bytes.restype = ctypes.c_size_t
@@ -66,7 +67,8 @@ def _load() -> ctypes.CDLL:
     lib.qf_amax_fakequant_noalloc.argtypes = [T, I, P, I, P, P, P]
     for f in (lib.qf_amax_tied, lib.qf_fakequant, lib.qf_pack, lib.qf_ste_backward,
               lib.qf_lora_merge, lib.qf_amax_tied_lora, lib.qf_fakequant_lora,
-              lib.qf_amax_fakequant, lib.qf_workspace_check, lib.qf_amax_fakequant_noalloc):
+              lib.qf_amax_fakequant, lib.qf_workspace_check, lib.qf_amax_fakequant_noalloc,
+              lib.qf_amax_fakequant_lora):
         f.restype = I
     lib.qf_status_string.argtypes = [I]
     lib.qf_status_string.restype = ctypes.c_char_p
@@ -81,10 +83,9 @@ lib = _load()
 
 # the entry points declared in include/qf.h
 EXPORTS = ("qf_amax_tied", "qf_fakequant", "qf_pack", "qf_ste_backward", "qf_lora_merge",
-           "qf_amax_tied_lora", "qf_fakequant_lora", "qf_amax_fakequant",
-           "qf_amax_fakequant_workspace_bytes", "qf_workspace_check",
-           "qf_amax_fakequant_noalloc", "qf_status_string",
-           "qf_last_error", "qf_version")
+           "qf_amax_tied_lora", "qf_fakequant_lora", "qf_amax_fakequant_lora",
+           "qf_amax_fakequant", "qf_amax_fakequant_workspace_bytes", "qf_workspace_check",
+           "qf_amax_fakequant_noalloc", "qf_status_string", "qf_last_error", "qf_version")
 
 
 def _check(status: int) -> None:
@@ -303,6 +304,23 @@ def qf_fakequant_lora(fmt, xs, adapters, ys=None, codes=None, scales=None, group
     ng = group_amax.numel() if group_amax is not None else 0
     _check(lib.qf_fakequant_lora(_fmt(fmt), arr, _lora(adapters), n, _ptr(group_amax), ng,
                                  _ptr(group_scale_out), _stream(stream)))
+
+
+def qf_amax_fakequant_lora(xs, adapters, ys=None, codes=None, scales=None, groups=None,
+                           group_amax=None, group_scale_out=None, stream=None) -> None:
+    """LoRA-QAD NVFP4 step: merged-weight group amax, then fake-quant + pack (one call)."""
+    arr, n = _desc(xs, ys, codes, scales, groups)
+    _check(lib.qf_amax_fakequant_lora(arr, _lora(adapters), n, _ptr(group_amax),
+                                      group_amax.numel(), _ptr(group_scale_out), _stream(stream)))
+
+
+def prepare_amax_fakequant_lora(xs, adapters, ys=None, codes=None, scales=None, groups=None,
+                                group_amax=None, group_scale_out=None) -> "Prepared":
+    arr, n = _desc(xs, ys, codes, scales, groups)
+    la = _lora(adapters)
+    keep = (arr, la, list(xs), list(adapters), ys, codes, scales, group_amax, group_scale_out)
+    return Prepared(lib.qf_amax_fakequant_lora,
+                    (arr, la, n, _ptr(group_amax), group_amax.numel(), _ptr(group_scale_out)), keep)
 
 
 def prepare_fakequant_lora(fmt, xs, adapters, ys=None, codes=None, scales=None, groups=None,

@@ -554,6 +554,58 @@ qf_status qf_fakequant_lora(qf_format f, const qf_tensor* t, const qf_lora* l, i
 }
 
 
+qf_status qf_amax_fakequant_lora(const qf_tensor* t, const qf_lora* l, int n,
+                                 float* d_group_amax, int n_groups, float* d_group_scale_out,
+                                 void* stream) {
+    g_err[0] = 0;
+    if (n_groups <= 0) return fail(QF_ERR_INVALID_ARG, "n_groups = %d <= 0", n_groups);
+    if (d_group_amax == nullptr) return fail(QF_ERR_INVALID_ARG, "d_group_amax is NULL");
+    std::vector<qf::LoraTensor> v;
+    int max_rank;
+    qf_status st = lora_tensors(t, l, n, 16, n_groups, true, true, &v, &max_rank);
+    if (st != QF_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(d_group_amax, 0, sizeof(float) * (size_t)n_groups, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+    bool all_y = true;
+    for (const qf::LoraTensor& d : v) all_y &= d.y != nullptr;
+    if (v.empty() || !all_y) {
+        // no room for the merged weight: form it twice (amax pass, then fused pass)
+        if (!v.empty()) {
+            st = lora_launch<qf::kLoraAmax>(v, max_rank, d_group_amax, nullptr, n_groups, s);
+            if (st != QF_OK) return st;
+        }
+        if (v.empty() && !d_group_scale_out) return QF_OK;
+        if (v.empty()) {
+            qf::LoraTensor none{};
+            none.rows = 0;
+            none.cols = 16;
+            none.col_groups = 1;
+            none.rank = 1;
+            v.push_back(none);
+        }
+        return lora_launch<qf::kLoraNV>(v, max_rank, d_group_amax, d_group_scale_out, n_groups, s);
+    }
+    // the merged weight is formed once, written into y with its group amax, and y is
+    // then quantized in place by the plain NVFP4 pass (every lane reads its block
+    // before it writes it, and blocks are disjoint)
+    st = lora_launch<qf::kLoraMergeAmax>(v, max_rank, d_group_amax, nullptr, n_groups, s);
+    if (st != QF_OK) return st;
+    std::vector<DevTensor> w;
+    w.reserve(v.size());
+    for (const qf::LoraTensor& d : v) {
+        DevTensor x{};
+        x.x = d.y;
+        x.y = d.y;
+        x.codes = d.codes;
+        x.scales = d.scales;
+        x.numel = d.rows * d.cols;
+        x.group = d.group;
+        w.push_back(x);
+    }
+    return launch_format(QF_NVFP4, 0, QF_X_BF16, w, d_group_amax, d_group_scale_out, n_groups, s);
+}
+
 qf_status qf_amax_tied(const qf_tensor* t, int n, float* d_group_amax, int n_groups,
                        float* d_tracked, void* stream) {
     g_err[0] = 0;
@@ -774,6 +826,6 @@ const char* qf_status_string(qf_status s) {
 
 const char* qf_last_error(void) { return g_err; }
 
-int qf_version(void) { return (1 << 16) | 5; }
+int qf_version(void) { return (1 << 16) | 6; }
 
 }  // extern "C"

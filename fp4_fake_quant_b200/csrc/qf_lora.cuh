@@ -31,7 +31,9 @@ constexpr int kLoraRows = 32;      // rows per CTA unit
 constexpr int kLoraCols = 1024;    // columns per CTA unit (8 warps x 128)
 constexpr int kLoraThreads = 256;
 
-enum LoraMode { kLoraNV = 0, kLoraMX = 1, kLoraMerge = 2, kLoraAmax = 3 };
+// kLoraMergeAmax writes the merged weight like kLoraMerge and folds its max |M| into
+// the tie-group amax like kLoraAmax, in one pass.
+enum LoraMode { kLoraNV = 0, kLoraMX = 1, kLoraMerge = 2, kLoraAmax = 3, kLoraMergeAmax = 4 };
 
 struct LoraTensor {
     const uint16_t* w;      // BF16 base [rows, cols]
@@ -77,7 +79,9 @@ __global__ void __launch_bounds__(kLoraThreads) k_lora(const __grid_constant__ L
     __shared__ __align__(16) float2 bsm[kLoraRows][R];      // (b, b) pairs
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int64_t cu = blockIdx.x;
-    if (MODE != kLoraAmax && cu == 0 && P.group_scale_out) {
+    constexpr bool kWritesMerged = MODE == kLoraMerge || MODE == kLoraMergeAmax;
+    constexpr bool kFoldsAmax = MODE == kLoraAmax || MODE == kLoraMergeAmax;
+    if (MODE == kLoraNV && cu == 0 && P.group_scale_out) {
         for (int g = threadIdx.x; g < P.n_groups; g += kLoraThreads)
             P.group_scale_out[g] = nv_tensor_scale(P.group_amax[g]);
     }
@@ -152,13 +156,14 @@ __global__ void __launch_bounds__(kLoraThreads) k_lora(const __grid_constant__ L
             x[h][0] = bf16_lo(xw[h][0]); x[h][1] = bf16_hi(xw[h][0]);
             x[h][2] = bf16_lo(xw[h][1]); x[h][3] = bf16_hi(xw[h][1]);
         }
-        if (MODE == kLoraMerge) {
+        if (kWritesMerged) {
 #pragma unroll
             for (int h = 0; h < 4; ++h)
                 if (colok && i0 + h < nrows && T.y)
                     *reinterpret_cast<uint2*>(T.y + (r0 + i0 + h) * T.cols + col0) =
                         make_uint2(xw[h][0], xw[h][1]);
-        } else {
+        }
+        if (MODE != kLoraMerge) {
             uint32_t m[4];
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
@@ -166,7 +171,7 @@ __global__ void __launch_bounds__(kLoraThreads) k_lora(const __grid_constant__ L
 #pragma unroll
                 for (int c = 0; c < 4; ++c) m[h] = max(m[h], __float_as_uint(x[h][c]) & 0x7FFFFFFFu);
             }
-            if (MODE == kLoraAmax) {
+            if (kFoldsAmax) {
 #pragma unroll
                 for (int h = 0; h < 4; ++h)
                     if (i0 + h < nrows) run = max(run, m[h]);
@@ -235,7 +240,7 @@ __global__ void __launch_bounds__(kLoraThreads) k_lora(const __grid_constant__ L
 #pragma unroll
         for (int h = 0; h < 4; ++h) wcur[h] = wnxt[h];
     }
-    if (MODE == kLoraAmax) {
+    if (kFoldsAmax) {
         // one atomic per CTA (its unit lies in one tensor), not one per warp
         __shared__ uint32_t wmax[kLoraThreads / 32];
 #pragma unroll

@@ -321,6 +321,24 @@ qf_status qf_fakequant_lora(qf_format f, const qf_tensor* t, const qf_lora* l, i
                             void* stream);
 
 /*
+ * qf_amax_fakequant_lora -- the LoRA-QAD NVFP4 step in one call: the tie-group amax
+ * of the merged weights (as qf_amax_tied_lora), then their fake-quant + pack (as
+ * qf_fakequant_lora with QF_NVFP4 on that amax).  The outputs are bit for bit those
+ * of the two calls.
+ *   When every non-empty tensor has a y, the merged weight is formed ONCE: one
+ *   pass writes BF16(W + scale * B A) into y and folds its max |M| into the group
+ *   amax, and the plain NVFP4 fused pass then quantizes y in place.  Otherwise the
+ *   merge is formed in both passes, as the two calls do.
+ *   t, l, n, n_groups   as for qf_fakequant_lora with QF_NVFP4.
+ *   d_group_amax        FP32[n_groups], overwritten with the merged weights' group amax.
+ *   d_group_scale_out   NULL, or FP32[n_groups] receiving each s_t.
+ * Errors: as qf_amax_tied_lora and qf_fakequant_lora.
+ */
+qf_status qf_amax_fakequant_lora(const qf_tensor* t, const qf_lora* l, int n,
+                                 float* d_group_amax, int n_groups, float* d_group_scale_out,
+                                 void* stream);
+
+/*
  * QF_Q4K_MSE -- the Q4_K format (identical 144-byte blocks and dequantization) with
  * an MSE-searched fit, the kind of post-training quantizer the project page uses as
  * its Q4_K PTQ baseline ("Key findings"; the pages do not give its steps).  Per
@@ -343,7 +361,7 @@ const char* qf_last_error(void);
 /* ABI version: (major << 16) | minor.  1.1 added qf_tensor.x_type (formerly a
  * reserved field that had to be 0, which still means BF16); 1.2 the LoRA calls;
  * 1.3 QF_Q4K_MSE; 1.4 qf_amax_fakequant, its workspace calls and QF_ERR_TIMEOUT;
- * 1.5 qf_amax_fakequant_noalloc. */
+ * 1.5 qf_amax_fakequant_noalloc; 1.6 qf_amax_fakequant_lora. */
 int qf_version(void);
 
 #ifdef __cplusplus

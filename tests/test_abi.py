@@ -58,7 +58,7 @@ def test_struct_layout_matches_header(qf):
 def test_status_strings(qf):
     for s in range(7):
         assert qf.lib.qf_status_string(s).decode().startswith("QF_")
-    assert qf.lib.qf_version() == (1 << 16) | 5
+    assert qf.lib.qf_version() == (1 << 16) | 6
 
 
 def _tensor(qf, x=0x1000, rows=4, cols=64, group=0, y=0x2000, codes=0x3000, scales=0x4000,
@@ -200,3 +200,10 @@ def test_lora_validation(qf):
     assert lib.qf_amax_tied_lora(t, lora(), 1, None, 1, None) == INV
     assert lib.qf_amax_tied_lora(_tensor(qf, group=3), lora(), 1, 0x7000, 2, None) == INV
     assert lib.qf_lora_merge(_tensor(qf, rows=0), lora(), 1, None) == 0                 # empty
+    one = lib.qf_amax_fakequant_lora
+    assert one(t, lora(), 1, None, 1, None, None) == INV                                  # no amax
+    assert one(t, lora(), 1, 0x7000, 0, None, None) == INV
+    assert one(_tensor(qf, cols=24), lora(), 1, 0x7000, 1, None, None) == SHAPE          # NVFP4: 16 | cols
+    assert one(_tensor(qf, group=1), lora(), 1, 0x7000, 1, None, None) == INV
+    assert one(_tensor(qf, y=0, codes=0, scales=0), lora(), 1, 0x7000, 1, None, None) == INV
+    assert one(t, lora(rank=40), 1, 0x7000, 1, None, None) == INV

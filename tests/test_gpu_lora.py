@@ -105,3 +105,59 @@ def test_lora_grouped_experts_with_tied_groups():
         assert_same(f"grouped lora y {i}", bits(outs[i][0]), y)
         assert_same(f"grouped lora codes {i}", u8(outs[i][1]), c)
         assert_same(f"grouped lora scales {i}", u8(outs[i][2]), s)
+
+
+@pytest.mark.parametrize("rows,cols,rank", SHAPES)
+@pytest.mark.parametrize("with_y", [True, False])
+def test_amax_fakequant_lora_one_call(rows, cols, rank, with_y):
+    """qf_amax_fakequant_lora: with y, the merged weight is formed once and quantized in
+    place; without y, it is formed in both passes.  Either way the bytes are the
+    oracle's (merge, then tie-group amax, then NVFP4)."""
+    if cols % 16:
+        pytest.skip("NVFP4 needs 16 | cols")
+    w, b, a = _case(rows, cols, rank, 5 * rows + rank)
+    scale = 24.0 / rank
+    merged = oracle.lora_merge(w, b, a, scale)
+    am = np.float32(oracle.amax(merged))
+    y, c, s, st = oracle.nvfp4(merged, am)
+    wd = w.to(DEV)
+    yo, co, so = qf.alloc_outputs("nvfp4", wd)
+    amax = torch.full((1,), float("nan"), device=DEV)
+    st_out = torch.full((1,), float("nan"), device=DEV)
+    qf.qf_amax_fakequant_lora([wd], [(b.to(DEV), a.to(DEV), scale)], [yo] if with_y else None,
+                              [co], [so], [0], amax, st_out)
+    torch.cuda.synchronize()
+    assert_same("one-call amax", amax.cpu().numpy().view(np.uint32), np.float32([am]).view(np.uint32))
+    assert_same("one-call s_t", st_out.cpu().numpy().view(np.uint32), np.float32([st]).view(np.uint32))
+    if with_y:
+        assert_same("one-call y", bits(yo), y)
+    assert_same("one-call codes", u8(co), c)
+    assert_same("one-call scales", u8(so), s)
+
+
+def test_amax_fakequant_lora_grouped():
+    """Experts with tied groups in one call, merged weights formed once."""
+    ts, ads, groups, merged = [], [], [], []
+    for e in range(3):
+        for j, (r, c) in enumerate([(96, 2048), (96, 2048), (256, 768)]):
+            w, b, a = _case(r, c, 8, 300 + 3 * e + j)
+            ts.append(w)
+            ads.append((b, a, 3.0))
+            groups.append(2 * e + (j == 2))
+            merged.append(oracle.lora_merge(w, b, a, 3.0))
+    am = np.zeros(6, np.float32)
+    for m, g in zip(merged, groups):
+        am[g] = max(am[g], np.float32(oracle.amax(m)))
+    xs = [t.to(DEV) for t in ts]
+    adapters = [(b.to(DEV), a.to(DEV), s) for b, a, s in ads]
+    amax = torch.empty(6, device=DEV)
+    outs = [qf.alloc_outputs("nvfp4", x) for x in xs]
+    qf.qf_amax_fakequant_lora(xs, adapters, [o[0] for o in outs], [o[1] for o in outs],
+                              [o[2] for o in outs], groups, amax)
+    torch.cuda.synchronize()
+    assert_same("grouped one-call amax", amax.cpu().numpy().view(np.uint32), am.view(np.uint32))
+    for i, m in enumerate(merged):
+        y, c, s, _ = oracle.nvfp4(m, am[groups[i]])
+        assert_same(f"grouped one-call y {i}", bits(outs[i][0]), y)
+        assert_same(f"grouped one-call codes {i}", u8(outs[i][1]), c)
+        assert_same(f"grouped one-call scales {i}", u8(outs[i][2]), s)
