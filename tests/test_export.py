@@ -1,0 +1,147 @@
+"""Export containers, decoded by the engines' own reference code (no GPU needed).
+
+The QATFactory project page (Method, "Export") ships NVFP4 and MXFP4 checkpoints
+in vLLM's compressed-tensors format and Q4_K as a llama.cpp GGUF file.  These
+tests pin the byte layout of the packed outputs against decoders that owe nothing
+to this repository:
+  * GGUF: llama.cpp's ``gguf`` package reads the file back and its reference Q4_K
+    dequantizer reproduces the oracle's BF16 fake-quant output bit for bit.
+  * compressed-tensors: its FP4 unpacker and torch's float8_e4m3fn decoding give
+    the E2M1 values and E4M3 scales the oracle used, and its E8M0 scale decoding
+    gives the MXFP4 values exactly.
+The packed bytes come from the oracle, whose bytes the GPU parity tests prove equal to
+the CUDA path's."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from fp4_fake_quant_b200 import export
+
+gguf = pytest.importorskip("gguf")
+pytest.importorskip("safetensors")
+
+
+def _bf16_bits(a32: np.ndarray) -> np.ndarray:
+    return workloads.bf16_bits(torch.from_numpy(np.ascontiguousarray(a32, np.float32))
+                               .to(torch.bfloat16)).reshape(-1)
+
+
+def test_gguf_q4k_decoded_by_llama_cpp_reference(tmp_path):
+    wl = workloads.q4k_weights(rows_scale=1 / 128)
+    names = ["blk.0.ffn_down.weight", "blk.0.ffn_up.weight"]
+    packed = []
+    for name, x in zip(names, wl["tensors"]):
+        y, blocks = oracle.q4k(x)
+        packed.append((name, x, y, blocks))
+    path = str(tmp_path / "q4k.gguf")
+    export.save_gguf_q4k(path, [(n, torch.from_numpy(b), x.shape[0], x.shape[1])
+                                for n, x, _, b in packed],
+                         kv={"general.name": "qf-export-test", "qf.block_size": 256})
+    r = gguf.GGUFReader(path)
+    got = {t.name: t for t in r.tensors}
+    assert set(got) == set(names)
+    for name, x, y, blocks in packed:
+        t = got[name]
+        assert t.tensor_type == gguf.GGMLQuantizationType.Q4_K
+        assert sorted(int(v) for v in t.shape) == sorted(x.shape)      # ggml lists ne0 = cols first
+        assert np.array_equal(np.asarray(t.data).reshape(-1), blocks.reshape(-1))
+        deq = gguf.quants.dequantize(np.asarray(t.data), t.tensor_type).reshape(-1)
+        assert np.array_equal(_bf16_bits(deq), y.reshape(-1)), name
+    kv = {f.name: f for f in r.fields.values()}
+    assert "general.name" in kv and "qf.block_size" in kv
+
+
+def _tied_small():
+    wl = workloads.nvfp4_tied(rows_scale=1 / 64, with_grads=False)
+    return wl["tensors"][3], oracle.amax(wl["tensors"][3])        # a gate-like [224, 4096]
+
+
+def test_compressed_tensors_nvfp4_layout(tmp_path):
+    from compressed_tensors.compressors.nvfp4.helpers import unpack_fp4_from_uint8
+    from safetensors.torch import load_file
+
+    x, amax = _tied_small()
+    rows, cols = x.shape
+    y, codes, scales, s_t = oracle.nvfp4(x, amax)
+    t = export.compressed_tensors_nvfp4("model.layers.0.mlp.gate_proj", torch.from_numpy(codes),
+                                        torch.from_numpy(scales), rows, cols, amax,
+                                        input_amax=3.5)
+    path = str(tmp_path / "nvfp4.safetensors")
+    export.save_safetensors(path, t)
+    back = load_file(path)
+    assert set(back) == set(t)
+    for k in t:
+        assert back[k].dtype == t[k].dtype and torch.equal(back[k].view(torch.uint8),
+                                                           t[k].view(torch.uint8)), k
+    p = "model.layers.0.mlp.gate_proj"
+    assert back[f"{p}.weight_packed"].shape == (rows, cols // 2)
+    assert back[f"{p}.weight_scale"].dtype == torch.float8_e4m3fn
+    # E2M1 values from compressed-tensors' unpacker, E4M3 scales from torch's float8 type
+    v = unpack_fp4_from_uint8(back[f"{p}.weight_packed"], rows, cols, dtype=torch.float32).numpy()
+    sb = back[f"{p}.weight_scale"].to(torch.float32).numpy()
+    S = (np.repeat(sb, 16, axis=1) * np.float32(s_t)).astype(np.float32)
+    assert np.array_equal(_bf16_bits(v * S), y.reshape(-1))
+    # the global scale follows compressed-tensors' convention: 2688 / amax in FP32
+    g = float(back[f"{p}.weight_global_scale"][0])
+    assert g == float(np.float32(2688.0) / np.float32(amax))
+    assert float(back[f"{p}.input_global_scale"][0]) == float(np.float32(2688.0) / np.float32(3.5))
+
+
+def test_compressed_tensors_nvfp4_decompressor_agrees():
+    """compressed-tensors' own NVFP4 decompressor rebuilds the weight from the exported
+    tensors.  It computes code * scale / global_scale in BF16, which rounds twice
+    where the training path rounds once, so it agrees with the oracle's y to within
+    two BF16 units in the last place."""
+    from compressed_tensors.compressors.nvfp4.base import NVFP4PackedCompressor
+    from compressed_tensors.quantization import QuantizationScheme
+    from compressed_tensors.quantization.quant_scheme import PRESET_SCHEMES
+
+    x, amax = _tied_small()
+    rows, cols = x.shape
+    y, codes, scales, _ = oracle.nvfp4(x, amax)
+    t = export.compressed_tensors_nvfp4("w", torch.from_numpy(codes), torch.from_numpy(scales),
+                                        rows, cols, amax)
+    sd = {k.split(".", 1)[1]: v for k, v in t.items()}
+    scheme = QuantizationScheme(targets=["Linear"], **PRESET_SCHEMES["NVFP4"])
+    w = NVFP4PackedCompressor.decompress(sd, scheme)["weight"].to(torch.float32).numpy().reshape(-1)
+    ours = torch.from_numpy(y.view(np.int16)).view(torch.bfloat16).to(torch.float32).numpy()
+    ulp = np.maximum(np.abs(ours), np.float32(2.0 ** -126)) * np.float32(2.0 ** -7)
+    assert np.all(np.abs(w - ours) <= 2 * ulp)
+    assert np.array_equal(np.sign(w), np.sign(ours))
+
+
+def test_compressed_tensors_mxfp4_layout():
+    from compressed_tensors.compressors.mx_utils import decompress_mx_scale
+    from compressed_tensors.compressors.nvfp4.helpers import unpack_fp4_from_uint8
+
+    wl = workloads.mxfp4_w4a4(rows_scale=1 / 128)
+    x = wl["tensors"][1]                                         # activations: Student-t
+    rows, cols = x.shape
+    y, codes, scales = oracle.mxfp4(x)
+    t = export.compressed_tensors_mxfp4("model.layers.0.self_attn.q_proj",
+                                        torch.from_numpy(codes), torch.from_numpy(scales),
+                                        rows, cols)
+    p = "model.layers.0.self_attn.q_proj"
+    assert t[f"{p}.weight_scale"].dtype == torch.uint8 and t[f"{p}.weight_scale"].shape == (rows, cols // 32)
+    v = unpack_fp4_from_uint8(t[f"{p}.weight_packed"], rows, cols, dtype=torch.float32)
+    s = decompress_mx_scale(t[f"{p}.weight_scale"]).to(torch.float32)
+    w = (v * torch.repeat_interleave(s, 32, dim=1)).numpy()    # code * 2^e: exact
+    assert np.array_equal(_bf16_bits(w), y.reshape(-1))
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4"])
+def test_quantization_config(fmt):
+    cfg = export.quantization_config(fmt)
+    assert cfg["format"] == f"{fmt}-pack-quantized"
+    assert cfg["quant_method"] == "compressed-tensors"
+    w = cfg["config_groups"]["group_0"]["weights"]
+    assert w["num_bits"] == 4 and w["type"] == "float"
+    assert w["group_size"] == (16 if fmt == "nvfp4" else 32)
+
+
+def test_global_scale_edge_cases():
+    assert export.nvfp4_global_scale(0.0) == 1.0                  # every block scale is 0
+    assert export.nvfp4_global_scale(2688.0) == 1.0
+    assert export.nvfp4_global_scale(1e-44) == 1.0                # 2688 / a overflows FP32
