@@ -741,22 +741,25 @@ __global__ void __launch_bounds__(THREADS) k_q4k(const __grid_constant__ Table<M
             // elements: q = clamp(RNE((x + mm) * inv), 0, 15); y = BF16(s*q - mm)
             uint32_t qw[8];                              // q of elements 4t..4t+3, one per byte
             uint32_t yw[16];
+            // two elements per step on the paired FP32 pipe (no paired product feeds an
+            // add: the scaled value goes through the clamp first)
+            const float2 mm2 = make_float2(f.mm, f.mm), inv2 = make_float2(f.inv, f.inv);
+            const float2 rnd2 = make_float2(kRound, kRound), nrnd2 = make_float2(-kRound, -kRound);
+            const float2 s2 = make_float2(f.s, f.s), nmm2 = make_float2(-f.mm, -f.mm);
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
-                float r[2];
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const float t = __fmul_rn(__fadd_rn(x.get(2 * k + h), f.mm), f.inv);
-                    r[h] = __fadd_rn(fminf(fmaxf(t, 0.0f), 15.0f), kRound);
-                }
-                if (k & 1) qw[k >> 1] = __byte_perm(qw[k >> 1], __byte_perm(__float_as_uint(r[0]),
-                                                    __float_as_uint(r[1]), 0x0040), 0x5410);
-                else qw[k >> 1] = __byte_perm(__float_as_uint(r[0]), __float_as_uint(r[1]), 0x0040);
+                const float2 t = mul2_rn(add2_rn(make_float2(x.get(2 * k), x.get(2 * k + 1)), mm2),
+                                         inv2);
+                const float2 r = add2_rn(make_float2(fminf(fmaxf(t.x, 0.0f), 15.0f),
+                                                     fminf(fmaxf(t.y, 0.0f), 15.0f)), rnd2);
+                if (k & 1) qw[k >> 1] = __byte_perm(qw[k >> 1], __byte_perm(__float_as_uint(r.x),
+                                                    __float_as_uint(r.y), 0x0040), 0x5410);
+                else qw[k >> 1] = __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x0040);
                 // y = RN(s*q - mm): s = d*sc has at most 17 significant bits and q at most 4,
                 // so s*q is exact and one fused multiply-add rounds exactly once, as the
                 // separate multiply and subtract do
-                yw[k] = cvt_bf16x2(__fmaf_rn(f.s, __fsub_rn(r[1], kRound), -f.mm),
-                                   __fmaf_rn(f.s, __fsub_rn(r[0], kRound), -f.mm));
+                const float2 yv = fma2_rn(s2, add2_rn(r, nrnd2), nmm2);
+                yw[k] = cvt_bf16x2(yv.y, yv.x);
             }
             if (T.y) {
                 // stage y back through this lane's own 64 bytes, then store coalesced
