@@ -698,6 +698,82 @@ __device__ __forceinline__ Q4kFit q4k_fit(const Elems<XT, 32>& x) {
     return f;
 }
 
+// Elements, BF16 output and the 144-byte blocks of one warp unit (MODE 0): lane
+// (b, j) holds sub-block j of super-block b in x with its fit f; sm_lane / sm_mine
+// are the warp's staging rows (coalesced and transposed views).
+template <typename XT>
+__device__ __forceinline__ void q4k_emit_unit(const DevTensor& T, int64_t e0, int nsb, int lane,
+                                              const Elems<XT, 32>& x, const Q4kFit& f,
+                                              uint32_t sm_lane, uint32_t sm_mine) {
+    const int b = lane & 3, j = lane >> 2;
+    const bool have = b < nsb;
+    const int64_t sb = (e0 >> 8) + b;                    // this lane's super-block in the tensor
+    // elements: q = clamp(RNE((x + mm) * inv), 0, 15); y = BF16(s*q - mm)
+    uint32_t qw[8];                              // q of elements 4t..4t+3, one per byte
+    uint32_t yw[16];
+    // two elements per step on the paired FP32 pipe (no paired product feeds an
+    // add: the scaled value goes through the clamp first)
+    const float2 mm2 = make_float2(f.mm, f.mm), inv2 = make_float2(f.inv, f.inv);
+    const float2 rnd2 = make_float2(kRound, kRound), nrnd2 = make_float2(-kRound, -kRound);
+    const float2 s2 = make_float2(f.s, f.s), nmm2 = make_float2(-f.mm, -f.mm);
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        const float2 t = mul2_rn(add2_rn(make_float2(x.get(2 * k), x.get(2 * k + 1)), mm2),
+                                 inv2);
+        const float2 r = add2_rn(make_float2(fminf(fmaxf(t.x, 0.0f), 15.0f),
+                                             fminf(fmaxf(t.y, 0.0f), 15.0f)), rnd2);
+        if (k & 1) qw[k >> 1] = __byte_perm(qw[k >> 1], __byte_perm(__float_as_uint(r.x),
+                                            __float_as_uint(r.y), 0x0040), 0x5410);
+        else qw[k >> 1] = __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x0040);
+        // y = RN(s*q - mm): s = d*sc has at most 17 significant bits and q at most 4,
+        // so s*q is exact and one fused multiply-add rounds exactly once, as the
+        // separate multiply and subtract do
+        const float2 yv = fma2_rn(s2, add2_rn(r, nrnd2), nmm2);
+        yw[k] = cvt_bf16x2(yv.y, yv.x);
+    }
+    if (T.y) {
+        // stage y back through this lane's own 64 bytes, then store coalesced
+#pragma unroll
+        for (int p = 0; p < 4; ++p)
+            sts128(sm_mine + 16 * p, make_uint4(yw[4 * p], yw[4 * p + 1], yw[4 * p + 2],
+                                                yw[4 * p + 3]));
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            if (k < nsb) st_v4(T.y + e0 + 256 * k + 8 * lane, lds128(sm_lane + k * kQ4kRow));
+    }
+    if (T.codes) {
+        // codes: byte l of chunk c = q[2c][l] | q[2c+1][l] << 4; the even sub-block's
+        // lane writes bytes 0-15 of the chunk, the odd one bytes 16-31 (partner = lane ^ 4)
+        const bool odd = j & 1;
+        uint32_t out[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            const uint32_t recv = __shfl_xor_sync(kFull, odd ? qw[t] : qw[4 + t], 4);
+            out[t] = odd ? (recv | (qw[4 + t] << 4)) : (qw[t] | (recv << 4));
+        }
+        uint8_t* blk = T.codes + sb * 144;
+        if (have) st_v4(blk + 16 + 16 * j, make_uint4(out[0], out[1], out[2], out[3]));
+        // header: d, dmin, then the 12 bytes of 6-bit scales and mins
+        const uint32_t smv = f.sc | (f.m << 8);
+        const uint32_t o4 = __shfl_xor_sync(kFull, smv, 16);      // sub-block j ^ 4
+        const uint32_t scB = o4 & 0xFF, mB = o4 >> 8;
+        const uint32_t pk = ((f.sc & 63) | ((scB >> 4) << 6)) |
+                            (((f.m & 63) | ((mB >> 4) << 6)) << 8) |
+                            (((scB & 15) | ((mB & 15) << 4)) << 16);
+        const uint32_t p1 = __shfl_sync(kFull, pk, b + 4);
+        const uint32_t p2 = __shfl_sync(kFull, pk, b + 8);
+        const uint32_t p3 = __shfl_sync(kFull, pk, b + 12);
+        if (j == 0 && have) {
+            const uint32_t l1 = __byte_perm(pk, p1, 0x0040), h1 = __byte_perm(p2, p3, 0x0040);
+            const uint32_t l2 = __byte_perm(pk, p1, 0x0051), h2 = __byte_perm(p2, p3, 0x0051);
+            const uint32_t l3 = __byte_perm(pk, p1, 0x0062), h3 = __byte_perm(p2, p3, 0x0062);
+            st_v4(blk, make_uint4(f.dbits | (f.dminbits << 16), __byte_perm(l1, h1, 0x5410),
+                                  __byte_perm(l2, h2, 0x5410), __byte_perm(l3, h3, 0x5410)));
+        }
+    }
+}
+
 // MODE 0: dequant (y) and/or 144-byte blocks (codes).  MODE 1: clipped STE, y = grad_x.
 template <typename XT, int MAXT, int MODE, int THREADS, bool MSE>
 __global__ void __launch_bounds__(THREADS) k_q4k(const __grid_constant__ Table<MAXT> P) {
@@ -736,72 +812,8 @@ __global__ void __launch_bounds__(THREADS) k_q4k(const __grid_constant__ Table<M
             __syncwarp();                                  // the previous unit's staging reads
         }
         const Q4kFit f = q4k_fit<XT, MSE>(x);
-        const int64_t sb = (e0 >> 8) + b;                // this lane's super-block in the tensor
         if (MODE == 0) {
-            // elements: q = clamp(RNE((x + mm) * inv), 0, 15); y = BF16(s*q - mm)
-            uint32_t qw[8];                              // q of elements 4t..4t+3, one per byte
-            uint32_t yw[16];
-            // two elements per step on the paired FP32 pipe (no paired product feeds an
-            // add: the scaled value goes through the clamp first)
-            const float2 mm2 = make_float2(f.mm, f.mm), inv2 = make_float2(f.inv, f.inv);
-            const float2 rnd2 = make_float2(kRound, kRound), nrnd2 = make_float2(-kRound, -kRound);
-            const float2 s2 = make_float2(f.s, f.s), nmm2 = make_float2(-f.mm, -f.mm);
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const float2 t = mul2_rn(add2_rn(make_float2(x.get(2 * k), x.get(2 * k + 1)), mm2),
-                                         inv2);
-                const float2 r = add2_rn(make_float2(fminf(fmaxf(t.x, 0.0f), 15.0f),
-                                                     fminf(fmaxf(t.y, 0.0f), 15.0f)), rnd2);
-                if (k & 1) qw[k >> 1] = __byte_perm(qw[k >> 1], __byte_perm(__float_as_uint(r.x),
-                                                    __float_as_uint(r.y), 0x0040), 0x5410);
-                else qw[k >> 1] = __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x0040);
-                // y = RN(s*q - mm): s = d*sc has at most 17 significant bits and q at most 4,
-                // so s*q is exact and one fused multiply-add rounds exactly once, as the
-                // separate multiply and subtract do
-                const float2 yv = fma2_rn(s2, add2_rn(r, nrnd2), nmm2);
-                yw[k] = cvt_bf16x2(yv.y, yv.x);
-            }
-            if (T.y) {
-                // stage y back through this lane's own 64 bytes, then store coalesced
-#pragma unroll
-                for (int p = 0; p < 4; ++p)
-                    sts128(sm_mine + 16 * p, make_uint4(yw[4 * p], yw[4 * p + 1], yw[4 * p + 2],
-                                                        yw[4 * p + 3]));
-                __syncwarp();
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    if (k < nsb) st_v4(T.y + e0 + 256 * k + 8 * lane, lds128(sm_lane + k * kQ4kRow));
-            }
-            if (T.codes) {
-                // codes: byte l of chunk c = q[2c][l] | q[2c+1][l] << 4; the even sub-block's
-                // lane writes bytes 0-15 of the chunk, the odd one bytes 16-31 (partner = lane ^ 4)
-                const bool odd = j & 1;
-                uint32_t out[4];
-#pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    const uint32_t recv = __shfl_xor_sync(kFull, odd ? qw[t] : qw[4 + t], 4);
-                    out[t] = odd ? (recv | (qw[4 + t] << 4)) : (qw[t] | (recv << 4));
-                }
-                uint8_t* blk = T.codes + sb * 144;
-                if (have) st_v4(blk + 16 + 16 * j, make_uint4(out[0], out[1], out[2], out[3]));
-                // header: d, dmin, then the 12 bytes of 6-bit scales and mins
-                const uint32_t smv = f.sc | (f.m << 8);
-                const uint32_t o4 = __shfl_xor_sync(kFull, smv, 16);      // sub-block j ^ 4
-                const uint32_t scB = o4 & 0xFF, mB = o4 >> 8;
-                const uint32_t pk = ((f.sc & 63) | ((scB >> 4) << 6)) |
-                                    (((f.m & 63) | ((mB >> 4) << 6)) << 8) |
-                                    (((scB & 15) | ((mB & 15) << 4)) << 16);
-                const uint32_t p1 = __shfl_sync(kFull, pk, b + 4);
-                const uint32_t p2 = __shfl_sync(kFull, pk, b + 8);
-                const uint32_t p3 = __shfl_sync(kFull, pk, b + 12);
-                if (j == 0 && have) {
-                    const uint32_t l1 = __byte_perm(pk, p1, 0x0040), h1 = __byte_perm(p2, p3, 0x0040);
-                    const uint32_t l2 = __byte_perm(pk, p1, 0x0051), h2 = __byte_perm(p2, p3, 0x0051);
-                    const uint32_t l3 = __byte_perm(pk, p1, 0x0062), h3 = __byte_perm(p2, p3, 0x0062);
-                    st_v4(blk, make_uint4(f.dbits | (f.dminbits << 16), __byte_perm(l1, h1, 0x5410),
-                                          __byte_perm(l2, h2, 0x5410), __byte_perm(l3, h3, 0x5410)));
-                }
-            }
+            q4k_emit_unit<XT>(T, e0, nsb, lane, x, f, sm_lane, sm_mine);
         } else {
             // clipped STE: keep grad where 0 <= (x + mm) * inv <= 15
             uint32_t keep = 0;
