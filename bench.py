@@ -382,6 +382,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.empty_cache()
     if rank == 0 and world == 1 and not args.no_per_format:
         result["per_format"] = per_format(qf, dev, args, l2)
+        result["export"] = export_timing(qf, dev)
     if rank == 0 and world == 1 and not args.no_cpu:
         result["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_rows_frac)
     return result
@@ -481,6 +482,55 @@ def per_format(qf, dev, args, l2):
         out[name] = d
         del W
         torch.cuda.empty_cache()
+    return out
+
+
+def export_timing(qf, dev):
+    """The engine containers of two workloads, written from the device bytes: pack on the
+    GPU, copy to the host, write the file (host-side; the disk is the box's)."""
+    import tempfile
+
+    import gguf  # noqa: F401  (imported outside the timed region: the first import takes ~1 s)
+    import safetensors.torch  # noqa: F401
+    from fp4_fake_quant_b200 import export
+    out = {}
+    with tempfile.TemporaryDirectory() as d:
+        wl = workloads.q4k_weights()
+        xs = [x.to(dev) for x in wl["tensors"]]
+        cs = [qf.alloc_outputs("q4k", x, want_y=False)[1] for x in xs]
+        qf.qf_pack("q4k", xs, cs)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        export.save_gguf_q4k(os.path.join(d, "q4k.gguf"),
+                             [(f"blk.0.{n}.weight", c, x.shape[0], x.shape[1])
+                              for n, c, x in zip(("ffn_down", "ffn_up"), cs, xs)])
+        dt = time.perf_counter() - t0
+        nb = sum(c.numel() for c in cs)
+        out["gguf_q4k"] = {"bytes": nb, "s": dt, "MB/s": nb / dt / 1e6,
+                           "what": "Q4_K down + up blocks: D2H copy + GGUF write"}
+        del xs, cs
+        wl = workloads.nvfp4_tied(with_grads=False)
+        xs = [x.to(dev) for x in wl["tensors"]]
+        ng = wl["n_groups"]
+        amax = torch.empty(ng, device=dev)
+        outs = [qf.alloc_outputs("nvfp4", x, want_y=False) for x in xs]
+        qf.qf_amax_tied(xs, wl["groups"], amax)
+        qf.qf_pack("nvfp4", xs, [o[1] for o in outs], [o[2] for o in outs], wl["groups"], amax)
+        torch.cuda.synchronize()
+        am = amax.cpu().numpy()
+        t0 = time.perf_counter()
+        tensors = {}
+        for n, x, o, g in zip(wl["names"], xs, outs, wl["groups"]):
+            tensors.update(export.compressed_tensors_nvfp4(f"layers.0.{n}", o[1], o[2],
+                                                           x.shape[0], x.shape[1], float(am[g])))
+        export.save_safetensors(os.path.join(d, "nvfp4.safetensors"), tensors)
+        dt = time.perf_counter() - t0
+        nb = sum(v.numel() * v.element_size() for v in tensors.values())
+        out["safetensors_nvfp4"] = {"bytes": nb, "s": dt, "MB/s": nb / dt / 1e6,
+                                    "what": "NVFP4 tied projections, compressed-tensors tensors: "
+                                            "D2H copy + safetensors write"}
+        del xs, outs
+    torch.cuda.empty_cache()
     return out
 
 
