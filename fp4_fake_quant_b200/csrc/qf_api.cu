@@ -603,7 +603,13 @@ qf_status qf_amax_fakequant_lora(const qf_tensor* t, const qf_lora* l, int n,
         x.group = d.group;
         w.push_back(x);
     }
-    return launch_format(QF_NVFP4, 0, QF_X_BF16, w, d_group_amax, d_group_scale_out, n_groups, s);
+    // coherent loads: this pass writes the buffer it reads
+    return launch_chunks(qf::k_nv<uint16_t, nvb_u<uint16_t>(), kSmallT, QF_NVB_THREADS,
+                                  QF_NVB_PREFETCH, 3>,
+                         qf::k_nv<uint16_t, nvb_u<uint16_t>(), kLargeT, QF_NVB_THREADS,
+                                  QF_NVB_PREFETCH, 3>,
+                         QF_NVB_THREADS, QF_NVB_WAVES, w, 512 * nvb_u<uint16_t>(), d_group_amax,
+                         d_group_scale_out, nullptr, n_groups, s);
 }
 
 qf_status qf_amax_tied(const qf_tensor* t, int n, float* d_group_amax, int n_groups,

@@ -192,7 +192,9 @@ __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w 
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 // 16-byte streaming load on the read-only path.  LD = 0: no L1 allocation and a
-// 256-byte L2 prefetch; 1: plain non-coherent load; 2: no L1 allocation.
+// 256-byte L2 prefetch; 1: plain non-coherent load; 2: no L1 allocation; 3: ordinary
+// (coherent) load, for a kernel that writes the buffer it reads (an in-place pass:
+// the .nc forms require the data to stay unwritten for the kernel's lifetime).
 template <int LD = 0>
 __device__ __forceinline__ uint4 ld_stream(const void* p) {
     uint4 v;
@@ -202,9 +204,12 @@ __device__ __forceinline__ uint4 ld_stream(const void* p) {
     else if (LD == 1)
         asm("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
             : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
-    else
+    else if (LD == 2)
         asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
             : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    else
+        asm volatile("ld.global.v4.u32 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p) : "memory");
     return v;
 }
 __device__ __forceinline__ void st_v4(void* p, uint4 v) {
@@ -533,7 +538,7 @@ __device__ __forceinline__ void nv_encode_unit(const DevTensor& T, int64_t e0, i
     }
 }
 
-template <typename XT, int U, int MAXT, int THREADS, int PREFETCH>
+template <typename XT, int U, int MAXT, int THREADS, int PREFETCH, int LD = QF_FP4_LD>
 __global__ void __launch_bounds__(THREADS) k_nv(const __grid_constant__ Table<MAXT> P) {
     const int lane = threadIdx.x & 31;
     const int64_t warp = (int64_t(blockIdx.x) * THREADS + threadIdx.x) >> 5;
@@ -547,7 +552,7 @@ __global__ void __launch_bounds__(THREADS) k_nv(const __grid_constant__ Table<MA
     if (u >= P.total_units) return;
     int ti = locate_tensor(P, u);
     Elems<XT, 16> cur[U], nxt[U];
-    nv_load_unit<XT, U, QF_FP4_LD>(P.t[ti], (u - P.t[ti].unit_begin) * kUnit, lane, cur);
+    nv_load_unit<XT, U, LD>(P.t[ti], (u - P.t[ti].unit_begin) * kUnit, lane, cur);
     int cur_t = -1;
     float s_t = 0.0f, six_st = 0.0f;
     while (true) {
@@ -555,7 +560,7 @@ __global__ void __launch_bounds__(THREADS) k_nv(const __grid_constant__ Table<MA
         int tn = ti;
         if (PREFETCH && un < P.total_units) {
             tn = find_tensor(P, ti, un);
-            nv_load_unit<XT, U, QF_FP4_LD>(P.t[tn], (un - P.t[tn].unit_begin) * kUnit, lane, nxt);
+            nv_load_unit<XT, U, LD>(P.t[tn], (un - P.t[tn].unit_begin) * kUnit, lane, nxt);
         }
         const DevTensor& T = P.t[ti];
         if (ti != cur_t) {
@@ -572,7 +577,7 @@ __global__ void __launch_bounds__(THREADS) k_nv(const __grid_constant__ Table<MA
             for (int i = 0; i < U; ++i) cur[i] = nxt[i];
         } else {
             ti = find_tensor(P, ti, u);
-            nv_load_unit<XT, U, QF_FP4_LD>(P.t[ti], (u - P.t[ti].unit_begin) * kUnit, lane, cur);
+            nv_load_unit<XT, U, LD>(P.t[ti], (u - P.t[ti].unit_begin) * kUnit, lane, cur);
         }
     }
 }

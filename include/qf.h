@@ -39,6 +39,9 @@
  *     which is bounded (see there).
  *     qf_last_error() gives a one-line description of the last failure on the
  *     calling thread.
+ *   - Outputs must not overlap the inputs or one another, except that
+ *     qf_ste_backward mode 0 accepts grad_x == grad_y and then launches nothing.  The
+ *     kernels read their inputs through the read-only (non-coherent) path.
  *   - Calls on the same stream are ordered; calls whose outputs overlap and that
  *     run concurrently on different streams race.
  *   - Numerics are fixed bit for bit (see each call); every result is
