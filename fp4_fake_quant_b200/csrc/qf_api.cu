@@ -49,6 +49,31 @@ qf_status cuda_fail(cudaError_t e, const char* what) {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int block_of(qf_format f) { return f == QF_NVFP4 ? 16 : f == QF_MXFP4 ? 32 : 256; }
+
+// Whether the byte ranges [a, a + na) and [b, b + nb) intersect (NULL or empty: no).
+bool overlap(const void* a, int64_t na, const void* b, int64_t nb) {
+    if (!a || !b || na <= 0 || nb <= 0) return false;
+    const uintptr_t pa = reinterpret_cast<uintptr_t>(a), pb = reinterpret_cast<uintptr_t>(b);
+    return pa < pb + (uintptr_t)nb && pb < pa + (uintptr_t)na;
+}
+
+// One tensor's input and outputs must be disjoint (the kernels read x through the
+// non-coherent path and write the outputs in the same pass).  Checked per tensor;
+// overlaps between different tensors of a call are the caller's to avoid.
+qf_status check_disjoint(const qf_tensor& t, int i, qf_format f, bool use_y, bool use_scales) {
+    const int64_t n = t.rows * t.cols;
+    const bool q4 = f == QF_Q4K || f == QF_Q4K_MSE;
+    const int64_t nx = n * (t.x_type == QF_X_F32 ? 4 : 2);
+    const int64_t ny = use_y ? n * 2 : 0;
+    const int64_t nc = q4 ? n / 256 * 144 : n / 2;
+    const int64_t ns = use_scales && !q4 ? n / block_of(f) : 0;
+    const void* y = use_y ? t.y : nullptr;
+    const void* sc = use_scales && !q4 ? t.scales : nullptr;
+    if (overlap(t.x, nx, y, ny) || overlap(t.x, nx, t.codes, nc) || overlap(t.x, nx, sc, ns) ||
+        overlap(y, ny, t.codes, nc) || overlap(y, ny, sc, ns) || overlap(t.codes, nc, sc, ns))
+        return fail(QF_ERR_INVALID_ARG, "tensor %d: x, y, codes and scales must not overlap", i);
+    return QF_OK;
+}
 bool known_format(qf_format f) {
     return f == QF_NVFP4 || f == QF_MXFP4 || f == QF_Q4K || f == QF_Q4K_MSE;
 }
@@ -254,6 +279,8 @@ qf_status fakequant_impl(qf_format f, const qf_tensor* t, int n, const float* d_
             return fail(QF_ERR_INVALID_ARG, "tensor %d: no output (y, codes, scales all NULL)", i);
         if (!aligned16(y) || !aligned16(t[i].codes))
             return fail(QF_ERR_ALIGN, "tensor %d: y / codes not 16-byte aligned", i);
+        st = check_disjoint(t[i], i, f, !pack_only, true);
+        if (st != QF_OK) return st;
         DevTensor d{};
         if (t[i].x_type != t[0].x_type)
             return fail(QF_ERR_INVALID_ARG, "tensor %d: x_type differs from tensor 0's", i);
@@ -350,6 +377,8 @@ qf_status lora_tensors(const qf_tensor* t, const qf_lora* l, int n, int cols_mul
             return fail(QF_ERR_INVALID_ARG, "tensor %d: no output", i);
         if (!aligned16(t[i].y) || !aligned16(t[i].codes))
             return fail(QF_ERR_ALIGN, "tensor %d: y / codes not 16-byte aligned", i);
+        st = check_disjoint(t[i], i, cols_multiple == 32 ? QF_MXFP4 : QF_NVFP4, true, true);
+        if (st != QF_OK) return st;
         qf::LoraTensor d{};
         d.w = static_cast<const uint16_t*>(t[i].x);
         d.b = static_cast<const uint16_t*>(l[i].b);
@@ -670,6 +699,8 @@ qf_status qf_amax_fakequant(const qf_tensor* t, int n, float* d_group_amax, int 
             return fail(QF_ERR_INVALID_ARG, "tensor %d: no output (y, codes, scales all NULL)", i);
         if (!aligned16(t[i].y) || !aligned16(t[i].codes))
             return fail(QF_ERR_ALIGN, "tensor %d: y / codes not 16-byte aligned", i);
+        st = check_disjoint(t[i], i, QF_NVFP4, true, true);
+        if (st != QF_OK) return st;
         DevTensor d{};
         d.x = t[i].x;
         d.y = static_cast<uint16_t*>(t[i].y);
@@ -732,6 +763,8 @@ qf_status qf_amax_fakequant_noalloc(const qf_tensor* t, int n, float* d_group_am
             return fail(QF_ERR_INVALID_ARG, "tensor %d: no output (y, codes, scales all NULL)", i);
         if (!aligned16(t[i].y) || !aligned16(t[i].codes))
             return fail(QF_ERR_ALIGN, "tensor %d: y / codes not 16-byte aligned", i);
+        st = check_disjoint(t[i], i, QF_NVFP4, true, true);
+        if (st != QF_OK) return st;
     }
     void* ws = nullptr;
     qf_status st = noalloc_ws(&ws);

@@ -101,6 +101,12 @@ def test_validation_codes(qf, pack):
     assert _fq(qf, 0, _tensor(qf), amax=0x5000, ng=0, pack=pack) == INV
     assert _fq(qf, 0, _tensor(qf, group=1), amax=0x5000, ng=1, pack=pack) == INV
     assert _fq(qf, 0, _tensor(qf, group=-1), amax=0x5000, ng=1, pack=pack) == INV
+    # a tensor's input and outputs must be disjoint
+    if not pack:                                   # (qf_pack ignores y)
+        assert _fq(qf, 1, _tensor(qf, y=0x1100), pack=pack) == INV
+    assert _fq(qf, 1, _tensor(qf, codes=0x1100), pack=pack) == INV
+    assert _fq(qf, 1, _tensor(qf, scales=0x3010), pack=pack) == INV        # inside codes
+    assert _fq(qf, 2, _tensor(qf, cols=256, codes=0x10F0), pack=pack) == INV  # Q4_K blocks over x
     # empty tensors are skipped without needing outputs
     assert _fq(qf, 1, _tensor(qf, rows=0, y=0, codes=0, scales=0), pack=pack) == OK
     assert qf.lib.qf_last_error() == b""
@@ -161,6 +167,7 @@ def test_amax_fakequant_validation(qf):
     assert call(_tensor(qf, x=0x1008)) == ALIGN
     two = (qf.binding.QfTensor * 2)(_tensor(qf)[0], _tensor(qf, x_type=1)[0])
     assert call(two, n=2) == INV
+    assert call(_tensor(qf, y=0x1100)) == INV                      # y overlaps x
     assert lib.qf_workspace_check(None, None) == INV
 
 
