@@ -161,3 +161,21 @@ def test_amax_fakequant_lora_grouped():
         assert_same(f"grouped one-call y {i}", bits(outs[i][0]), y)
         assert_same(f"grouped one-call codes {i}", u8(outs[i][1]), c)
         assert_same(f"grouped one-call scales {i}", u8(outs[i][2]), s)
+
+
+@pytest.mark.parametrize("rank_pad", [4, 8, 16])
+def test_merge_accumulates_in_increasing_k(rank_pad):
+    """The oracle pin's worked case on the device: products 1, 2^-8, 2^-24, 2^-24 in
+    increasing k give BF16 1.0; in decreasing k, 1 + 2^-7.  Extra zero ranks (rank_pad)
+    add exact zeros.  Every column carries the same products."""
+    cols = 32
+    prods = [1.0, 2.0 ** -4, 2.0 ** -12, 2.0 ** -12] + [0.0] * (rank_pad - 4)
+    for order, want in ((1, 0x3F80), (-1, 0x3F81)):
+        p = prods[:4][::order] + prods[4:]
+        b = torch.tensor([p], dtype=torch.bfloat16, device=DEV)
+        a = torch.tensor(p, dtype=torch.bfloat16, device=DEV)[:, None].repeat(1, cols).contiguous()
+        w = torch.zeros(1, cols, dtype=torch.bfloat16, device=DEV)
+        m = torch.empty_like(w)
+        qf.qf_lora_merge([w], [(b, a, 1.0)], [m])
+        torch.cuda.synchronize()
+        assert np.all(bits(m) == want), (order, [hex(v) for v in bits(m)[:4]])

@@ -81,3 +81,22 @@ def test_merge_locality():
     m = oracle.lora_merge(w, b, a2, 0.25)
     diff_cols = np.nonzero((m != base).any(axis=0))[0]
     assert list(diff_cols) == [17]
+
+
+def test_accumulation_order_is_increasing_k():
+    """A hand-worked case that tells the summation orders apart.  The products
+    b_k * a_k are 1, 2^-8, 2^-24, 2^-24 (each exact).
+      increasing k:  1 + 2^-8 is exact; adding 2^-24 is a tie at half an FP32 ulp
+                     and rounds to the even 1 + 2^-8, twice; BF16(1 + 2^-8) is again
+                     a tie, to the even 1.0.
+      decreasing k or the exact sum:  2^-24 + 2^-24 + 2^-8 + 1 = 1 + 2^-8 + 2^-23,
+                     which BF16 rounds up to 1 + 2^-7.
+    The oracle must give 1.0 (W = 0, scale = 1)."""
+    b = bf16([[1.0, 2.0 ** -4, 2.0 ** -12, 2.0 ** -12]])
+    a = bf16([[1.0], [2.0 ** -4], [2.0 ** -12], [2.0 ** -12]])
+    w = bf16([[0.0]])
+    got = f32(oracle.lora_merge(w, b, a, 1.0).astype(np.uint32))
+    assert got.reshape(-1).tolist() == [1.0]
+    # the same products in decreasing k reach the other side of the BF16 tie
+    rev = f32(oracle.lora_merge(w, b[:, ::-1].copy(), a[::-1, :].copy(), 1.0).astype(np.uint32))
+    assert rev.reshape(-1).tolist() == [1.0 + 2.0 ** -7]
