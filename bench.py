@@ -262,8 +262,11 @@ def make_workload(name: str, qf, dev, seed_shift: int = 0):
         # prepared calls: the descriptor array is marshalled once, as a training loop would
         if name == "activation":
             W["pre"] = qf.prepare_amax_tied(xs, groups, cur, amax)     # amax <- max(amax, cur)
+            W["one_call"] = qf.prepare_amax_fakequant(xs, Y, C, S, groups, cur, tracked=amax,
+                                                      group_scale_out=so)
         else:
             W["pre"] = qf.prepare_amax_tied(xs, groups, amax)
+            W["one_call"] = qf.prepare_amax_fakequant(xs, Y, C, S, groups, amax, group_scale_out=so)
         W["fq"] = qf.prepare_fakequant(fmt, xs, Y, C, S, groups, amax, so)
         W["step_bytes"] = W["fq_bytes"] + in_b * numel
         W["launches"] = 2 * chunks
@@ -450,6 +453,12 @@ def per_format(qf, dev, args, l2):
                       "amax_GB/s": W["in_bytes"] * W["numel"] / t_pre / 1e6,
                       "step_us": t_step * 1e3,
                       "step_GB/s": W["step_bytes"] / t_step / 1e6})
+        if "one_call" in W:
+            t1 = timed_calls(W["one_call"], it, warm, flush)
+            d.update({"one_call_step_us": t1 * 1e3,
+                      "one_call_step_GB/s": W["step_bytes"] / t1 / 1e6,
+                      "one_call_is": "qf_amax_fakequant without a workspace: amax grid, then "
+                                     "the fused grid as its programmatic dependent"})
         if "two_call" in W:
             t2 = timed_calls(W["two_call"], it, warm, flush)
             d.update({"step_is": ("qf_amax_fakequant_lora: merge once into y, then NVFP4 in place"

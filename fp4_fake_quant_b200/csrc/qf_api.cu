@@ -133,11 +133,31 @@ void fill_table(Table<MAXT>& P, const std::vector<DevTensor>& v, size_t begin, s
     P.n = (int)count;
 }
 
-// Launch `kernel<MAXT>` over v in chunks of at most kLargeT tensors.
+// Launch as a programmatic dependent of the previous kernel in the stream: this grid
+// may start once every CTA of that one has run griddepcontrol.launch_dependents, and
+// waits for its results with griddepcontrol.wait.
+template <typename K, typename T>
+cudaError_t launch_dependent(K kernel, unsigned grid, int threads, const T& P, cudaStream_t s) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, P);
+}
+
+// Launch `kernel<MAXT>` over v in chunks of at most kLargeT tensors (as programmatic
+// dependents of the previous kernel when `dependent`).
 template <typename KS, typename KL>
 qf_status launch_chunks(KS small_kernel, KL large_kernel, int threads, int waves,
                         const std::vector<DevTensor>& v, int64_t unit_elems, const float* amax,
-                        float* scale_out, float* tracked, int n_groups, cudaStream_t s) {
+                        float* scale_out, float* tracked, int n_groups, cudaStream_t s,
+                        bool dependent = false) {
     Launch Ls, Ll;
     qf_status st = launch_shape(small_kernel, threads, waves, &Ls);
     if (st != QF_OK) return st;
@@ -159,12 +179,22 @@ qf_status launch_chunks(KS small_kernel, KL large_kernel, int threads, int waves
             Table<kSmallT> P;
             fill_table(P, v, b, cnt, unit_elems);
             P.group_amax = amax; P.group_scale_out = so; P.tracked = tracked; P.n_groups = n_groups;
-            small_kernel<<<grid_for(Ls, P.total_units), threads, 0, s>>>(P);
+            if (dependent) {
+                cudaError_t e = launch_dependent(small_kernel, grid_for(Ls, P.total_units), threads, P, s);
+                if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx");
+            } else {
+                small_kernel<<<grid_for(Ls, P.total_units), threads, 0, s>>>(P);
+            }
         } else {
             Table<kLargeT> Q;              // ~27 KB kernel parameter
             fill_table(Q, v, b, cnt, unit_elems);
             Q.group_amax = amax; Q.group_scale_out = so; Q.tracked = tracked; Q.n_groups = n_groups;
-            large_kernel<<<grid_for(Ll, Q.total_units), threads, 0, s>>>(Q);
+            if (dependent) {
+                cudaError_t e = launch_dependent(large_kernel, grid_for(Ll, Q.total_units), threads, Q, s);
+                if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx");
+            } else {
+                large_kernel<<<grid_for(Ll, Q.total_units), threads, 0, s>>>(Q);
+            }
         }
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
@@ -732,12 +762,27 @@ qf_status qf_amax_fakequant(const qf_tensor* t, int n, float* d_group_amax, int 
             : oneshot_launch<uint16_t, kLargeT>(v, d_group_amax, d_tracked, d_group_scale_out,
                                                 n_groups, ws, s);
     }
-    // two launches: the tie-group amax, then the fused pass on the scale it gives
+    // two launches: the tie-group amax, then the fused pass on the scale it gives, as a
+    // programmatic dependent of the amax grid (its first loads overlap that grid's end)
     st = amax_launch(v, x_type, d_group_amax, n_groups, d_tracked, s);
     if (st != QF_OK) return st;
     if (v.empty() && !d_group_scale_out) return QF_OK;
-    return launch_format(QF_NVFP4, 0, x_type, v, d_tracked ? d_tracked : d_group_amax,
-                         d_group_scale_out, n_groups, s);
+    const float* am = d_tracked ? d_tracked : d_group_amax;
+    if (v.empty())
+        return launch_format(QF_NVFP4, 0, x_type, v, am, d_group_scale_out, n_groups, s);
+    if (x_type == QF_X_F32)
+        return launch_chunks(qf::k_nv<float, nvb_u<float>(), kSmallT, QF_NVB_THREADS,
+                                      QF_NVB_PREFETCH, QF_FP4_LD, true>,
+                             qf::k_nv<float, nvb_u<float>(), kLargeT, QF_NVB_THREADS,
+                                      QF_NVB_PREFETCH, QF_FP4_LD, true>,
+                             QF_NVB_THREADS, QF_NVB_WAVES, v, 512 * nvb_u<float>(), am,
+                             d_group_scale_out, nullptr, n_groups, s, true);
+    return launch_chunks(qf::k_nv<uint16_t, nvb_u<uint16_t>(), kSmallT, QF_NVB_THREADS,
+                                  QF_NVB_PREFETCH, QF_FP4_LD, true>,
+                         qf::k_nv<uint16_t, nvb_u<uint16_t>(), kLargeT, QF_NVB_THREADS,
+                                  QF_NVB_PREFETCH, QF_FP4_LD, true>,
+                         QF_NVB_THREADS, QF_NVB_WAVES, v, 512 * nvb_u<uint16_t>(), am,
+                         d_group_scale_out, nullptr, n_groups, s, true);
 }
 
 qf_status qf_amax_fakequant_noalloc(const qf_tensor* t, int n, float* d_group_amax,

@@ -538,21 +538,31 @@ __device__ __forceinline__ void nv_encode_unit(const DevTensor& T, int64_t e0, i
     }
 }
 
-template <typename XT, int U, int MAXT, int THREADS, int PREFETCH, int LD = QF_FP4_LD>
+// DEP_AMAX: launched as a programmatic dependent of the amax kernel that produces
+// P.group_amax (and writes nothing this kernel reads otherwise).  The first unit of
+// x is loaded before griddepcontrol.wait -- x was final before the amax kernel
+// started -- and the group amax is read only after it, so the loads of this grid's
+// first wave overlap the end of the amax grid.
+template <typename XT, int U, int MAXT, int THREADS, int PREFETCH, int LD = QF_FP4_LD,
+          bool DEP_AMAX = false>
 __global__ void __launch_bounds__(THREADS) k_nv(const __grid_constant__ Table<MAXT> P) {
     const int lane = threadIdx.x & 31;
     const int64_t warp = (int64_t(blockIdx.x) * THREADS + threadIdx.x) >> 5;
     const int64_t nwarps = (int64_t(gridDim.x) * THREADS) >> 5;
     constexpr int kUnit = 512 * U;
+    int64_t u = warp;
+    int ti = 0;
+    Elems<XT, 16> cur[U], nxt[U];
+    if (u < P.total_units) {
+        ti = locate_tensor(P, u);
+        nv_load_unit<XT, U, LD>(P.t[ti], (u - P.t[ti].unit_begin) * kUnit, lane, cur);
+    }
+    if (DEP_AMAX) asm volatile("griddepcontrol.wait;" ::: "memory");
     if (blockIdx.x == 0 && P.group_scale_out) {
         for (int g = threadIdx.x; g < P.n_groups; g += THREADS)
             P.group_scale_out[g] = nv_tensor_scale(P.group_amax[g]);
     }
-    int64_t u = warp;
     if (u >= P.total_units) return;
-    int ti = locate_tensor(P, u);
-    Elems<XT, 16> cur[U], nxt[U];
-    nv_load_unit<XT, U, LD>(P.t[ti], (u - P.t[ti].unit_begin) * kUnit, lane, cur);
     int cur_t = -1;
     float s_t = 0.0f, six_st = 0.0f;
     while (true) {
@@ -862,6 +872,9 @@ __global__ void __launch_bounds__(THREADS) k_q4k(const __grid_constant__ Table<M
 // group's FP32 bits (non-negative floats order like their bit patterns).
 template <typename XT, int U, int MAXT, int THREADS>
 __global__ void __launch_bounds__(THREADS) k_amax(const __grid_constant__ Table<MAXT> P) {
+    // a programmatic dependent (the fused NVFP4 pass) may launch once every CTA of
+    // this grid has started; it waits for this grid's results before reading them
+    asm volatile("griddepcontrol.launch_dependents;");
     const int lane = threadIdx.x & 31;
     constexpr int kUnit = 256 * U;
     constexpr int kWarps = THREADS / 32;
