@@ -747,7 +747,7 @@ qf_status qf_amax_fakequant(const qf_tensor* t, int n, float* d_group_amax, int 
     qf_status st = dev_props(&D);
     if (st != QF_OK) return st;
     const bool one = d_workspace != nullptr && !v.empty() && v.size() <= (size_t)kLargeT &&
-                     D.coop && in_bytes * 3 <= (int64_t)D.l2;
+                     D.coop && in_bytes * QF_ONESHOT_L2_DIV <= (int64_t)D.l2;
     if (one) {
         uint32_t* ws = static_cast<uint32_t*>(d_workspace);
         if (v.size() <= (size_t)kSmallT)

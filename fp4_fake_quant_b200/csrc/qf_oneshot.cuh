@@ -34,8 +34,8 @@ constexpr uint32_t kOneshotErrTimeout = 1u;
 #ifndef QF_ONESHOT_MINB
 #define QF_ONESHOT_MINB 1       // minimum resident CTAs per SM asked of the register allocator
 #endif
-#ifndef QF_ONESHOT_PF
-#define QF_ONESHOT_PF 0         // 1: the encode pass loads the next unit while encoding this one
+#ifndef QF_ONESHOT_L2_DIV
+#define QF_ONESHOT_L2_DIV 3     // single-launch path when all input bytes <= L2 size / this
 #endif
 
 __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
@@ -148,8 +148,6 @@ __global__ void __launch_bounds__(THREADS, QF_ONESHOT_MINB)
         ti = locate_tensor(P, warp);
         int cur_t = -1;
         float s_t = 0.0f, six_st = 0.0f;
-        Elems<XT, 16> v[U], nx[U];
-        if (QF_ONESHOT_PF) nv_load_unit<XT, U, 1>(P.t[ti], (warp - P.t[ti].unit_begin) * kUnit, lane, v);
         for (int64_t u = warp; u < P.total_units; u += nwarps) {
             ti = find_tensor(P, ti, u);
             const DevTensor& T = P.t[ti];
@@ -159,19 +157,9 @@ __global__ void __launch_bounds__(THREADS, QF_ONESHOT_MINB)
                 cur_t = ti;
             }
             const int64_t e0 = (u - T.unit_begin) * kUnit;
-            if (QF_ONESHOT_PF) {
-                const int64_t un = u + nwarps;
-                if (un < P.total_units) {
-                    const int tn = find_tensor(P, ti, un);
-                    nv_load_unit<XT, U, 1>(P.t[tn], (un - P.t[tn].unit_begin) * kUnit, lane, nx);
-                }
-                nv_encode_unit<XT, U>(T, e0, lane, v, s_t, six_st);
-#pragma unroll
-                for (int i = 0; i < U; ++i) v[i] = nx[i];
-            } else {
-                nv_load_unit<XT, U, 1>(T, e0, lane, v);
-                nv_encode_unit<XT, U>(T, e0, lane, v, s_t, six_st);
-            }
+            Elems<XT, 16> v[U];
+            nv_load_unit<XT, U, 1>(T, e0, lane, v);
+            nv_encode_unit<XT, U>(T, e0, lane, v, s_t, six_st);
         }
     }
 
