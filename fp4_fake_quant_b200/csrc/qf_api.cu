@@ -768,7 +768,9 @@ qf_status qf_amax_fakequant(const qf_tensor* t, int n, float* d_group_amax, int 
     if (st != QF_OK) return st;
     if (v.empty() && !d_group_scale_out) return QF_OK;
     const float* am = d_tracked ? d_tracked : d_group_amax;
-    if (v.empty())
+    // grouped launches over many tensors measured slower as dependents (their early
+    // loads compete with the amax grid's long tail): plain stream order for those
+    if (v.empty() || v.size() > (size_t)kSmallT)
         return launch_format(QF_NVFP4, 0, x_type, v, am, d_group_scale_out, n_groups, s);
     if (x_type == QF_X_F32)
         return launch_chunks(qf::k_nv<float, nvb_u<float>(), kSmallT, QF_NVB_THREADS,
