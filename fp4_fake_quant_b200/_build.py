@@ -10,7 +10,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libqf.so")
 SOURCES = ["qf_api.cu"]
-HEADERS = ["qf_device.cuh", "qf_lora.cuh", "qf_oneshot.cuh"]
+HEADERS = sorted(f for f in os.listdir(CSRC) if f.endswith(".cuh"))   # every header counts
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
