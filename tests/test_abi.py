@@ -49,6 +49,40 @@ def test_header_compiles_as_c():
     assert r.returncode == 0, r.stderr
 
 
+def test_c_program_links_and_calls(qf, tmp_path):
+    """The boundary is usable from plain C: a C99 program links libqf.so and gets the
+    documented answers from calls that need no GPU."""
+    src = r"""
+#include <stdio.h>
+#include <string.h>
+#include "qf.h"
+int main(void) {
+    qf_tensor t;
+    memset(&t, 0, sizeof t);
+    t.x = (const void*)0x1000; t.rows = 4; t.cols = 48; t.y = (void*)0x2000;
+    t.codes = (void*)0x3000; t.scales = (void*)0x4000;
+    if (qf_version() != ((1 << 16) | 6)) return 1;
+    if (strncmp(qf_status_string(QF_ERR_SHAPE), "QF_ERR_SHAPE", 12) != 0) return 2;
+    if (qf_fakequant(QF_MXFP4, &t, 1, NULL, 0, NULL, NULL) != QF_ERR_SHAPE) return 3;
+    if (qf_last_error()[0] == 0) return 4;
+    if (qf_amax_fakequant_workspace_bytes(1) != 256) return 5;
+    if (qf_amax_tied(&t, 1, NULL, 1, NULL, NULL) != QF_ERR_INVALID_ARG) return 6;
+    printf("ok\n");
+    return 0;
+}
+"""
+    c = tmp_path / "abi.c"
+    c.write_text(src)
+    exe = tmp_path / "abi"
+    lib_dir = os.path.dirname(qf.binding.LIB_PATH)
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.dirname(HEADER),
+                        str(c), "-L", lib_dir, "-lqf", f"-Wl,-rpath,{lib_dir}", "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
+
+
 def test_struct_layout_matches_header(qf):
     T = qf.binding.QfTensor
     assert ctypes.sizeof(T) == 56
