@@ -74,6 +74,14 @@
 #ifndef QF_Q4K_WAVES
 #define QF_Q4K_WAVES 1
 #endif
+#ifndef QF_Q4K_MINB
+#define QF_Q4K_MINB 0           // > 0: minimum resident CTAs per SM asked of the register allocator
+#endif
+#if QF_Q4K_MINB > 0
+#define QF_Q4K_BOUNDS(t) __launch_bounds__(t, QF_Q4K_MINB)
+#else
+#define QF_Q4K_BOUNDS(t) __launch_bounds__(t)
+#endif
 #ifndef QF_AMAX_THREADS
 #define QF_AMAX_THREADS 256
 #endif
@@ -791,7 +799,7 @@ __device__ __forceinline__ void q4k_emit_unit(const DevTensor& T, int64_t e0, in
 
 // MODE 0: dequant (y) and/or 144-byte blocks (codes).  MODE 1: clipped STE, y = grad_x.
 template <typename XT, int MAXT, int MODE, int THREADS, bool MSE>
-__global__ void __launch_bounds__(THREADS) k_q4k(const __grid_constant__ Table<MAXT> P) {
+__global__ void QF_Q4K_BOUNDS(THREADS) k_q4k(const __grid_constant__ Table<MAXT> P) {
     __shared__ __align__(16) uint8_t stage[THREADS / 32][kQ4kWarpBytes];
     constexpr bool kBf16 = sizeof(XT) == 2;
     const int lane = threadIdx.x & 31;
