@@ -466,6 +466,27 @@ def per_format(qf, dev, args, l2):
                                   "qf_amax_fakequant, one cooperative launch"),
                       "two_launch_step_us": t2 * 1e3,
                       "two_launch_step_GB/s": W["step_bytes"] / t2 / 1e6})
+        if name == "nvfp4_tied":
+            # STE backward of the same tensors (reported beside the step, not in it: the
+            # identity is an alias in a training step): identity copy, 4 B per element, and
+            # the clipped mask, 6 B per element (reads x and grad_y, writes grad_x)
+            g = torch.Generator(device=dev).manual_seed(7)
+            gys = [(torch.randn(x.shape, generator=g, device=dev) * 1e-3).to(torch.bfloat16)
+                   for x in W["xs"]]
+            gxs = [torch.empty_like(t) for t in gys]
+            am = torch.empty(W["n_groups"], device=dev)
+            qf.qf_amax_tied(W["xs"], W["groups"], am)
+
+            def ste(mode):
+                for x, gy, gx, grp in zip(W["xs"], gys, gxs, W["groups"]):
+                    qf.qf_ste_backward(gy, gx, mode, "nvfp4", x, grp, am)
+            t_id = timed_calls(lambda: ste(0), it, warm, flush)
+            t_cl = timed_calls(lambda: ste(1), it, warm, flush)
+            d.update({"ste_identity_us": t_id * 1e3,
+                      "ste_identity_GB/s": 4 * W["numel"] / t_id / 1e6,
+                      "ste_clipped_us": t_cl * 1e3,
+                      "ste_clipped_GB/s": 6 * W["numel"] / t_cl / 1e6})
+            del gys, gxs
         if name.startswith("moe_"):
             xs, fmt = W["xs"], W["fmt"]
             n = len(xs)

@@ -224,10 +224,6 @@ qf_status check_tensor(const qf_tensor& t, int i, int need_cols_multiple, int n_
 }
 
 // The kernels of each format with their launch shapes (XT: input element type).
-template <typename XT, int MAXT, int MODE>
-constexpr auto nv_kernel() {
-    return qf::k_fp4<true, XT, kFp4U, MAXT, MODE, QF_NV_THREADS, QF_NV_PREFETCH>;
-}
 // FP32 input holds twice the bytes per element in registers: half the sub-tiles per unit
 template <typename XT>
 constexpr int nvb_u() { return sizeof(XT) == 2 ? QF_NVB_U : (QF_NVB_U + 1) / 2; }
@@ -252,8 +248,10 @@ qf_status launch_format_t(qf_format f, int mode, const std::vector<DevTensor>& v
             return launch_chunks(nv_block_kernel<XT, kSmallT>(), nv_block_kernel<XT, kLargeT>(),
                                  QF_NVB_THREADS, QF_NVB_WAVES, v, 512 * nvb_u<XT>(), am, so, nullptr,
                                  ng, s);
-        return launch_chunks(nv_kernel<XT, kSmallT, 1>(), nv_kernel<XT, kLargeT, 1>(), QF_NV_THREADS,
-                             QF_NV_WAVES, v, 256 * kFp4U, am, nullptr, nullptr, ng, s);
+        return launch_chunks(qf::k_nv_ste<XT, nvb_u<XT>(), kSmallT, QF_NVB_THREADS>,
+                             qf::k_nv_ste<XT, nvb_u<XT>(), kLargeT, QF_NVB_THREADS>,
+                             QF_NVB_THREADS, QF_NVB_WAVES, v, 512 * nvb_u<XT>(), am, nullptr,
+                             nullptr, ng, s);
     }
     if (f == QF_MXFP4) {
         if (mode == 0)

@@ -41,15 +41,6 @@
 #ifndef QF_MX_PREFETCH
 #define QF_MX_PREFETCH 0
 #endif
-#ifndef QF_NV_THREADS
-#define QF_NV_THREADS 256       // NVFP4 clipped STE (k_fp4)
-#endif
-#ifndef QF_NV_WAVES
-#define QF_NV_WAVES 4
-#endif
-#ifndef QF_NV_PREFETCH
-#define QF_NV_PREFETCH 1
-#endif
 #ifndef QF_NVB_THREADS
 #define QF_NVB_THREADS 128      // NVFP4 fused pass, one lane per block (k_nv)
 #endif
@@ -403,11 +394,14 @@ __device__ __forceinline__ void load_unit(const DevTensor& T, int64_t e0, int la
         const int64_t e = e0 + s * 256 + lane * 8;
         const bool ok = e < T.numel;
         L.v[s].template load<QF_FP4_LD>(x + e, ok);
-        if (MODE == 1) L.gv[s] = ok ? ld_stream<QF_FP4_LD>(T.g + e) : make_uint4(0, 0, 0, 0);
+        // coherent: grad_x may be grad_y (each element is read before its thread writes it)
+        if (MODE == 1) L.gv[s] = ok ? ld_stream<3>(T.g + e) : make_uint4(0, 0, 0, 0);
     }
 }
 
-// MXFP4 fused fake-quant + pack (MODE 0), or the NVFP4 / MXFP4 clipped STE (MODE 1).
+// MXFP4 fused fake-quant + pack (MODE 0), or the MXFP4 clipped STE (MODE 1); the
+// library launches it with NV = false (NVFP4 has the lane-per-block k_nv / k_nv_ste,
+// and the NV = true form is kept as the same kernel's 8-element-lane variant).
 // A unit is U sub-tiles of 256 elements.
 template <bool NV, typename XT, int U, int MAXT, int MODE, int THREADS, int PREFETCH>
 __global__ void __launch_bounds__(THREADS) k_fp4(const __grid_constant__ Table<MAXT> P) {
@@ -596,6 +590,67 @@ __global__ void __launch_bounds__(THREADS) k_nv(const __grid_constant__ Table<MA
         } else {
             ti = find_tensor(P, ti, u);
             nv_load_unit<XT, U, LD>(P.t[ti], (u - P.t[ti].unit_begin) * kUnit, lane, cur);
+        }
+    }
+}
+
+// NVFP4 clipped STE with one lane per 16-element block (the k_nv layout): the lane
+// derives its block's scale from x exactly as the forward pass does and keeps the
+// gradient of every element with |x * (1/S)| <= 6 (a zero x counts as 0).  grad_y is
+// read with ordinary loads: grad_x may be grad_y.
+template <typename XT, int U, int MAXT, int THREADS>
+__global__ void __launch_bounds__(THREADS) k_nv_ste(const __grid_constant__ Table<MAXT> P) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = (int64_t(blockIdx.x) * THREADS + threadIdx.x) >> 5;
+    const int64_t nwarps = (int64_t(gridDim.x) * THREADS) >> 5;
+    constexpr int kUnit = 512 * U;
+    if (warp >= P.total_units) return;
+    int ti = locate_tensor(P, warp);
+    int cur_t = -1;
+    float s_t = 0.0f, six_st = 0.0f;
+    for (int64_t u = warp; u < P.total_units; u += nwarps) {
+        ti = find_tensor(P, ti, u);
+        const DevTensor& T = P.t[ti];
+        if (ti != cur_t) {
+            s_t = nv_tensor_scale(P.group_amax[T.group]);
+            six_st = __fmul_rn(6.0f, s_t);
+            cur_t = ti;
+        }
+        const int64_t e0 = (u - T.unit_begin) * kUnit;
+        Elems<XT, 16> x[U];
+        nv_load_unit<XT, U, QF_FP4_LD>(T, e0, lane, x);
+        uint4 g[U][2];
+#pragma unroll
+        for (int s = 0; s < U; ++s) {
+            const int64_t e = e0 + s * 512 + lane * 16;
+            const bool ok = e < T.numel;
+            g[s][0] = ok ? ld_stream<3>(T.g + e) : make_uint4(0, 0, 0, 0);
+            g[s][1] = ok ? ld_stream<3>(T.g + e + 8) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int s = 0; s < U; ++s) {
+            const int64_t e = e0 + s * 512 + lane * 16;
+            uint32_t sb;
+            float S, inv;
+            nv_block_scale(__uint_as_float(x[s].amax_bits()), s_t, six_st, sb, S, inv);
+            const bool inf_inv = isinf(inv);
+            uint32_t keep = 0;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                float q = __fmul_rn(x[s].get(k), inv);
+                if (inf_inv && x[s].get(k) == 0.0f) q = x[s].get(k);
+                keep |= (uint32_t)(fabsf(q) <= 6.0f) << k;
+            }
+            uint32_t w[8] = {g[s][0].x, g[s][0].y, g[s][0].z, g[s][0].w,
+                             g[s][1].x, g[s][1].y, g[s][1].z, g[s][1].w};
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                w[k] = (((keep >> (2 * k)) & 1u) ? (w[k] & 0xFFFFu) : 0u) |
+                       (((keep >> (2 * k + 1)) & 1u) ? (w[k] & 0xFFFF0000u) : 0u);
+            if (e < T.numel) {
+                st_v4(T.y + e, make_uint4(w[0], w[1], w[2], w[3]));
+                st_v4(T.y + e + 8, make_uint4(w[4], w[5], w[6], w[7]));
+            }
         }
     }
 }
@@ -848,7 +903,7 @@ __global__ void QF_Q4K_BOUNDS(THREADS) k_q4k(const __grid_constant__ Table<MAXT>
             uint4 v[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k)
-                v[k] = k < nsb ? ld_stream<0>(T.g + e0 + 256 * k + 8 * lane) : make_uint4(0, 0, 0, 0);
+                v[k] = k < nsb ? ld_stream<3>(T.g + e0 + 256 * k + 8 * lane) : make_uint4(0, 0, 0, 0);
             __syncwarp();
 #pragma unroll
             for (int k = 0; k < 4; ++k) sts128(sm_lane + k * kQ4kRow, v[k]);

@@ -40,8 +40,9 @@
  *     qf_last_error() gives a one-line description of the last failure on the
  *     calling thread.
  *   - Outputs must not overlap the inputs or one another, except that
- *     qf_ste_backward mode 0 accepts grad_x == grad_y and then launches nothing.  The
- *     kernels read their inputs through the read-only (non-coherent) path.
+ *     qf_ste_backward accepts grad_x == grad_y (mode 0 then launches nothing; mode 1
+ *     reads the gradient with ordinary loads, each element before it is written).
+ *     The kernels read x through the read-only (non-coherent) path.
  *   - Calls on the same stream are ordered; calls whose outputs overlap and that
  *     run concurrently on different streams race.
  *   - Numerics are fixed bit for bit (see each call); every result is

@@ -392,3 +392,22 @@ def test_full_q4k_mse_sampled_rows():
     for i, x in enumerate(wl["tensors"]):
         compare_rows("q4k_mse", x, res["y"][i], res["codes"][i], None,
                      sample_rows(x.shape[0], 24, 500 + i), label=f"q4k mse[{i}]")
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4", "q4k"])
+def test_clipped_ste_in_place(fmt):
+    """Clipped STE with grad_x == grad_y gives the out-of-place result (and the oracle's)."""
+    wl = workloads.nvfp4_tied(rows_scale=1 / 64)
+    x = wl["tensors"][3]
+    gy = wl["grads"][3]
+    am = float(oracle.amax(x))
+    want = oracle.ste_backward(gy, 1, fmt, x, am)
+    xd, g1 = x.to(DEV), gy.to(DEV)
+    amax = torch.tensor([am], device=DEV)
+    out = torch.empty_like(g1)
+    qf.qf_ste_backward(g1, out, 1, fmt, xd, 0, amax)
+    g2 = gy.to(DEV)
+    qf.qf_ste_backward(g2, g2, 1, fmt, xd, 0, amax)               # in place
+    torch.cuda.synchronize()
+    assert_same(f"{fmt} clipped STE", bits(out), want)
+    assert_same(f"{fmt} clipped STE in place", bits(g2), want)
