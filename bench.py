@@ -391,6 +391,27 @@ def run_ours(args, rank, world, local_rank):
     return result
 
 
+def graph_timed(fn, iters, flush):
+    """Median device time (ms) of `fn` captured once in a CUDA graph and replayed, so
+    the host's launch rate is not what is measured; None if capture fails."""
+    try:
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            fn()                                    # fills the host-side caches
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        t = timed_calls(g.replay, iters, 2, flush)
+        del g
+        return t
+    except Exception:                               # noqa: BLE001 (reported as unavailable)
+        torch.cuda.synchronize()
+        return None
+
+
 class L2Flush:
     """Evicts the timed kernel's data from L2 between timed calls.
 
@@ -508,7 +529,39 @@ def per_format(qf, dev, args, l2):
                 for c in calls:
                     c()
             t_loop = timed_calls(looped, max(3, it // 4), 1, flush)
-            d.update({"one_expert_at_a_time_us": t_loop * 1e3, "grouped_speedup": t_loop / t_fq})
+            t_loop_g = graph_timed(looped, max(3, it // 4), flush)
+            d.update({"one_expert_at_a_time_us": t_loop * 1e3, "grouped_speedup": t_loop / t_fq,
+                      "one_expert_at_a_time_graph_us": None if t_loop_g is None else t_loop_g * 1e3})
+            if fmt == "nvfp4":
+                # the whole NVFP4 step one expert at a time (amax of its two tie groups, then
+                # its fused pass): two calls per expert, or one qf_amax_fakequant per expert
+                # (a 9.4 MB expert takes the single-launch path)
+                ws = qf.alloc_workspace(2, dev)
+                two, one = [], []
+                for e in range(n // 3):
+                    sl = slice(3 * e, 3 * e + 3)
+                    am_e = torch.empty(2, device=dev)
+                    two.append((qf.prepare_amax_tied(xs[sl], [0, 0, 1], am_e),
+                                qf.prepare_fakequant(fmt, xs[sl], Y[sl], C[sl], S[sl], [0, 0, 1],
+                                                     am_e)))
+                    one.append(qf.prepare_amax_fakequant(xs[sl], Y[sl], C[sl], S[sl], [0, 0, 1],
+                                                         am_e, workspace=ws))
+
+                def two_loop():
+                    for a, b in two:
+                        a()
+                        b()
+
+                def one_loop():
+                    for c in one:
+                        c()
+                # replayed from CUDA graphs: host launch cost out of the measurement
+                t2 = graph_timed(two_loop, max(3, it // 4), flush)
+                t1 = graph_timed(one_loop, max(3, it // 4), flush)
+                d.update({"step_one_expert_at_a_time_two_calls_graph_us":
+                          None if t2 is None else t2 * 1e3,
+                          "step_one_expert_at_a_time_one_launch_graph_us":
+                          None if t1 is None else t1 * 1e3})
         out[name] = d
         del W
         torch.cuda.empty_cache()
