@@ -27,7 +27,10 @@
 
 namespace qf {
 
-constexpr int kLoraRows = 32;      // rows per CTA unit
+#ifndef QF_LORA_ROWS
+#define QF_LORA_ROWS 64
+#endif
+constexpr int kLoraRows = QF_LORA_ROWS;   // rows per CTA unit (a multiple of 4)
 constexpr int kLoraCols = 1024;    // columns per CTA unit (8 warps x 128)
 constexpr int kLoraThreads = 256;
 
