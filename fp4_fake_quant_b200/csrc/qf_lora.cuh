@@ -10,8 +10,8 @@
 // fixed order makes the result reproducible bit for bit (tensor cores are not
 // used because their accumulation order is not specified).
 //
-// Layout: lane l owns 4 consecutive columns, a warp a 128-column slab, a CTA 8
-// slabs (1024 columns) by kLoraRows rows.  The warp keeps its A slab (r x 4 FP32)
+// Layout: lane l owns 4 consecutive columns, a warp a 128-column slab, a CTA
+// kLoraThreads / 32 slabs (1024 columns at 256 threads) by kLoraRows rows.  The warp keeps its A slab (r x 4 FP32)
 // in registers across the CTA's rows; the CTA stages its kLoraRows rows of B in
 // shared memory as FP32, so every B read is a broadcast.  W, y and codes accesses
 // are contiguous 256-, 256- and 64-byte warp runs per row.
@@ -31,8 +31,11 @@ namespace qf {
 #define QF_LORA_ROWS 64
 #endif
 constexpr int kLoraRows = QF_LORA_ROWS;   // rows per CTA unit (a multiple of 4)
-constexpr int kLoraCols = 1024;    // columns per CTA unit (8 warps x 128)
-constexpr int kLoraThreads = 256;
+#ifndef QF_LORA_THREADS
+#define QF_LORA_THREADS 256
+#endif
+constexpr int kLoraThreads = QF_LORA_THREADS;
+constexpr int kLoraCols = kLoraThreads / 32 * 128;   // columns per CTA unit (128 per warp)
 
 // kLoraMergeAmax writes the merged weight like kLoraMerge and folds its max |M| into
 // the tie-group amax like kLoraAmax, in one pass.
