@@ -860,12 +860,10 @@ qf_status qf_ste_backward(qf_format f, const void* grad_y, void* grad_x, int64_t
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (mode == 0) {
         if (numel == 0 || grad_x == grad_y) return QF_OK;
-        Launch L;
-        qf_status st = launch_shape(qf::k_copy, kThreads, 1, &L);
-        if (st != QF_OK) return st;
-        const int64_t vec = (numel + 7) / 8;
-        const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(
-            (vec + kThreads - 1) / kThreads, int64_t(L.sms) * L.per_sm));
+        if (overlap(grad_y, numel * 2, grad_x, numel * 2))
+            return fail(QF_ERR_INVALID_ARG, "grad_x overlaps grad_y without being equal to it");
+        const int64_t vec = numel / 8;
+        const int grid = (int)std::max<int64_t>(1, (vec + 4 * kThreads - 1) / (4 * kThreads));
         qf::k_copy<<<grid, kThreads, 0, s>>>(static_cast<const uint16_t*>(grad_y),
                                              static_cast<uint16_t*>(grad_x), numel);
         cudaError_t e = cudaGetLastError();

@@ -1037,18 +1037,20 @@ __global__ void k_amax_tail(const __grid_constant__ Table<MAXT> P) {
 // ------------------------------------------------------------------ STE identity
 __global__ void __launch_bounds__(kThreads) k_copy(const uint16_t* __restrict__ src,
                                                    uint16_t* __restrict__ dst, int64_t n) {
+    // one CTA per 4 * kThreads 16-byte vectors, all four loads in flight before the stores
     const int64_t nvec = n >> 3;
-    const int64_t stride = int64_t(gridDim.x) * kThreads;
-    int64_t i = int64_t(blockIdx.x) * kThreads + threadIdx.x;
-    for (; i + 3 * stride < nvec; i += 4 * stride) {
-        uint4 a = ld_stream<1>(src + 8 * i), b = ld_stream<1>(src + 8 * (i + stride));
-        uint4 c = ld_stream<1>(src + 8 * (i + 2 * stride)), d = ld_stream<1>(src + 8 * (i + 3 * stride));
-        st_v4(dst + 8 * i, a);
-        st_v4(dst + 8 * (i + stride), b);
-        st_v4(dst + 8 * (i + 2 * stride), c);
-        st_v4(dst + 8 * (i + 3 * stride), d);
+    const int64_t base = int64_t(blockIdx.x) * (4 * kThreads) + threadIdx.x;
+    uint4 v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int64_t i = base + j * kThreads;
+        if (i < nvec) v[j] = ld_stream<0>(src + 8 * i);
     }
-    for (; i < nvec; i += stride) st_v4(dst + 8 * i, ld_stream<1>(src + 8 * i));
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int64_t i = base + j * kThreads;
+        if (i < nvec) st_v4(dst + 8 * i, v[j]);
+    }
     if (blockIdx.x == 0 && threadIdx.x < (n & 7)) {
         const int64_t e = (nvec << 3) + threadIdx.x;
         dst[e] = src[e];

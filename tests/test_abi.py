@@ -168,6 +168,7 @@ def test_amax_and_ste_validation(qf):
     assert lib.qf_ste_backward(0, 0x1008, 0x2000, 64, 0, None, None, 0, None) == ALIGN
     assert lib.qf_ste_backward(0, 0, 0x2000, 64, 0, None, None, 0, None) == INV
     assert lib.qf_ste_backward(0, 0x1000, 0x1000, 64, 0, None, None, 0, None) == 0  # aliased
+    assert lib.qf_ste_backward(0, 0x1000, 0x1010, 64, 0, None, None, 0, None) == INV  # partly
     assert lib.qf_ste_backward(9, 0x1000, 0x2000, 256, 1, _tensor(qf), None, 0, None) == UNSUP
     assert lib.qf_ste_backward(1, 0x1000, 0x2000, 256, 1, None, None, 0, None) == INV
     assert lib.qf_ste_backward(1, 0x1000, 0x2000, 255, 1, _tensor(qf), None, 0, None) == SHAPE
