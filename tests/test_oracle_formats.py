@@ -531,3 +531,33 @@ def test_f32_codes_brute_force_and_decoder():
                           .astype(np.float64))
     y, b = oracle.q4k(x)
     assert np.array_equal(oracle.q4k_decode(b, xf.size), y)
+
+
+def test_codes_and_scales_stay_in_range():
+    """Every stored field is a valid value of its type, even for extreme inputs.
+    E4M3 scales are finite and at most 448 (never the NaN encodings 0x7F / 0xFF) and
+    never negative. E8M0 bytes are never 0xFF (NaN). Q4_K d and dmin are finite,
+    non-negative FP16, and sc, m fit 6 bits."""
+    rng = np.random.default_rng(11)
+    mags = [1e-30, 1e-6, 0.02, 1.0, 3e4, 3e38]
+    xs = []
+    for m in mags:
+        a = rng.standard_normal((4, 256)).astype(np.float32) * np.float32(m)
+        a[0, :7] = [0.0, -0.0, m, -m, 6 * m, -448 * m, 1e-45]
+        xs.append(workloads.to_bf16(a))
+    for x in xs:
+        xb = workloads.bf16_bits(x)
+        f = np.abs(x.float().numpy())
+        if np.isfinite(f).all() and f.max() < 1e38:
+            _, _, sc, _ = oracle.nvfp4(xb, float(f.max()))
+            assert not np.any((sc & 0x7F) == 0x7F) and not np.any(sc & 0x80)
+            assert np.all(sc.view(ml_dtypes.float8_e4m3fn).astype(np.float32) <= 448.0)
+        _, _, e8 = oracle.mxfp4(xb)
+        assert not np.any(e8 == 0xFF)
+        if f.max() < 4e6:                      # inside the Q4_K range: 63 * 65504 bounds min_j
+            _, blocks = oracle.q4k(xb)
+            blk = blocks.reshape(-1, 144)
+            d = blk[:, 0:2].copy().view(np.float16).astype(np.float32)
+            dm = blk[:, 2:4].copy().view(np.float16).astype(np.float32)
+            assert np.isfinite(d).all() and np.isfinite(dm).all()
+            assert (d >= 0).all() and (dm >= 0).all()
