@@ -72,15 +72,28 @@ class ClockSampler:
 
     def __init__(self, index: int):
         self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.matched = None
         self._stop = threading.Event()
         try:
             import pynvml
             pynvml.nvmlInit()
             self.nv = pynvml
-            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.h, self.matched = self._handle(pynvml, index)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
         except Exception:
             self.nv = None
+
+    @staticmethod
+    def _handle(pynvml, index: int):
+        """The NVML handle of CUDA device `index`.  NVML numbers every GPU of the machine
+        while CUDA numbers the visible ones (CUDA_VISIBLE_DEVICES), so the device is
+        found by its UUID; the index is the fallback."""
+        try:
+            u = str(torch.cuda.get_device_properties(index).uuid)
+            u = u if u.startswith("GPU-") else "GPU-" + u
+            return pynvml.nvmlDeviceGetHandleByUUID(u.encode()), "uuid"
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(index), "index"
 
     def sample_once(self):
         if self.nv is None:
@@ -111,7 +124,8 @@ class ClockSampler:
         if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["nvml unavailable"]}
         return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+                "reasons": sorted(self.reasons), "samples": len(self.samples),
+                "device_by": self.matched}
 
 
 def csrc_digest() -> str:
