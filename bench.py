@@ -658,7 +658,7 @@ def _oracle_pass(fmt, tensors, threads):
             elif fmt == "mxfp4":
                 list(pool.map(oracle.mxfp4, parts))
             else:
-                list(pool.map(oracle.q4k, parts))
+                list(pool.map(lambda p: oracle.q4k(p, mse=fmt == "q4k_mse"), parts))
             n += x.numel()
     return n
 
@@ -668,11 +668,19 @@ def cpu_baseline(name, frac):
     host core of this process's affinity mask, and on one core."""
     import oracle
     oracle.build()
-    wl = {"w4a4": workloads.mxfp4_w4a4, "q4k": workloads.q4k_weights,
-          "nvfp4_tied": lambda: workloads.nvfp4_tied(with_grads=False),
-          "nvfp4_weight": workloads.nvfp4_weight, "activation": workloads.nvfp4_activation,
-          }.get(name, workloads.mxfp4_w4a4)()
-    fmt = {"w4a4": "mxfp4", "q4k": "q4k"}.get(name, "nvfp4")
+    gen = {"w4a4": workloads.mxfp4_w4a4, "q4k": workloads.q4k_weights,
+           "q4k_mse": workloads.q4k_weights,
+           "q4k_f32": lambda: workloads.q4k_weights(dtype="f32"),
+           "nvfp4_tied": lambda: workloads.nvfp4_tied(with_grads=False),
+           "nvfp4_tied_f32": lambda: workloads.nvfp4_tied(with_grads=False, dtype="f32"),
+           "nvfp4_weight": workloads.nvfp4_weight, "activation": workloads.nvfp4_activation,
+           "moe_nvfp4": workloads.moe_experts, "moe_mxfp4": workloads.moe_experts,
+           "moe_q4k": workloads.moe_experts}
+    fmt = {"w4a4": "mxfp4", "q4k": "q4k", "q4k_mse": "q4k_mse", "q4k_f32": "q4k",
+           "moe_mxfp4": "mxfp4", "moe_q4k": "q4k"}.get(name, "nvfp4")
+    if name not in gen:                     # LoRA: the oracle's fake-quant of the bases alone
+        gen[name] = lambda: workloads.nvfp4_tied(with_grads=False)
+    wl = gen[name]()
     sample = [x[: max(1, int(x.shape[0] * frac))] for x in wl["tensors"]]
     cores = _host_cores()
     t0 = time.perf_counter()
@@ -682,11 +690,12 @@ def cpu_baseline(name, frac):
     t0 = time.perf_counter()
     n1 = _oracle_pass(fmt, one, 1)
     dt_one = time.perf_counter() - t0
-    return {"value": n * BYTES_PER_ELEM[fmt] / dt_all / 1e9, "unit": UNIT, "cores": cores,
+    bpe = BYTES_PER_ELEM[fmt] + sample[0].element_size() - 2      # FP32 input reads 4 B
+    return {"value": n * bpe / dt_all / 1e9, "unit": UNIT, "cores": cores,
             "kind": "oracle",
             "sample": f"first {frac:.3g} of the rows of every tensor ({n} elements), scalar C, "
                       f"rows split over {cores} host threads, {dt_all:.1f} s",
-            "single_core_value": n1 * BYTES_PER_ELEM[fmt] / dt_one / 1e9,
+            "single_core_value": n1 * bpe / dt_one / 1e9,
             "single_core_sample": f"a quarter of that sample ({n1} elements) on one thread, "
                                   f"{dt_one:.1f} s"}
 
