@@ -11,16 +11,25 @@
 // used because their accumulation order is not specified).
 //
 // Layout: lane l owns 4 consecutive columns, a warp a 128-column slab, a CTA
-// kLoraThreads / 32 slabs (1024 columns at 256 threads) by kLoraRows rows.  The warp keeps its A slab (r x 4 FP32)
-// in registers across the CTA's rows; the CTA stages its kLoraRows rows of B in
-// shared memory as FP32, so every B read is a broadcast.  W, y and codes accesses
-// are contiguous 256-, 256- and 64-byte warp runs per row.
+// kLoraThreads / 32 slabs (1024 columns at 256 threads) by kLoraRows rows.  The warp
+// keeps its A slab (r x 4 FP32) in registers across the CTA's rows; the CTA stages its
+// kLoraRows rows of B in shared memory as FP32, so every B read is a broadcast.  W, y
+// and codes accesses are contiguous 256-, 256- and 64-byte warp runs per row.
 //
 // The products run on sm_100's paired FP32 pipe: one fma.rn.f32x2 updates the
 // accumulators of two adjacent columns, each rounded exactly as a scalar
 // fma.rn.f32 would be (and, the products being exact, as a separate multiply and
-// add would be).  B is stored in shared memory with every value twice, so one
-// 16-byte load yields the (b, b) operand pairs of two consecutive k.
+// add would be).  Operands and accumulators live in 64-bit registers from load to
+// use, so no pair is ever repacked.  B is stored in shared memory with every value
+// twice, so one 16-byte load yields the (b, b) operand pairs of two consecutive k.
+//
+// W arrives 4 rows per step.  The merge and amax modes, whose arithmetic per byte is
+// lightest, keep QF_LORA_STAGES steps of it in flight through a per-lane cp.async
+// ring in shared memory (each lane reads back only what it copied, so the ring needs
+// no barrier and its waits are the hardware's cp.async.wait_group); the quantizing
+// modes load the next step into registers and prefetch further rows to L2.  Whole
+// tiles of the merge and amax modes run a guard-free copy of the row loop.  Maxima
+// are taken on the packed BF16 merged values, two 16-bit magnitudes at a time.
 #pragma once
 
 #include "qf_device.cuh"
@@ -36,6 +45,18 @@ constexpr int kLoraRows = QF_LORA_ROWS;   // rows per CTA unit (a multiple of 4)
 #endif
 constexpr int kLoraThreads = QF_LORA_THREADS;
 constexpr int kLoraCols = kLoraThreads / 32 * 128;   // columns per CTA unit (128 per warp)
+#ifndef QF_LORA_STAGES
+#define QF_LORA_STAGES 4        // merge / amax modes: W ring depth in 4-row steps (cp.async)
+#endif
+#ifndef QF_LORA_NV_STAGES
+#define QF_LORA_NV_STAGES 0     // NVFP4 / MXFP4 modes: the same (0: register prefetch)
+#endif
+#ifndef QF_LORA_PF
+#define QF_LORA_PF 4            // with register prefetch: L2 prefetch distance, 4-row steps
+#endif
+#ifndef QF_LORA_FULL
+#define QF_LORA_FULL 1          // guard-free copy of the unit loop for whole tiles: 0 none,
+#endif                          // 1 merge / amax modes, 2 every mode
 
 // kLoraMergeAmax writes the merged weight like kLoraMerge and folds its max |M| into
 // the tie-group amax like kLoraAmax, in one pass.
@@ -78,11 +99,72 @@ __device__ __forceinline__ int lora_locate(const LoraTable<MAXT>& P, int64_t u) 
     return lo;
 }
 
+// Packed FP32 pairs kept in 64-bit registers from load to use, so the paired pipe's
+// operands need no repacking: lo = the pair's first (lower-address) value.
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+    uint64_t d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+    return d;
+}
+__device__ __forceinline__ float2 unpk2(uint64_t v) {
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+    return r;
+}
+// d = a * b + c on both halves, each rounded once (the products here are exact)
+__device__ __forceinline__ uint64_t fma2_pk(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+// per-half unsigned 16-bit max: the max |v| of BF16 pairs once their sign bits are cleared
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+// FP32 bits of the larger of the two BF16 magnitudes in a max_u16x2 result
+__device__ __forceinline__ uint32_t bf16x2_max_bits(uint32_t m) {
+    return max(m & 0xFFFFu, m >> 16) << 16;
+}
+
+// L2 prefetch of the line holding p; nothing waits for it
+__device__ __forceinline__ void prefetch_line_l2(const void* p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+// 8-byte asynchronous copy global -> shared; src_bytes = 0 writes zeros and reads nothing
+__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dst), "l"(src),
+                 "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// blocks (in hardware) until at most N of this thread's copy groups are pending
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr) : "memory");
+    return v;
+}
+
+template <bool B>
+struct FullTile { static constexpr bool value = B; };
+
 // R: compile-time rank capacity (the runtime rank is <= R; A and B are zero-padded,
 // which adds exact zeros to an accumulator that is never -0, so results do not change).
 template <int MODE, int R, int MAXT>
 __global__ void __launch_bounds__(kLoraThreads) k_lora(const __grid_constant__ LoraTable<MAXT> P) {
-    __shared__ __align__(16) float2 bsm[kLoraRows][R];      // (b, b) pairs
+    __shared__ __align__(16) uint64_t bsm[kLoraRows][R];     // (b, b) FP32 pairs
+    // W ring: every lane copies its own 8 bytes of each row into its own slots and reads
+    // only those back, so the ring needs no barrier (48 KB of static shared memory caps
+    // the depth at rank 32)
+    constexpr int kWantStages = MODE == kLoraNV || MODE == kLoraMX ? QF_LORA_NV_STAGES
+                                                                   : QF_LORA_STAGES;
+    constexpr int kStages = R > 16 && kWantStages > 3 ? 3 : kWantStages;
+    constexpr int kPf = kStages == 0 ? QF_LORA_PF : 0;
+    constexpr int kRing = kStages > 0 ? kStages : 1;
+    __shared__ __align__(16) uint2 wring[kRing][4][kLoraThreads];
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int64_t cu = blockIdx.x;
     constexpr bool kWritesMerged = MODE == kLoraMerge || MODE == kLoraMergeAmax;
@@ -98,24 +180,38 @@ __global__ void __launch_bounds__(kLoraThreads) k_lora(const __grid_constant__ L
     const int64_t c_base = (local % T.col_groups) * kLoraCols;
     const int64_t rows_left = T.rows - r0;
     const int nrows = rows_left < kLoraRows ? (int)rows_left : kLoraRows;
+    const int64_t cols = T.cols;
     const int64_t col0 = c_base + wid * 128 + lane * 4;
-    const bool colok = col0 < T.cols;          // cols % 16 == 0: a lane is all in or all out
+    const bool colok = col0 < cols;            // cols % 16 == 0: a lane is all in or all out
     const int rank = T.rank;
+    const float scale = T.scale;
+
+    // with register prefetch, W rows reach L2 kPf 4-row steps before the step that
+    // loads them: the warp's slab of a row is 256 bytes (fewer at the last column
+    // group), two lines, one lane each
+    const int64_t wcol0 = c_base + wid * 128;
+    const int pf_bytes = wcol0 < cols ? (int)(min(cols - wcol0, (int64_t)128) * 2) : 0;
+    const uint16_t* wslab = T.w + r0 * cols + wcol0;
+    if (kPf > 0) {
+        for (int rr = lane >> 1; rr < 4 * kPf; rr += 16)
+            if (128 * (lane & 1) < pf_bytes && 4 + rr < nrows)
+                prefetch_line_l2(wslab + (4 + rr) * cols + 64 * (lane & 1));
+    }
 
     // this CTA's rows of B as FP32, zero-padded to R
     for (int idx = threadIdx.x; idx < kLoraRows * R; idx += kLoraThreads) {
         const int i = idx / R, k = idx % R;
         const float b = (i < nrows && k < rank) ? bf16_lo(T.b[(r0 + i) * rank + k]) : 0.0f;
-        bsm[i][k] = make_float2(b, b);
+        bsm[i][k] = pk2(b, b);
     }
     // this lane's 4 columns of A as FP32 pairs (columns 0,1 and 2,3), zero-padded to R
-    float2 a[R][2];
+    uint64_t a[R][2];
 #pragma unroll
     for (int k = 0; k < R; ++k) {
         uint2 v = make_uint2(0, 0);
-        if (k < rank && colok) v = *reinterpret_cast<const uint2*>(T.a + k * T.cols + col0);
-        a[k][0] = make_float2(bf16_lo(v.x), bf16_hi(v.x));
-        a[k][1] = make_float2(bf16_lo(v.y), bf16_hi(v.y));
+        if (k < rank && colok) v = *reinterpret_cast<const uint2*>(T.a + k * cols + col0);
+        a[k][0] = pk2(bf16_lo(v.x), bf16_hi(v.x));
+        a[k][1] = pk2(bf16_lo(v.y), bf16_hi(v.y));
     }
     __syncthreads();
 
@@ -124,67 +220,100 @@ __global__ void __launch_bounds__(kLoraThreads) k_lora(const __grid_constant__ L
         s_t = nv_tensor_scale(P.group_amax[T.group]);
         six_st = __fmul_rn(6.0f, s_t);
     }
-    uint32_t run = 0;                          // amax mode: running max |M| (FP32 bits)
+    uint32_t run = 0;                          // amax modes: max |M| so far, per BF16 half
 
-    auto load_w = [&](int i0, uint2 (&wv)[4]) {
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-            const bool ok = colok && i0 + h < nrows;
-            wv[h] = ok ? *reinterpret_cast<const uint2*>(T.w + (r0 + i0 + h) * T.cols + col0)
-                       : make_uint2(0, 0);
-        }
-    };
-    uint2 wcur[4], wnxt[4];
-    load_w(0, wcur);
-    for (int i0 = 0; i0 < nrows; i0 += 4) {
-        if (i0 + 4 < nrows) load_w(i0 + 4, wnxt);          // the next 4 rows, in flight meanwhile
-        // merged values of 4 rows x this lane's 4 columns
-        float x[4][4];
-        uint32_t xw[4][2];                                   // the same, as packed BF16 pairs
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-            const int i = min(i0 + h, nrows - 1);            // rows past the end are not stored
-            float2 acc01 = make_float2(0.0f, 0.0f), acc23 = make_float2(0.0f, 0.0f);
-#pragma unroll
-            for (int k = 0; k < R; k += 2) {
-                const float4 bk = *reinterpret_cast<const float4*>(&bsm[i][k]);
-                const float2 b0 = make_float2(bk.x, bk.y), b1 = make_float2(bk.z, bk.w);
-                acc01 = fma2_rn(b0, a[k][0], acc01);
-                acc23 = fma2_rn(b0, a[k][1], acc23);
-                acc01 = fma2_rn(b1, a[k + 1][0], acc01);
-                acc23 = fma2_rn(b1, a[k + 1][1], acc23);
-            }
-            // scalar: a paired product must not feed an add (see mul2_rn)
-            xw[h][0] = cvt_bf16x2(__fadd_rn(bf16_hi(wcur[h].x), __fmul_rn(T.scale, acc01.y)),
-                                  __fadd_rn(bf16_lo(wcur[h].x), __fmul_rn(T.scale, acc01.x)));
-            xw[h][1] = cvt_bf16x2(__fadd_rn(bf16_hi(wcur[h].y), __fmul_rn(T.scale, acc23.y)),
-                                  __fadd_rn(bf16_lo(wcur[h].y), __fmul_rn(T.scale, acc23.x)));
-            x[h][0] = bf16_lo(xw[h][0]); x[h][1] = bf16_hi(xw[h][0]);
-            x[h][2] = bf16_lo(xw[h][1]); x[h][3] = bf16_hi(xw[h][1]);
-        }
-        if (kWritesMerged) {
+    // One CTA unit: FULL when all kLoraRows rows exist and the lane's columns do, so no
+    // access needs a guard.  Otherwise rows past the end re-read the last row (their
+    // merged values repeat that row's, which leaves every max unchanged, and they are
+    // never stored) and a lane past the last column reads zeros (merged value +0).
+    const uint16_t* wbase = T.w + r0 * cols + col0;
+    auto unit = [&](auto tag) {
+        constexpr bool FULL = decltype(tag)::value;
+        const int n = FULL ? kLoraRows : nrows;
+        auto row = [&](int i) { return FULL ? i : min(i, n - 1); };
+        auto load_w = [&](int i0, uint2 (&wv)[4]) {
 #pragma unroll
             for (int h = 0; h < 4; ++h)
-                if (colok && i0 + h < nrows && T.y)
-                    *reinterpret_cast<uint2*>(T.y + (r0 + i0 + h) * T.cols + col0) =
-                        make_uint2(xw[h][0], xw[h][1]);
+                wv[h] = (FULL || colok)
+                            ? *reinterpret_cast<const uint2*>(wbase + row(i0 + h) * cols)
+                            : make_uint2(0, 0);
+        };
+        const uint32_t ring = (uint32_t)__cvta_generic_to_shared(&wring[0][0][threadIdx.x]);
+        // rows 4 it .. 4 it + 3 into ring stage it % kStages (one copy group per step,
+        // empty past the last row, so the group count stays uniform)
+        auto issue = [&](int it) {
+            if (4 * it < n) {
+                const uint32_t dst = ring + (uint32_t)((it % kRing) * 4 * kLoraThreads * 8);
+#pragma unroll
+                for (int h = 0; h < 4; ++h)
+                    cp_async8(dst + h * kLoraThreads * 8,
+                              (FULL || colok) ? (const void*)(wbase + row(4 * it + h) * cols)
+                                              : (const void*)T.w,
+                              (FULL || colok) ? 8u : 0u);
+            }
+            cp_async_commit();
+        };
+        uint2 wcur[4], wnxt[4];
+        if constexpr (kStages > 0) {
+#pragma unroll
+            for (int st = 0; st < kStages - 1; ++st) issue(st);
+        } else {
+            load_w(0, wcur);
         }
-        if (MODE != kLoraMerge) {
-            uint32_t m[4];
+#pragma unroll 1
+        for (int i0 = 0; i0 < n; i0 += 4) {
+            if constexpr (kStages > 0) {
+                const int it = i0 >> 2;
+                cp_async_wait<kStages - 2>();              // this step's group has landed
+                const uint32_t src = ring + (uint32_t)((it % kRing) * 4 * kLoraThreads * 8);
+#pragma unroll
+                for (int h = 0; h < 4; ++h) wcur[h] = lds64(src + h * kLoraThreads * 8);
+                issue(it + kStages - 1);                   // refills the stage read last step
+            }
+            if (kPf > 0 && lane < 8) {
+                const int rr = i0 + 4 + 4 * kPf + (lane >> 1);
+                if (128 * (lane & 1) < pf_bytes && rr < nrows)
+                    prefetch_line_l2(wslab + rr * cols + 64 * (lane & 1));
+            }
+            if (kStages == 0 && i0 + 4 < n) load_w(i0 + 4, wnxt);   // next 4 rows, in flight
+            // merged values of 4 rows x this lane's 4 columns, as packed BF16 pairs
+            uint32_t xw[4][2];
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
-                m[h] = 0;
+                const int i = row(i0 + h);
+                uint64_t acc01 = 0, acc23 = 0;           // (+0, +0)
 #pragma unroll
-                for (int c = 0; c < 4; ++c) m[h] = max(m[h], __float_as_uint(x[h][c]) & 0x7FFFFFFFu);
+                for (int k = 0; k < R; k += 2) {
+                    const ulonglong2 bk = *reinterpret_cast<const ulonglong2*>(&bsm[i][k]);
+                    acc01 = fma2_pk(bk.x, a[k][0], acc01);
+                    acc23 = fma2_pk(bk.x, a[k][1], acc23);
+                    acc01 = fma2_pk(bk.y, a[k + 1][0], acc01);
+                    acc23 = fma2_pk(bk.y, a[k + 1][1], acc23);
+                }
+                // scalar: a paired product must not feed an add (see mul2_rn)
+                const float2 s01 = unpk2(acc01), s23 = unpk2(acc23);
+                xw[h][0] = cvt_bf16x2(__fadd_rn(bf16_hi(wcur[h].x), __fmul_rn(scale, s01.y)),
+                                      __fadd_rn(bf16_lo(wcur[h].x), __fmul_rn(scale, s01.x)));
+                xw[h][1] = cvt_bf16x2(__fadd_rn(bf16_hi(wcur[h].y), __fmul_rn(scale, s23.y)),
+                                      __fadd_rn(bf16_lo(wcur[h].y), __fmul_rn(scale, s23.x)));
+            }
+            if (kWritesMerged) {
+#pragma unroll
+                for (int h = 0; h < 4; ++h)
+                    if (FULL || (colok && i0 + h < n))
+                        *reinterpret_cast<uint2*>(T.y + (r0 + i0 + h) * cols + col0) =
+                            make_uint2(xw[h][0], xw[h][1]);
             }
             if (kFoldsAmax) {
 #pragma unroll
                 for (int h = 0; h < 4; ++h)
-                    if (i0 + h < nrows) run = max(run, m[h]);
-            } else {
+                    run = max_u16x2(run, max_u16x2(xw[h][0] & 0x7FFF7FFFu, xw[h][1] & 0x7FFF7FFFu));
+            } else if (MODE == kLoraNV || MODE == kLoraMX) {
                 // block max over the 4 (NVFP4, 16 elements) or 8 (MXFP4, 32) lanes of the block
+                uint32_t m[4];
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
+                    m[h] = bf16x2_max_bits(max_u16x2(xw[h][0] & 0x7FFF7FFFu, xw[h][1] & 0x7FFF7FFFu));
                     m[h] = max(m[h], __shfl_xor_sync(kFull, m[h], 1));
                     m[h] = max(m[h], __shfl_xor_sync(kFull, m[h], 2));
                     if (MODE == kLoraMX) m[h] = max(m[h], __shfl_xor_sync(kFull, m[h], 4));
@@ -216,18 +345,20 @@ __global__ void __launch_bounds__(kLoraThreads) k_lora(const __grid_constant__ L
                 }
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
+                    const float x[4] = {bf16_lo(xw[h][0]), bf16_hi(xw[h][0]),
+                                        bf16_lo(xw[h][1]), bf16_hi(xw[h][1])};
                     const float2 inv2 = make_float2(inv[h], inv[h]);
-                    const float2 q01 = mul2_rn(make_float2(x[h][0], x[h][1]), inv2);
-                    const float2 q23 = mul2_rn(make_float2(x[h][2], x[h][3]), inv2);
+                    const float2 q01 = mul2_rn(make_float2(x[0], x[1]), inv2);
+                    const float2 q23 = mul2_rn(make_float2(x[2], x[3]), inv2);
                     float q[4] = {q01.x, q01.y, q23.x, q23.y};
                     if (MODE == kLoraNV && __builtin_expect(isinf(inv[h]), 0)) {
 #pragma unroll
                         for (int c = 0; c < 4; ++c)
-                            if (x[h][c] == 0.0f) q[c] = x[h][c];
+                            if (x[c] == 0.0f) q[c] = x[c];
                     }
                     const uint32_t b0 = cvt_e2m1x2(q[1], q[0]), b1 = cvt_e2m1x2(q[3], q[2]);
-                    if (!colok || i0 + h >= nrows) continue;
-                    const int64_t e = (r0 + i0 + h) * T.cols + col0;   // flat element index
+                    if (!FULL && (!colok || i0 + h >= n)) continue;
+                    const int64_t e = (r0 + i0 + h) * cols + col0;   // flat element index
                     if (T.y) {
                         const uint32_t h0 = cvt_e2m1x2_f16x2(b0), h1 = cvt_e2m1x2_f16x2(b1);
                         const float2 S2 = make_float2(S[h], S[h]);
@@ -242,13 +373,22 @@ __global__ void __launch_bounds__(kLoraThreads) k_lora(const __grid_constant__ L
                         T.scales[e >> (MODE == kLoraNV ? 4 : 5)] = (uint8_t)sbyte[h];
                 }
             }
-        }
+            if constexpr (kStages == 0) {
 #pragma unroll
-        for (int h = 0; h < 4; ++h) wcur[h] = wnxt[h];
-    }
+                for (int h = 0; h < 4; ++h) wcur[h] = wnxt[h];
+            }
+        }
+        if constexpr (kStages > 0) cp_async_wait<0>();
+    };
+    constexpr bool kSplitFull = QF_LORA_FULL == 2 || (QF_LORA_FULL == 1 && MODE != kLoraNV &&
+                                                      MODE != kLoraMX);
+    if (kSplitFull && nrows == kLoraRows && colok) unit(FullTile<true>{});
+    else unit(FullTile<false>{});
+
     if (kFoldsAmax) {
         // one atomic per CTA (its unit lies in one tensor), not one per warp
         __shared__ uint32_t wmax[kLoraThreads / 32];
+        run = bf16x2_max_bits(run);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) run = max(run, __shfl_xor_sync(kFull, run, o));
         if (lane == 0) wmax[wid] = run;
