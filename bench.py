@@ -64,6 +64,24 @@ def peaks():
     return 6650.0, "fallback"
 
 
+# The MSE-searched Q4_K fit is bound by FP32 arithmetic, not by HBM.  Its algorithmic
+# work per element: x + min once; for each of the nine trial scales the scaled value,
+# the clamp to [0, 15] (two operations), the rounding, s*q - min (two), x - dq and the
+# squared-error update (two), 9 operations; the sub-block min/max scan (two); the final
+# quantize-dequantize (x + mm, the product, clamp, rounding, s*q - mm) and the BF16
+# rounding (eight).  Each counts as one lane-slot of the FP32 pipe; per-sub-block work
+# (the trial divides, the 6-bit scale fit) is left out.
+MSE_OPS_PER_ELEM = 1 + 9 * 9 + 2 + 8
+FP32_LANES_PER_SM = 128                       # 4 SM sub-partitions x 32 FP32 lanes
+
+
+def fp32_peak_tops(dev, sm_max_mhz) -> tuple:
+    """FP32 pipe peak in tera-operations/s: SMs x 128 lanes x the maximum SM clock."""
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    mhz, src = (float(sm_max_mhz), "NVML max SM clock") if sm_max_mhz else (1965.0, "1965 MHz")
+    return sms * FP32_LANES_PER_SM * mhz * 1e6 / 1e12, f"{sms} SMs x 128 FP32 lanes x {src}"
+
+
 class ClockSampler:
     """Samples the SM clock and the clock-event reasons through NVML (read only)."""
 
@@ -371,11 +389,23 @@ def run_ours(args, rank, world, local_rank):
 
     peak, peak_kind = peaks()
     achieved = W["fq_bytes"] / (kern_ms * 1e-3) / 1e9
-    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "traffic": traffic_for(W["kernel"], W["name"]),
-                "peak_source": f"{peak_kind} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
-                "kernel": W["kernel"], "bytes_per_launch": W["fq_bytes"],
-                "launch_us": kern_ms * 1e3}
+    clocks = clk.summary()
+    if W["fmt"] == "q4k_mse":
+        tops, how = fp32_peak_tops(dev, clocks.get("sm_max_mhz"))
+        ach = numel * MSE_OPS_PER_ELEM / (kern_ms * 1e-3) / 1e12
+        roofline = {"bound": "alu", "achieved": ach, "peak": tops, "unit": "TOP/s",
+                    "frac": ach / tops, "traffic": traffic_for(W["kernel"], W["name"]),
+                    "peak_source": f"derived: {how}",
+                    "ops_per_element": MSE_OPS_PER_ELEM, "kernel": W["kernel"],
+                    "ops_per_launch": numel * MSE_OPS_PER_ELEM, "launch_us": kern_ms * 1e3,
+                    "hbm": {"achieved": achieved, "peak": peak, "unit": "GB/s",
+                            "frac": achieved / peak}}
+    else:
+        roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                    "frac": achieved / peak, "traffic": traffic_for(W["kernel"], W["name"]),
+                    "peak_source": f"{peak_kind} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                    "kernel": W["kernel"], "bytes_per_launch": W["fq_bytes"],
+                    "launch_us": kern_ms * 1e3}
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -394,12 +424,12 @@ def run_ours(args, rank, world, local_rank):
         "roofline": roofline,
         "e2e": e2e,
         "gpu_launches": args.steps * W["launches"],
-        "clocks": clk.summary(),
+        "clocks": clocks,
     }
     del W, flush_buf
     torch.cuda.empty_cache()
     if rank == 0 and world == 1 and not args.no_per_format:
-        result["per_format"] = per_format(qf, dev, args, l2)
+        result["per_format"] = per_format(qf, dev, args, l2, clocks.get("sm_max_mhz"))
         result["export"] = export_timing(qf, dev)
     if rank == 0 and world == 1 and not args.no_cpu:
         result["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_rows_frac)
@@ -461,7 +491,7 @@ def timed_calls(fn, iters, warm, flush):
     return float(statistics.median(times))
 
 
-def per_format(qf, dev, args, l2):
+def per_format(qf, dev, args, l2, sm_max_mhz=None):
     peak, _ = peaks()
     flush = L2Flush(dev, l2)
     out = {}
@@ -482,6 +512,11 @@ def per_format(qf, dev, args, l2):
              # back-to-back calls without a flush: a tensor that fits in L2 is read from it
              "fused_hot_l2_us": t_hot * 1e3,
              "fused_hot_l2_GB/s": fq_bytes / (t_hot * 1e-3) / 1e9}
+        if W["fmt"] == "q4k_mse":
+            tops, how = fp32_peak_tops(dev, sm_max_mhz)
+            ach = W["numel"] * MSE_OPS_PER_ELEM / (t_fq * 1e-3) / 1e12
+            d["alu_bound"] = {"ops_per_element": MSE_OPS_PER_ELEM, "achieved_TOP/s": ach,
+                              "peak_TOP/s": tops, "frac": ach / tops, "peak_source": how}
         if pre_fn is not None:
             t_pre = timed_calls(pre_fn, it, warm, flush)
             t_step = timed_calls(lambda: run_step(W), it, warm, flush)

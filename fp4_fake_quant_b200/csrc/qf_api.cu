@@ -235,9 +235,11 @@ template <typename XT, int MAXT, int MODE>
 constexpr auto mx_kernel() {
     return qf::k_fp4<false, XT, kFp4U, MAXT, MODE, QF_MX_THREADS, QF_MX_PREFETCH>;
 }
+template <typename XT>
+constexpr int q4k_threads() { return sizeof(XT) == 2 ? QF_Q4K_THREADS : QF_Q4K_F32_THREADS; }
 template <typename XT, int MAXT, int MODE, bool MSE>
 constexpr auto q4k_kernel() {
-    return qf::k_q4k<XT, MAXT, MODE, QF_Q4K_THREADS, MSE>;
+    return qf::k_q4k<XT, MAXT, MODE, q4k_threads<XT>(), MSE>;
 }
 
 template <typename XT>
@@ -263,18 +265,18 @@ qf_status launch_format_t(qf_format f, int mode, const std::vector<DevTensor>& v
     if (f == QF_Q4K_MSE) {
         if (mode == 0)
             return launch_chunks(q4k_kernel<XT, kSmallT, 0, true>(),
-                                 q4k_kernel<XT, kLargeT, 0, true>(), QF_Q4K_THREADS,
+                                 q4k_kernel<XT, kLargeT, 0, true>(), q4k_threads<XT>(),
                                  QF_Q4K_WAVES, v, 1024, nullptr, nullptr, nullptr, 0, s);
         return launch_chunks(q4k_kernel<XT, kSmallT, 1, true>(), q4k_kernel<XT, kLargeT, 1, true>(),
-                             QF_Q4K_THREADS, QF_Q4K_WAVES, v, 1024, nullptr, nullptr, nullptr, 0,
+                             q4k_threads<XT>(), QF_Q4K_WAVES, v, 1024, nullptr, nullptr, nullptr, 0,
                              s);
     }
     if (mode == 0)
         return launch_chunks(q4k_kernel<XT, kSmallT, 0, false>(),
-                             q4k_kernel<XT, kLargeT, 0, false>(), QF_Q4K_THREADS, QF_Q4K_WAVES, v,
+                             q4k_kernel<XT, kLargeT, 0, false>(), q4k_threads<XT>(), QF_Q4K_WAVES, v,
                              1024, nullptr, nullptr, nullptr, 0, s);
     return launch_chunks(q4k_kernel<XT, kSmallT, 1, false>(), q4k_kernel<XT, kLargeT, 1, false>(),
-                         QF_Q4K_THREADS, QF_Q4K_WAVES, v, 1024, nullptr, nullptr, nullptr, 0, s);
+                         q4k_threads<XT>(), QF_Q4K_WAVES, v, 1024, nullptr, nullptr, nullptr, 0, s);
 }
 
 qf_status launch_format(qf_format f, int mode, int x_type, const std::vector<DevTensor>& v,

@@ -62,6 +62,9 @@
 #ifndef QF_Q4K_THREADS
 #define QF_Q4K_THREADS 512
 #endif
+#ifndef QF_Q4K_F32_THREADS
+#define QF_Q4K_F32_THREADS 128  // the same for FP32 input (its lanes read their sub-blocks directly)
+#endif
 #ifndef QF_Q4K_WAVES
 #define QF_Q4K_WAVES 1
 #endif
@@ -186,6 +189,25 @@ __device__ __forceinline__ float2 fma2_rn(float2 a, float2 b, float2 c) {
         "mov.b64 rc, {%6, %7};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
         : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
     return d;
+}
+// Asynchronous 8-byte copy global -> shared; src_bytes = 0 writes zeros and
+// reads nothing.  A thread's copies complete in commit-group order; cp_async_wait<N>
+// blocks in hardware until at most N of the thread's groups are pending.
+__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dst), "l"(src),
+                 "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr) : "memory");
+    return v;
+}
+// L2 prefetch of the line holding p; nothing waits for it
+__device__ __forceinline__ void prefetch_line_l2(const void* p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }

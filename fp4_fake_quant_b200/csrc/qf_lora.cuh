@@ -128,25 +128,6 @@ __device__ __forceinline__ uint32_t bf16x2_max_bits(uint32_t m) {
     return max(m & 0xFFFFu, m >> 16) << 16;
 }
 
-// L2 prefetch of the line holding p; nothing waits for it
-__device__ __forceinline__ void prefetch_line_l2(const void* p) {
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
-}
-
-// 8-byte asynchronous copy global -> shared; src_bytes = 0 writes zeros and reads nothing
-__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src, uint32_t src_bytes) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dst), "l"(src),
-                 "r"(src_bytes) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-// blocks (in hardware) until at most N of this thread's copy groups are pending
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-__device__ __forceinline__ uint2 lds64(uint32_t addr) {
-    uint2 v;
-    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr) : "memory");
-    return v;
-}
 
 template <bool B>
 struct FullTile { static constexpr bool value = B; };
