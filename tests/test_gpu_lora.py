@@ -23,7 +23,12 @@ def _case(rows, cols, rank, seed):
     return w, b, a
 
 
-SHAPES = [(37, 1040, 3), (64, 2048, 8), (33, 768, 16), (40, 4096, 32), (1, 32, 1)]
+# Whole 64-row tiles take a guard-free path and ragged ones the guarded path; the merge
+# and amax modes bring W through a 4-step ring at rank <= 16 and a 3-step ring at rank
+# 32.  (130, 1040, 16), (200, 1536, 12) and (128, 2048, 32) mix whole tiles, a ragged
+# row tail and a partial 1024-column group in one tensor.
+SHAPES = [(37, 1040, 3), (64, 2048, 8), (33, 768, 16), (40, 4096, 32), (1, 32, 1),
+          (130, 1040, 16), (200, 1536, 12), (128, 2048, 32)]
 
 
 @pytest.mark.parametrize("rows,cols,rank", SHAPES)
