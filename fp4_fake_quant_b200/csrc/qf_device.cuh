@@ -708,8 +708,10 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
 // and the rounding to an integer); the products scale*q and r*r, which are added
 // to, stay scalar.  The error is accumulated as (dq - x)^2, whose square equals
 // that of x - dq bit for bit (round-to-nearest is symmetric, so dq - x is exactly
-// -(x - dq)).
-template <typename XT>
+// -(x - dq)).  x + min_j >= +0 always (min_j >= -min x), so with a finite reciprocal
+// the scaled value is >= +0 and only the upper clamp can act: LOWER = false drops the
+// lower one.  LOWER = true keeps it for a reciprocal that overflowed (0 * inf).
+template <typename XT, bool LOWER>
 __device__ __forceinline__ float2 q4k_sub_err2(const Elems<XT, 32>& x, float2 scale, float min_j) {
     const float2 inv = make_float2(__frcp_rn(scale.x), __frcp_rn(scale.y));
     const float2 rnd = make_float2(kRound, kRound), nrnd = make_float2(-kRound, -kRound);
@@ -719,7 +721,8 @@ __device__ __forceinline__ float2 q4k_sub_err2(const Elems<XT, 32>& x, float2 sc
         const float xk = x.get(k);
         const float xm = __fadd_rn(xk, min_j);
         const float2 t = mul2_rn(make_float2(xm, xm), inv);
-        const float2 c = make_float2(fminf(fmaxf(t.x, 0.0f), 15.0f), fminf(fmaxf(t.y, 0.0f), 15.0f));
+        const float2 c = LOWER ? make_float2(fminf(fmaxf(t.x, 0.0f), 15.0f), fminf(fmaxf(t.y, 0.0f), 15.0f))
+                               : make_float2(fminf(t.x, 15.0f), fminf(t.y, 15.0f));
         const float2 q = add2_rn(add2_rn(c, rnd), nrnd);
         const float2 dq = make_float2(__fsub_rn(__fmul_rn(scale.x, q.x), min_j),
                                       __fsub_rn(__fmul_rn(scale.y, q.y), min_j));
@@ -729,18 +732,15 @@ __device__ __forceinline__ float2 q4k_sub_err2(const Elems<XT, 32>& x, float2 sc
     }
     return err;
 }
-
 // MSE-searched sub-block scale: with the offset fixed, try scale = (hi + min_j) / n
 // for n = 15 (the min/max fit) and then 14, 14.5, 15.5, 16, 16.5, 17, 17.5, 18; keep
 // the least squared error (a later trial must be strictly smaller).  The errors are
 // computed two trials at a time and then compared in trial order.
-template <typename XT>
-__device__ __forceinline__ float q4k_search_scale(const Elems<XT, 32>& x, float hi, float min_j) {
-    const float range = __fadd_rn(hi, min_j);
-    float best = __fdiv_rn(range, 15.0f);
-    if (best == 0.0f) return best;
+template <typename XT, bool LOWER>
+__device__ __forceinline__ float q4k_search_scale_t(const Elems<XT, 32>& x, float range,
+                                                    float best, float s18, float min_j) {
     const float s14 = __fdiv_rn(range, 14.0f);
-    const float2 e0 = q4k_sub_err2(x, make_float2(best, s14), min_j);
+    const float2 e0 = q4k_sub_err2<XT, LOWER>(x, make_float2(best, s14), min_j);
     float best_err = e0.x;
     if (e0.y < best_err) {
         best_err = e0.y;
@@ -752,8 +752,8 @@ __device__ __forceinline__ float q4k_search_scale(const Elems<XT, 32>& x, float 
     for (int p = 0; p < 4; ++p) {
         const float na = p == 0 ? 14.5f : p == 1 ? 16.0f : p == 2 ? 17.0f : 18.0f;
         const float nb = p == 0 ? 15.5f : p == 1 ? 16.5f : p == 2 ? 17.5f : 18.0f;
-        const float2 sc = make_float2(__fdiv_rn(range, na), __fdiv_rn(range, nb));
-        const float2 err = q4k_sub_err2(x, sc, min_j);
+        const float2 sc = make_float2(p == 3 ? s18 : __fdiv_rn(range, na), __fdiv_rn(range, nb));
+        const float2 err = q4k_sub_err2<XT, LOWER>(x, sc, min_j);
         if (err.x < best_err) {
             best_err = err.x;
             best = sc.x;
@@ -764,6 +764,17 @@ __device__ __forceinline__ float q4k_search_scale(const Elems<XT, 32>& x, float 
         }
     }
     return best;
+}
+template <typename XT>
+__device__ __forceinline__ float q4k_search_scale(const Elems<XT, 32>& x, float hi, float min_j) {
+    const float range = __fadd_rn(hi, min_j);
+    const float best = __fdiv_rn(range, 15.0f);
+    if (best == 0.0f) return best;
+    // range / 18 is the smallest trial scale: when its reciprocal is finite, so are all
+    const float s18 = __fdiv_rn(range, 18.0f);
+    if (__frcp_rn(s18) <= 3.402823466e38f)
+        return q4k_search_scale_t<XT, false>(x, range, best, s18, min_j);
+    return q4k_search_scale_t<XT, true>(x, range, best, s18, min_j);
 }
 
 // Per-lane fit of one sub-block; returns the super-block's FP16 d / dmin bits, this
