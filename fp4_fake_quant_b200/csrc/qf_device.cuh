@@ -376,7 +376,7 @@ __device__ __forceinline__ void fp4_lane(const Elems<XT, 8>& x, float s_t, float
         const uint32_t c = E > 2u ? E - 2u : 0u;
         o.scale = c;
         inv = __uint_as_float((254u - c) << 23);                          // 2^-e
-        S = c ? __uint_as_float(c << 23) : __uint_as_float(0x00200000u);  // 2^e
+        S = c ? __uint_as_float(c << 23) : __uint_as_float(0x00400000u);  // 2^e (2^-127: subnormal)
     }
 #pragma unroll
     for (int k = 0; k < 8; ++k) o.q[k] = __fmul_rn(x.get(k), inv);

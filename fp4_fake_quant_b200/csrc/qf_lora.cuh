@@ -321,7 +321,7 @@ __global__ void __launch_bounds__(kLoraThreads) k_lora(const __grid_constant__ L
                         const uint32_t E = m[h] >> 23;
                         sbyte[h] = E > 2u ? E - 2u : 0u;
                         inv[h] = __uint_as_float((254u - sbyte[h]) << 23);
-                        S[h] = sbyte[h] ? __uint_as_float(sbyte[h] << 23) : __uint_as_float(0x00200000u);
+                        S[h] = sbyte[h] ? __uint_as_float(sbyte[h] << 23) : __uint_as_float(0x00400000u);
                     }
                 }
 #pragma unroll

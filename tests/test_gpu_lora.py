@@ -82,6 +82,35 @@ def test_lora_fakequant_equals_merge_then_quantize(fmt, rows, cols, rank):
     assert torch.equal(y2, yo) and torch.equal(c2, co) and torch.equal(s2, so)
 
 
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4"])
+def test_lora_fakequant_near_min_normal(fmt):
+    """Merged weights just above the smallest normal (BF16 bit patterns 0x0080..0x00BF):
+    an MXFP4 block there takes scale byte 0 (2^-127) with nonzero codes."""
+    g = torch.Generator().manual_seed(21)
+    bits16 = torch.randint(0x0080, 0x00C0, (4, 256), generator=g, dtype=torch.int32)
+    bits16 = torch.where(torch.rand(4, 256, generator=g) < 0.5, bits16, bits16 | 0x8000)
+    w = bits16.to(torch.int16).view(torch.bfloat16).contiguous()
+    b = torch.zeros(4, 2, dtype=torch.bfloat16)
+    a = torch.zeros(2, 256, dtype=torch.bfloat16)
+    merged = oracle.lora_merge(w, b, a, 1.0)
+    if fmt == "nvfp4":
+        y, c, s, _ = oracle.nvfp4(merged, oracle.amax(merged))
+    else:
+        y, c, s = oracle.mxfp4(merged)
+    wd = w.to(DEV)
+    yo, co, so = qf.alloc_outputs(fmt, wd)
+    amax = torch.empty(1, device=DEV)
+    adapters = [(b.to(DEV), a.to(DEV), 1.0)]
+    if fmt == "nvfp4":
+        qf.qf_amax_fakequant_lora([wd], adapters, [yo], [co], [so], [0], amax)
+    else:
+        qf.qf_fakequant_lora(fmt, [wd], adapters, [yo], [co], [so])
+    torch.cuda.synchronize()
+    assert_same(f"lora {fmt} near-min y", bits(yo), y)
+    assert_same(f"lora {fmt} near-min codes", u8(co), c)
+    assert_same(f"lora {fmt} near-min scales", u8(so), s)
+
+
 def test_lora_grouped_experts_with_tied_groups():
     """Several adapted tensors in one launch (gate/up tied, down its own group)."""
     ts, ads, groups, merged = [], [], [], []

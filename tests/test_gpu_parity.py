@@ -159,13 +159,24 @@ def _edge_tensors():
     out.append(("ragged", ragged))
     pos = workloads.normal_with_outliers(5, 256, 0.02, 0.0, 1.0, 9, 0).abs() + 0.001
     out.append(("positive", pos.to(torch.bfloat16)))
+    # values just above the smallest normal (BF16 bit patterns 0x0080..0x00BF, mixed signs):
+    # a sub-block's range is below 18 * 2^-128, so its trial scales' reciprocals overflow
+    # (the MSE search's 0 * inf case); row 0 holds such a sub-block inside a normal
+    # super-block
+    g = torch.Generator().manual_seed(11)
+    lo = torch.randint(0x0080, 0x00C0, (2, 256), generator=g, dtype=torch.int32)
+    lo = torch.where(torch.rand(2, 256, generator=g) < 0.5, lo, lo | 0x8000).to(torch.int16)
+    mixed = workloads.normal_with_outliers(2, 256, 0.02, 0.0, 1.0, 12, 0)
+    mixed.view(torch.int16)[0, 32:64] = lo[0, 32:64]
+    out.append(("near_min_normal_in_normal", mixed))
+    out.append(("near_min_normal", lo.view(torch.bfloat16).contiguous()))
     return out
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4", "q4k"])
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4", "q4k", "q4k_mse"])
 def test_edge_cases_each_alone(fmt):
     for name, x in _edge_tensors():
-        if fmt == "q4k" and name == "huge":
+        if fmt in ("q4k", "q4k_mse") and name == "huge":
             continue        # beyond what Q4_K's FP16 super-block scale can hold
         res = run_fakequant(fmt, [x])
         am = oracle.tied_amax([x], [0], 1) if fmt == "nvfp4" else None
