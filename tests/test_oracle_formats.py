@@ -379,6 +379,31 @@ def test_nvfp4_monotone_within_block():
 
 
 # ----------------------------------------------------------------------------- degenerate cases
+def test_mxfp4_blocks_below_2_pow_minus_124_take_byte_0():
+    """A block whose max is below 2^-124 has floor(log2 amax) - 2 < -127, so its E8M0 byte
+    clamps to 0 (e = -127).  Its codes are the nearest E2M1 values of x * 2^127, and y is
+    code * 2^-127 exactly: float64 arithmetic here, nonzero codes included."""
+    rng = np.random.default_rng(31)
+    h = rng.integers(0x0080, 0x00C0, (4, 256)).astype(np.uint16)      # 2^-126 .. 1.5 * 2^-126
+    h |= (rng.random((4, 256)) < 0.5).astype(np.uint16) << 15
+    h[1, 32:64] = rng.integers(0x0001, 0x0080, 32).astype(np.uint16)  # BF16 subnormals
+    y, c, s = oracle.mxfp4(h)
+    assert np.all(s == 0)
+    xf = f32_of(h).astype(np.float64).reshape(-1)
+    a = np.abs(xf * 2.0 ** 127)
+    dist = np.abs(a[:, None] - E2M1[None, :])
+    cand = dist == dist.min(axis=1, keepdims=True)
+    even = cand & (np.arange(8)[None, :] % 2 == 0)
+    idx = np.where(even.any(axis=1), even.argmax(axis=1), cand.argmax(axis=1))
+    got = unpack_nibbles(c)
+    assert np.array_equal(got & 7, idx)
+    assert np.count_nonzero(got & 7) > 100
+    want = bits_of((e2m1_val(got) * 2.0 ** -127).astype(np.float32))
+    # a value that rounds to code 0 keeps its sign: -0 for negative inputs
+    want = np.where((got & 7) == 0, (h.reshape(-1) & 0x8000), want).astype(np.uint16)
+    assert np.array_equal(y, want)
+
+
 def test_degenerate_inputs():
     z = np.zeros((2, 64), np.uint16)
     z[0, 3] = 0x8000                                            # a negative zero
