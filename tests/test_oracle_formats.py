@@ -424,6 +424,24 @@ def test_degenerate_inputs():
     assert np.all(s == 0) and not np.any(np.isnan(f32_of(y)))
 
 
+def test_nvfp4_block_whose_scale_underflows_encodes_signed_zeros():
+    """A block far below the tie-group max gets E4M3 scale 0 (amax_b / (6 s_t) rounds to
+    0), so S = 0 and inv = 0: every element encodes as a zero of its own sign (code 0 or
+    8) and dequantizes to that zero, whatever its magnitude."""
+    x = np.zeros((1, 64), np.float32)
+    x[0, 0] = 1.0                                   # the group max: s_t = 1 / 2688
+    rng = np.random.default_rng(41)
+    x[0, 16:] = rng.uniform(1e-9, 2e-9, 48) * np.where(rng.random(48) < 0.5, -1.0, 1.0)
+    h = bits_of(torch.from_numpy(x).to(torch.bfloat16).to(torch.float32).numpy())
+    y, c, s, st = oracle.nvfp4(h, 1.0)
+    assert st == np.float32(1.0) / np.float32(2688.0)
+    assert s[0] != 0 and np.all(s[1:] == 0)
+    got = unpack_nibbles(c)[16:]
+    sign = (h[0, 16:] >> 15).astype(np.uint8)
+    assert np.all(got == 8 * sign)                  # +0 for positive inputs, -0 for negative
+    assert np.array_equal(y.reshape(-1)[16:], (h[0, 16:] & 0x8000).astype(np.uint16))
+
+
 def test_nvfp4_scale_reciprocal_overflow_keeps_zero_signs():
     """A block scale S below 2^-128 has 1/S = inf; zeros stay zeros of their sign."""
     x = np.zeros((1, 16), np.uint16)
