@@ -405,6 +405,19 @@ def test_full_q4k_mse_sampled_rows():
                      sample_rows(x.shape[0], 24, 500 + i), label=f"q4k mse[{i}]")
 
 
+def test_q4k_clipped_ste_at_both_ends_of_the_code_range():
+    """Elements that scale to exactly 0 and exactly 15 keep their gradient on the device
+    too (the super-block of workloads.q4k_ste_ends)."""
+    x = workloads.q4k_ste_ends()
+    g = workloads.normal_with_outliers(1, 256, 1e-3, 0.0, 1.0, 52, 0)
+    want = oracle.ste_backward(g, 1, "q4k", x)
+    assert want.reshape(-1)[32] != 0 and want.reshape(-1)[64] != 0
+    out = torch.empty(1, 256, dtype=torch.bfloat16, device=DEV)
+    qf.qf_ste_backward(g.to(DEV), out, mode=1, fmt="q4k", x=x.to(DEV))
+    torch.cuda.synchronize()
+    assert_same("q4k clipped STE ends", bits(out), want)
+
+
 @pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4", "q4k"])
 def test_clipped_ste_in_place(fmt):
     """Clipped STE with grad_x == grad_y gives the out-of-place result (and the oracle's)."""

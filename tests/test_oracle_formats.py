@@ -496,6 +496,25 @@ def test_ste_clipped_mask_is_saturation(fmt):
         assert (~keep).sum() > 0                               # saturation does occur
 
 
+def test_q4k_clipped_ste_keeps_both_ends_of_the_code_range():
+    """The Q4_K clipped STE keeps the gradient where 0 <= (x + mm) * inv <= 15, ends
+    included.  The super-block of workloads.q4k_ste_ends hits both ends exactly (its
+    construction is checked here: d = 2^-8, dmin = 65 * 2^-20, sc[1] = 32, m[2] = 1), and
+    its element at -2^-8 lies below its quantized offset and is clipped."""
+    xb = workloads.q4k_ste_ends()
+    h = workloads.bf16_bits(xb).reshape(1, 256)
+    d, dm, sc, m, q = oracle.q4k_fit_one(h)
+    f16 = np.array([d, dm], np.uint16).view(np.float16).astype(np.float64)
+    assert f16[0] == 2.0 ** -8 and f16[1] == 65 * 2.0 ** -20
+    assert sc[1] == 32 and m[2] == 1 and m[1] == 0 and q[32] == 15 and q[64] == 0
+    g = torch.ones(1, 256, dtype=torch.bfloat16)
+    gx = oracle.ste_backward(g, 1, "q4k", xb).reshape(-1)
+    one = workloads.bf16_bits(g).reshape(-1)[0]
+    assert gx[32] == one                             # (x + mm) * inv == 15 exactly
+    assert gx[64] == one                             # (x + mm) * inv == 0 exactly
+    assert gx[1] == 0                                # (x + mm) * inv < 0: clipped
+
+
 def test_q4k_negative_values_rounding_to_code_zero_dequantize_to_positive_zero():
     """Q4_K codes are unsigned integers: a sub-block whose stored min is 0 but that
     holds small negative values dequantizes them from the integer code 0 to +0."""

@@ -142,6 +142,24 @@ def nvfp4_activation(rows_scale: float = 1.0, seed: int = 5):
     return {"tensors": [a], "names": ["act"], "groups": [0], "n_groups": 1}
 
 
+def q4k_ste_ends(seed: int = 51) -> torch.Tensor:
+    """One BF16 Q4_K super-block [1, 256] whose values put elements exactly on both ends
+    of the clipped STE's range [0, 15]: sub-block 0 spans -2^-8 .. 944 * 2^-8 (so its
+    scale is 63 * 2^-8 and d = 2^-8), sub-block 1 peaks at 1.875 = 15 * 2^-3 (sc = 32,
+    scale 2^-3), and sub-block 2's minimum is -65 * 2^-20 (= dmin, m = 1).  Element 32
+    scales to 15 exactly, element 64 to 0 exactly, element 1 below 0."""
+    rng = _rng(seed, 0)
+    x = np.zeros(256, np.float64)
+    x[0:32] = rng.uniform(0, 3.6, 32)
+    x[0], x[1] = 944 * 2.0 ** -8, -2.0 ** -8
+    x[32:64] = rng.uniform(0, 1.8, 32)
+    x[32] = 1.875
+    x[64:96] = rng.uniform(0, 0.5, 32)
+    x[64] = -65 * 2.0 ** -20
+    x[96:] = rng.uniform(0, 1.0, 160)
+    return to_bf16(x.reshape(1, 256))
+
+
 def bf16_bits(t: torch.Tensor) -> np.ndarray:
     """View a CPU BF16 tensor as a numpy uint16 array of bit patterns."""
     return t.contiguous().view(torch.int16).numpy().view(np.uint16)
