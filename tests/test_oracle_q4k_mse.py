@@ -53,6 +53,21 @@ def test_on_grid_blocks_keep_the_min_max_fit():
     assert s == np.float32(np.float32(v.max() + 0.5) / np.float32(15.0))
 
 
+def test_equal_errors_keep_the_earlier_trial():
+    """Trials are taken in the order 15, 14, 14.5, ... and a later one must be strictly
+    better.  A two-valued sub-block {0, 210 * 2^-10} (210 = 14 * 15) is exact on both
+    the n = 15 grid (scale 14 * 2^-10) and the n = 14 grid (scale 15 * 2^-10): both
+    errors are 0, every other trial's is positive, and the search keeps n = 15."""
+    hi = np.float32(210 * 2.0 ** -10)
+    rng = np.random.default_rng(61)
+    v = np.where(rng.random(32) < 0.5, np.float32(0), hi).astype(np.float32)
+    v[0], v[1] = 0, hi
+    cands = [np.float32(hi / np.float32(n)) for n in GRID]
+    errs = [err64(v, float(c), 0.0) for c in cands]
+    assert errs[0] == 0 and errs[1] == 0 and min(errs[2:]) > 0
+    assert oracle.q4k_search_scale(v, float(hi), 0.0) == cands[0]
+
+
 def test_mse_fit_decoder_and_total_error():
     wl = workloads.q4k_weights(rows_scale=1 / 256)
     tot_mm = tot_mse = 0.0
