@@ -154,6 +154,21 @@ def test_valid_call_without_a_gpu_reports_cuda_error(qf):
     assert qf.lib.qf_last_error().decode()
 
 
+def test_adjacent_buffers_are_disjoint(qf):
+    """Buffers that touch but do not overlap pass validation: x, y, codes and scales
+    laid out back to back (4 x 64 MXFP4: 512 B of x, 512 B of y, 128 B of codes, 8 B of
+    scales).  Without a GPU the call then fails at its first CUDA step (QF_ERR_CUDA),
+    which shows that the argument checks accepted it."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present (the pointers are fake)")
+    arr = _tensor(qf, x=0x10000, y=0x10200, codes=0x10400, scales=0x10480)
+    assert _fq(qf, 1, arr) == 5
+    assert "overlap" not in qf.lib.qf_last_error().decode()
+    arr = _tensor(qf, x=0x10000, y=0x101F0)        # y starts 16 bytes before x ends
+    assert _fq(qf, 1, arr) == 1
+
+
 def test_amax_and_ste_validation(qf):
     INV, SHAPE, ALIGN, UNSUP = 1, 2, 3, 4
     lib = qf.lib
