@@ -24,6 +24,16 @@ def reduce_group_amax(group_amax: torch.Tensor, group=None) -> torch.Tensor:
     return group_amax
 
 
+def fold_tracked(group_amax: torch.Tensor, tracked: Optional[torch.Tensor]) -> torch.Tensor:
+    """In place: tracked <- max(tracked, group_amax), then group_amax <- tracked, the
+    value the step quantizes with (the tracked amax is a running max kept across
+    steps).  With tracked None, group_amax is left as it is."""
+    if tracked is not None:
+        torch.maximum(tracked, group_amax, out=tracked)
+        group_amax.copy_(tracked)
+    return group_amax
+
+
 def amax_tied_sharded(xs: Sequence[torch.Tensor], groups: Sequence[int],
                       group_amax: torch.Tensor, tracked: Optional[torch.Tensor] = None,
                       group=None, stream=None) -> torch.Tensor:
@@ -33,7 +43,4 @@ def amax_tied_sharded(xs: Sequence[torch.Tensor], groups: Sequence[int],
     from .binding import qf_amax_tied
     qf_amax_tied(xs, groups, group_amax, None, stream)
     reduce_group_amax(group_amax, group)
-    if tracked is not None:
-        torch.maximum(tracked, group_amax, out=tracked)
-        group_amax.copy_(tracked)
-    return group_amax
+    return fold_tracked(group_amax, tracked)

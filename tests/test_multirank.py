@@ -27,7 +27,7 @@ def _worker(rank, world, port, out):
     try:
         import oracle
         import workloads
-        from fp4_fake_quant_b200.distributed import reduce_group_amax
+        from fp4_fake_quant_b200.distributed import fold_tracked, reduce_group_amax
         # each rank holds a shard (half the rows) of every tensor of two tie groups
         wl = workloads.nvfp4_tied(rows_scale=1 / 64, with_grads=False)
         shards = [t[rank * (t.shape[0] // world):(rank + 1) * (t.shape[0] // world)]
@@ -37,6 +37,12 @@ def _worker(rank, world, port, out):
         full = oracle.tied_amax([t[: (t.shape[0] // world) * world] for t in wl["tensors"]],
                                 wl["groups"], 2)
         ok_amax = bool(np.array_equal(local.numpy().view(np.uint32), full.view(np.uint32)))
+        # a tracked amax above the step's amax in group 0 and below it in group 1: both
+        # ranks end with tracked = max(tracked, global amax) and quantize with it
+        tracked = torch.tensor([float(full[0]) * 2, float(full[1]) / 2], dtype=torch.float32)
+        want = np.maximum(tracked.numpy(), full)
+        fold_tracked(local, tracked)
+        ok_amax &= bool(np.array_equal(tracked.numpy(), want) and np.array_equal(local.numpy(), want))
         # the benchmark's aggregation: max over ranks of each device time, and the
         # whole-job value = world x bytes per step / slowest step
         import bench
