@@ -34,9 +34,11 @@
  *     is asynchronous on that stream.
  *   - Arguments are validated on the host before anything is launched; an
  *     invalid call returns an error status and launches nothing.  A CUDA launch
- *     failure returns QF_ERR_CUDA.  Kernels never trap.  The one wait in the
- *     library is the grid barrier of qf_amax_fakequant's single-launch path,
- *     which is bounded (see there).
+ *     failure returns QF_ERR_CUDA.  Kernels never trap.  The one wait on other
+ *     threads in the library is the grid barrier of qf_amax_fakequant's
+ *     single-launch path, which is bounded (see there).  The LoRA kernels also
+ *     wait, in hardware (cp.async.wait_group), for their own asynchronous copies
+ *     of W into shared memory.
  *     qf_last_error() gives a one-line description of the last failure on the
  *     calling thread.
  *   - Outputs must not overlap the inputs or one another, except that
