@@ -433,7 +433,53 @@ def run_ours(args, rank, world, local_rank):
         result["export"] = export_timing(qf, dev)
     if rank == 0 and world == 1 and not args.no_cpu:
         result["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_rows_frac)
+    if "per_format" in result:
+        # last key of the line, so that a reader that keeps only its tail sees every workload
+        result["per_format_summary"] = format_summary(args.workload, result, peak)
     return result
+
+
+def _r(v, nd=3):
+    """Round to `nd` significant digits (None stays None)."""
+    if v is None:
+        return None
+    return float(f"{v:.{nd}g}")
+
+
+def format_summary(headline: str, result: dict, peak: float) -> dict:
+    """Compact per-workload figures: [fused_us, fused_frac, step_us, step_frac], where
+    fused is the fake-quant+pack launch alone and step the workload's whole step through
+    its one-call entry point (NVFP4: amax + fused pass; LoRA: merge + amax + fused
+    pass); fractions are of the measured HBM copy peak, at the algorithmic bytes."""
+    out = {"cols": ["fused_us", "fused_frac", "step_us", "step_frac"], "peak_GB/s": peak}
+    r = result["roofline"]
+    step_frac = result["value"] / result["n_gpus"] / peak
+    out[headline] = [_r(r["launch_us"]), _r(r["hbm"]["frac"] if r["bound"] == "alu" else r["frac"]),
+                     _r(result["ms_per_step"] * 1e3), _r(step_frac)]
+    moe, ste = {}, None
+    for name, d in result["per_format"].items():
+        if "one_call_step_us" in d:
+            su, sg = d["one_call_step_us"], d["one_call_step_GB/s"]
+        elif "step_us" in d:
+            su, sg = d["step_us"], d["step_GB/s"]
+        else:
+            su, sg = d["fused_us"], d["fused_GB/s"]
+        out[name] = [_r(d["fused_us"]), _r(d["fused_frac_of_hbm_peak"]), _r(su), _r(sg / peak)]
+        if "alu_bound" in d:
+            out[name + "_alu_frac"] = _r(d["alu_bound"]["frac"])
+        if "one_expert_at_a_time_us" in d:
+            moe[d["format"]] = [_r(d["fused_us"]), _r(d["one_expert_at_a_time_graph_us"]),
+                                _r(d["one_expert_at_a_time_us"])]
+        if "ste_identity_us" in d:
+            ste = [_r(d["ste_identity_us"]), _r(d["ste_identity_GB/s"] / peak),
+                   _r(d["ste_clipped_us"]), _r(d["ste_clipped_GB/s"] / peak)]
+    if moe:
+        out["moe_grouped_vs_per_expert_us"] = {"cols": ["grouped", "per_expert_graph",
+                                                        "per_expert_eager"], **moe}
+    if ste is not None:
+        out["ste_tied"] = {"cols": ["identity_us", "identity_frac", "clipped_us",
+                                    "clipped_frac"], "v": ste}
+    return out
 
 
 def graph_timed(fn, iters, flush):

@@ -65,10 +65,13 @@ def _load() -> ctypes.CDLL:
     lib.qf_amax_fakequant_workspace_bytes.restype = ctypes.c_size_t
     lib.qf_workspace_check.argtypes = [P, P]
     lib.qf_amax_fakequant_noalloc.argtypes = [T, I, P, I, P, P, P]
+    lib.qf_noalloc_check.argtypes = [P]
+    lib.qf_test_barrier_timeout.argtypes = [ctypes.c_uint]
+    lib.qf_test_barrier_timeout.restype = None
     for f in (lib.qf_amax_tied, lib.qf_fakequant, lib.qf_pack, lib.qf_ste_backward,
               lib.qf_lora_merge, lib.qf_amax_tied_lora, lib.qf_fakequant_lora,
               lib.qf_amax_fakequant, lib.qf_workspace_check, lib.qf_amax_fakequant_noalloc,
-              lib.qf_amax_fakequant_lora):
+              lib.qf_amax_fakequant_lora, lib.qf_noalloc_check):
         f.restype = I
     lib.qf_status_string.argtypes = [I]
     lib.qf_status_string.restype = ctypes.c_char_p
@@ -85,7 +88,8 @@ lib = _load()
 EXPORTS = ("qf_amax_tied", "qf_fakequant", "qf_pack", "qf_ste_backward", "qf_lora_merge",
            "qf_amax_tied_lora", "qf_fakequant_lora", "qf_amax_fakequant_lora",
            "qf_amax_fakequant", "qf_amax_fakequant_workspace_bytes", "qf_workspace_check",
-           "qf_amax_fakequant_noalloc", "qf_status_string", "qf_last_error", "qf_version")
+           "qf_amax_fakequant_noalloc", "qf_noalloc_check", "qf_test_barrier_timeout",
+           "qf_status_string", "qf_last_error", "qf_version")
 
 
 def _check(status: int) -> None:
@@ -268,8 +272,20 @@ def qf_amax_fakequant_noalloc(xs, ys=None, codes=None, scales=None, groups=None,
 
 
 def qf_workspace_check(workspace: torch.Tensor, stream=None) -> None:
-    """Synchronize and raise QfError(QF_ERR_TIMEOUT) if a grid barrier gave up."""
+    """Synchronize, clear the workspace's error flags, and raise QfError(QF_ERR_TIMEOUT)
+    if a grid barrier gave up."""
     _check(lib.qf_workspace_check(_ptr(workspace), _stream(stream)))
+
+
+def qf_noalloc_check(stream=None) -> None:
+    """qf_workspace_check for the static workspace of qf_amax_fakequant_noalloc."""
+    _check(lib.qf_noalloc_check(_stream(stream)))
+
+
+def qf_test_barrier_timeout(polls: int) -> None:
+    """Testing aid: with polls > 0 the single-launch grid barrier waits for one CTA
+    more than exist and gives up after `polls` polls; 0 restores normal operation."""
+    lib.qf_test_barrier_timeout(int(polls))
 
 
 def _lora(adapters):

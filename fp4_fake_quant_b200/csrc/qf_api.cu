@@ -7,6 +7,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -466,10 +467,13 @@ qf_status amax_launch(const std::vector<DevTensor>& v, int x_type, float* d_grou
 }
 
 // ------------------------------------------------------------------ one-shot NVFP4
-size_t oneshot_ws_bytes(int n_groups) {
-    const size_t b = sizeof(uint32_t) * ((size_t)qf::kOneshotHeaderWords + (size_t)n_groups);
-    return (b + 255) / 256 * 256;
+constexpr size_t oneshot_ws_bytes(int n_groups) {
+    return (sizeof(uint32_t) * ((size_t)qf::kOneshotHeaderWords + (size_t)n_groups) + 255) / 256 *
+           256;
 }
+
+// Polls of the forced barrier timeout (qf_test_barrier_timeout); 0 = normal operation.
+std::atomic<uint32_t> g_test_polls{0};
 
 // L2 size and cooperative-launch support of the current device, queried once per
 // host thread and device.
@@ -512,7 +516,8 @@ qf_status oneshot_launch(const std::vector<DevTensor>& v, float* am, float* trac
     // at most one CTA per resident slot: every CTA must be resident for the barrier,
     // which the cooperative launch guarantees (or refuses to launch)
     const int grid = grid_for(L, P.total_units);
-    void* args[] = {&P, &ws};
+    uint32_t test_polls = g_test_polls.load(std::memory_order_relaxed);
+    void* args[] = {&P, &ws, &test_polls};
     cudaError_t e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kernel), dim3(grid),
                                                 dim3(QF_ONESHOT_THREADS), args, 0, s);
     if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchCooperativeKernel");
@@ -521,10 +526,12 @@ qf_status oneshot_launch(const std::vector<DevTensor>& v, float* am, float* trac
 
 // ------------------------------------------------------------------ static scratch
 // The workspace of qf_amax_fakequant_noalloc: module-level device memory, one copy per
-// device, never allocated at run time.  Capacity: the header words plus one word per
-// tie group, for up to QF_NOALLOC_MAX_GROUPS groups.
-constexpr int kNoallocWords = qf::kOneshotHeaderWords + QF_NOALLOC_MAX_GROUPS;
-__device__ __align__(256) uint32_t g_noalloc_ws[kNoallocWords];
+// device, never allocated at run time.  Capacity: the workspace qf_amax_fakequant needs
+// for QF_NOALLOC_MAX_GROUPS tie groups (header words plus one word per group, rounded
+// up to 256 bytes), so every byte a call clears or uses lies inside the array.
+constexpr size_t kNoallocBytes = oneshot_ws_bytes(QF_NOALLOC_MAX_GROUPS);
+static_assert(kNoallocBytes % sizeof(uint32_t) == 0, "whole words");
+__device__ __align__(256) uint32_t g_noalloc_ws[kNoallocBytes / sizeof(uint32_t)];
 
 // Its address on the current device, looked up once per device (with that device
 // current, as cudaGetSymbolAddress requires) and kept.
@@ -816,27 +823,52 @@ qf_status qf_amax_fakequant_noalloc(const qf_tensor* t, int n, float* d_group_am
     void* ws = nullptr;
     qf_status st = noalloc_ws(&ws);
     if (st != QF_OK) return st;
-    // the part of the workspace this call uses must start at zero: clear it on the
-    // call's stream, whatever an earlier call (or a timed-out one) left there
+    // the counters and slots this call uses must start at zero: clear them on the call's
+    // stream, whatever an earlier call left there.  The error word (word 0) is kept: a
+    // timeout stays visible to qf_noalloc_check until that call clears it.
     const size_t bytes = oneshot_ws_bytes(n_groups);
-    cudaError_t e = cudaMemsetAsync(ws, 0, bytes, static_cast<cudaStream_t>(stream));
+    constexpr size_t kKeep = sizeof(uint32_t);              // the error word
+    cudaError_t e = cudaMemsetAsync(static_cast<char*>(ws) + kKeep, 0, bytes - kKeep,
+                                    static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
     return qf_amax_fakequant(t, n, d_group_amax, n_groups, d_tracked, d_group_scale_out, ws, bytes,
                              stream);
 }
 
+// Synchronizes `stream`, then reads the error word of a one-shot workspace and clears it.
+static qf_status check_and_clear(const void* d_workspace, void* stream) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    uint32_t* word = static_cast<uint32_t*>(const_cast<void*>(d_workspace)) + qf::kOneshotErrWord;
+    uint32_t err = 0;
+    e = cudaMemcpy(&err, word, sizeof err, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy");
+    if (err == 0) return QF_OK;
+    const uint32_t zero = 0;
+    e = cudaMemcpy(word, &zero, sizeof zero, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy");
+    if (err & qf::kOneshotErrTimeout)
+        return fail(QF_ERR_TIMEOUT, "a grid barrier gave up waiting; that call (and any later "
+                                    "call on this workspace before this check) wrote no outputs");
+    return fail(QF_ERR_CUDA, "unknown workspace error flags %#x", err);
+}
+
 qf_status qf_workspace_check(const void* d_workspace, void* stream) {
     g_err[0] = 0;
     if (d_workspace == nullptr) return fail(QF_ERR_INVALID_ARG, "workspace is NULL");
-    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
-    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
-    uint32_t err = 0;
-    e = cudaMemcpy(&err, static_cast<const uint32_t*>(d_workspace) + 2, sizeof err,
-                   cudaMemcpyDeviceToHost);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy");
-    if (err & qf::kOneshotErrTimeout)
-        return fail(QF_ERR_TIMEOUT, "a grid barrier gave up waiting; clear the workspace before reuse");
-    return QF_OK;
+    return check_and_clear(d_workspace, stream);
+}
+
+qf_status qf_noalloc_check(void* stream) {
+    g_err[0] = 0;
+    void* ws = nullptr;
+    qf_status st = noalloc_ws(&ws);
+    if (st != QF_OK) return st;
+    return check_and_clear(ws, stream);
+}
+
+void qf_test_barrier_timeout(unsigned int polls) {
+    g_test_polls.store(polls, std::memory_order_relaxed);
 }
 
 qf_status qf_fakequant(qf_format f, const qf_tensor* t, int n, const float* d_group_amax,
@@ -910,6 +942,6 @@ const char* qf_status_string(qf_status s) {
 
 const char* qf_last_error(void) { return g_err; }
 
-int qf_version(void) { return (1 << 16) | 6; }
+int qf_version(void) { return (1 << 16) | 7; }
 
 }  // extern "C"

@@ -11,14 +11,21 @@
 //            CTA-level combine);
 //   barrier  a grid-wide arrive counter; all CTAs are co-resident (cooperative launch),
 //            and the wait is bounded: after kOneshotSpinLimit polls the CTA sets the
-//            workspace's error word and returns without writing its outputs;
+//            workspace's error word and skips phase 2 (its outputs stay unwritten);
 //   phase 2  every CTA re-reads the same units -- now L2 hits -- and encodes them
 //            exactly as k_nv does.
-// The last CTA to finish resets the workspace (slots and counters) to zero, so a
-// zeroed workspace stays valid for the next call on the same stream.
+// Every CTA departs through a second counter, whether it passed the barrier or gave
+// up; the last one out resets the slots and both counters, so the workspace is zero
+// again after every call, a timed-out one included.  The error word is sticky: it
+// stays set until the host clears it (qf_workspace_check), and a call that finds it
+// set at entry does no work at all, so no later call can encode from a partial amax.
 //
-// Workspace layout (32-bit words): [0] arrive count, [1] depart count, [2] error
-// flags, [3] unused, [4 + g] group g's running max |x| as FP32 bits.
+// Every fold of the amax (slots, the tracked running value) takes the max of the FP32
+// bit patterns as unsigned integers, as k_amax does: for values >= +0 that is the
+// float max, and a NaN (sign bit clear) wins, on both paths of the call alike.
+//
+// Workspace layout (32-bit words): [0] error flags, [1] reserved (0), [2] arrive
+// count, [3] depart count, [4 + g] group g's running max |x| as FP32 bits.
 #pragma once
 
 #include "qf_device.cuh"
@@ -28,6 +35,7 @@ namespace qf {
 constexpr int kOneshotHeaderWords = 4;
 constexpr uint32_t kOneshotSpinLimit = 1u << 22;    // polls, ~256 ns apart: about a second
 constexpr uint32_t kOneshotErrTimeout = 1u;
+constexpr int kOneshotErrWord = 0, kOneshotArriveWord = 2, kOneshotDepartWord = 3;
 #ifndef QF_ONESHOT_THREADS
 #define QF_ONESHOT_THREADS 256
 #endif
@@ -53,18 +61,29 @@ __device__ __forceinline__ uint32_t ld_relaxed_gpu(const uint32_t* p) {
 // amax, max-accumulated in place; when given, s_t comes from the updated running
 // value (the activation reading), otherwise from this call's amax.
 // P.group_scale_out (nullable): s_t per group.
+// test_polls: 0 in normal use.  N > 0 makes the barrier wait for one CTA more than the
+// grid holds, polling at most N times, so that every CTA gives up: the timeout path
+// runs with every CTA present and no fault.
 template <typename XT, int U, int MAXT, int THREADS>
 __global__ void __launch_bounds__(THREADS, QF_ONESHOT_MINB)
-    k_nv_oneshot(const __grid_constant__ Table<MAXT> P, uint32_t* __restrict__ ws) {
+    k_nv_oneshot(const __grid_constant__ Table<MAXT> P, uint32_t* __restrict__ ws,
+                 uint32_t test_polls) {
     constexpr int kWarps = THREADS / 32;
     constexpr int kUnit = 512 * U;
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int64_t warp = int64_t(blockIdx.x) * kWarps + wid;
     const int64_t nwarps = int64_t(gridDim.x) * kWarps;
     uint32_t* slot = ws + kOneshotHeaderWords;
+    __shared__ int s_flag;
+
+    // a sticky error left by an earlier call: do nothing, so the caller's check sees it
+    if (threadIdx.x == 0) s_flag = ld_relaxed_gpu(ws + kOneshotErrWord) != 0u;
+    __syncthreads();
+    const bool skip = s_flag;
+    __syncthreads();
 
     // ---- phase 1: max |x| per tie group over this warp's units
-    int ti = warp < P.total_units ? locate_tensor(P, warp) : 0;
+    int ti = warp < P.total_units && !skip ? locate_tensor(P, warp) : 0;
     int g = -1;
     uint32_t run = 0;
     auto warp_max = [&]() {
@@ -73,7 +92,7 @@ __global__ void __launch_bounds__(THREADS, QF_ONESHOT_MINB)
         for (int o = 16; o > 0; o >>= 1) a = max(a, __shfl_xor_sync(kFull, a, o));
         return a;
     };
-    for (int64_t u = warp; u < P.total_units; u += nwarps) {
+    for (int64_t u = skip ? P.total_units : warp; u < P.total_units; u += nwarps) {
         ti = find_tensor(P, ti, u);
         const DevTensor& T = P.t[ti];
         if (T.group != g) {
@@ -89,7 +108,6 @@ __global__ void __launch_bounds__(THREADS, QF_ONESHOT_MINB)
     }
     __shared__ int wgrp[kWarps];
     __shared__ uint32_t wmax[kWarps];
-    __shared__ int s_flag;
     {
         const uint32_t a = warp_max();
         if (lane == 0) {
@@ -114,26 +132,31 @@ __global__ void __launch_bounds__(THREADS, QF_ONESHOT_MINB)
     // ---- grid barrier (bounded)
     if (threadIdx.x == 0) {
         __threadfence();                                    // this CTA's slot updates first
-        atomicAdd(ws + 0, 1u);
-        uint32_t polls = 0;
-        bool done = ld_acquire_gpu(ws + 0) >= gridDim.x;
-        while (!done && ++polls < kOneshotSpinLimit) {
-            __nanosleep(256);
-            done = ld_acquire_gpu(ws + 0) >= gridDim.x;
+        atomicAdd(ws + kOneshotArriveWord, 1u);
+        bool done = false;
+        if (!skip) {
+            const uint32_t target = gridDim.x + (test_polls ? 1u : 0u);
+            const uint32_t limit = test_polls ? test_polls : kOneshotSpinLimit;
+            uint32_t polls = 0;
+            done = ld_acquire_gpu(ws + kOneshotArriveWord) >= target;
+            while (!done && ++polls < limit) {
+                __nanosleep(256);
+                done = ld_acquire_gpu(ws + kOneshotArriveWord) >= target;
+            }
+            if (!done) atomicOr(ws + kOneshotErrWord, kOneshotErrTimeout);
         }
-        if (!done) atomicOr(ws + 2, kOneshotErrTimeout);
         s_flag = done;
     }
     __syncthreads();
-    if (!s_flag) return;                                    // outputs left unwritten
+    const bool go = s_flag;                                 // false: outputs left unwritten
 
     // ---- group statistics out (CTA 0)
     auto eff_amax = [&](int grp) {
-        float a = __uint_as_float(ld_relaxed_gpu(slot + grp));
-        if (P.tracked) a = fmaxf(a, P.tracked[grp]);
-        return a;
+        uint32_t a = ld_relaxed_gpu(slot + grp);
+        if (P.tracked) a = max(a, __float_as_uint(P.tracked[grp]));
+        return __uint_as_float(a);
     };
-    if (blockIdx.x == 0) {
+    if (go && blockIdx.x == 0) {
         for (int q = threadIdx.x; q < P.n_groups; q += THREADS) {
             const float cur = __uint_as_float(ld_relaxed_gpu(slot + q));
             const float e = eff_amax(q);
@@ -144,7 +167,7 @@ __global__ void __launch_bounds__(THREADS, QF_ONESHOT_MINB)
     }
 
     // ---- phase 2: encode the same units (their lines are in L2 now)
-    if (warp < P.total_units) {
+    if (go && warp < P.total_units) {
         ti = locate_tensor(P, warp);
         int cur_t = -1;
         float s_t = 0.0f, six_st = 0.0f;
@@ -163,18 +186,20 @@ __global__ void __launch_bounds__(THREADS, QF_ONESHOT_MINB)
         }
     }
 
-    // ---- depart; the last CTA out leaves the workspace zeroed for the next call
+    // ---- depart (every CTA, whether it passed the barrier or gave up); the last CTA
+    // out leaves the slots and counters zeroed for the next call
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
-        s_flag = atomicAdd(ws + 1, 1u) == gridDim.x - 1;
+        s_flag = atomicAdd(ws + kOneshotDepartWord, 1u) == gridDim.x - 1;
     }
     __syncthreads();
     if (s_flag) {
+        __threadfence();
         for (int q = threadIdx.x; q < P.n_groups; q += THREADS) slot[q] = 0u;
         if (threadIdx.x == 0) {
-            ws[0] = 0u;
-            ws[1] = 0u;
+            ws[kOneshotArriveWord] = 0u;
+            ws[kOneshotDepartWord] = 0u;
         }
     }
 }

@@ -137,7 +137,10 @@ typedef struct qf_tensor {
  *   d_tracked       NULL, or FP32[n_groups]: updated in place to
  *                     max(d_tracked[g], d_group_amax[g])  (the running amax a
  *                     training loop keeps for activations; pass it as the
- *                     d_group_amax of qf_fakequant to quantize with it).
+ *                     d_group_amax of qf_fakequant to quantize with it).  Its
+ *                     values must be >= +0 (start it at +0): the max is taken on
+ *                     the FP32 bit patterns as unsigned integers, which is the
+ *                     float max there (a NaN, outside the formats, propagates).
  *   Only x, rows, cols, group and x_type of each tensor are read; cols may be any
  *   value >= 0 here.  n == 0 only clears d_group_amax.
  * Errors: t == NULL with n > 0, n < 0, n_groups <= 0, d_group_amax == NULL,
@@ -214,10 +217,18 @@ qf_status qf_fakequant(qf_format f, const qf_tensor* t, int n, const float* d_gr
  *                      workspaces.
  *   workspace_bytes    its size.
  * The barrier wait is bounded (about a second of polling).  A CTA that gives up
- * sets an error flag in the workspace and writes none of its outputs.
- * qf_workspace_check then reports QF_ERR_TIMEOUT, and the workspace must be
- * zeroed again before reuse.  A cooperative launch guarantees that every CTA is
- * resident, so the wait completes unless a CTA faults.
+ * sets an error flag in the workspace and writes none of its outputs; every CTA
+ * still leaves the workspace's counters and slots zeroed.  The flag is sticky: until
+ * qf_workspace_check reads and clears it, every later call on that workspace does no
+ * work at all (its outputs are left as they were), so no call can encode from a
+ * partial amax.  Check the workspace after any call whose outputs matter.  A
+ * cooperative launch guarantees that every CTA is resident, so the wait completes
+ * unless a CTA faults.
+ * Amax folding: every max (the group amax, the running value) is taken on the FP32
+ *   bit patterns as unsigned integers, as qf_amax_tied does; that is the float max for
+ *   values >= +0, so the running amax must start at +0 (or any value >= +0).  A NaN in
+ *   x or in d_tracked is outside the formats (inputs are finite), but both paths of
+ *   this call give the same bytes for it: the NaN propagates into the amax.
  * Errors: as qf_fakequant; a workspace smaller than needed -> QF_ERR_INVALID_ARG,
  *   not 16-byte aligned -> QF_ERR_ALIGN.
  */
@@ -235,8 +246,10 @@ size_t qf_amax_fakequant_workspace_bytes(int n_groups);
  * counterpart: this is an interface convenience, not part of the method.
  *
  * The results are bit for bit those of qf_amax_fakequant with a caller workspace.
- * The call first clears the part of the static workspace it uses (one
- * cudaMemsetAsync on `stream`), then runs qf_amax_fakequant on it.
+ * The call first clears the counters and slots of the static workspace (one
+ * cudaMemsetAsync on `stream`), then runs qf_amax_fakequant on it.  Its error word is
+ * not cleared: a barrier timeout stays recorded, and every later call does no work,
+ * until qf_noalloc_check reads and clears it.
  * Limit: n_groups <= 4092; larger counts return QF_ERR_INVALID_ARG (use
  * qf_amax_fakequant with a workspace of your own).
  * The static workspace is shared by every call on the device.  Two calls that may
@@ -250,8 +263,22 @@ qf_status qf_amax_fakequant_noalloc(const qf_tensor* t, int n, float* d_group_am
                                     void* stream);
 
 /* Synchronizes `stream`, then reads the error flags of a qf_amax_fakequant
- * workspace: QF_OK, or QF_ERR_TIMEOUT if a grid barrier gave up. */
+ * workspace and clears them: QF_OK, or QF_ERR_TIMEOUT if a grid barrier gave up
+ * (that call, and every later call on the workspace before this check, wrote no
+ * outputs).  The workspace is ready for reuse either way. */
 qf_status qf_workspace_check(const void* d_workspace, void* stream);
+
+/* qf_workspace_check for the static workspace of qf_amax_fakequant_noalloc on the
+ * current device. */
+qf_status qf_noalloc_check(void* stream);
+
+/* Testing aid for the timeout path of the single-launch grid barrier.  With polls > 0,
+ * every later qf_amax_fakequant* call of this process that takes the single-launch
+ * path waits for one CTA more than its grid holds, polls at most `polls` times
+ * (about 256 ns apart), and gives up: the timeout is reported as above, with every
+ * CTA present and nothing faulted.  polls == 0 (the default) restores normal
+ * operation.  Not for production use. */
+void qf_test_barrier_timeout(unsigned int polls);
 
 /*
  * qf_pack -- the engine-layout export and weight sync (project page, Method,
@@ -367,7 +394,8 @@ const char* qf_last_error(void);
 /* ABI version: (major << 16) | minor.  1.1 added qf_tensor.x_type (formerly a
  * reserved field that had to be 0, which still means BF16); 1.2 the LoRA calls;
  * 1.3 QF_Q4K_MSE; 1.4 qf_amax_fakequant, its workspace calls and QF_ERR_TIMEOUT;
- * 1.5 qf_amax_fakequant_noalloc; 1.6 qf_amax_fakequant_lora. */
+ * 1.5 qf_amax_fakequant_noalloc; 1.6 qf_amax_fakequant_lora; 1.7 sticky workspace
+ * error flags, qf_noalloc_check and qf_test_barrier_timeout. */
 int qf_version(void);
 
 #ifdef __cplusplus

@@ -2,6 +2,8 @@
 and compare its bytes with the oracle's.  Bit-exact comparisons only."""
 from __future__ import annotations
 
+import os
+
 import numpy as np
 import torch
 
@@ -145,3 +147,28 @@ def sample_rows(R: int, k: int, seed: int):
     rows = set(rng.choice(R, size=min(k, R), replace=False).tolist())
     rows |= {0, R - 1}
     return sorted(rows)
+
+
+def host_threads() -> int:
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except Exception:  # pragma: no cover
+        return max(1, os.cpu_count() or 1)
+
+
+def row_parts(n_rows: int, parts: int):
+    cuts = [n_rows * i // parts for i in range(parts + 1)]
+    return [(a, b) for a, b in zip(cuts[:-1], cuts[1:]) if b > a]
+
+
+def oracle_whole(fmt: str, x_cpu, amax_g: float = 0.0, pool=None):
+    """The oracle's (y, codes, scales) of one whole tensor, its rows split into ranges
+    that run on host threads (the oracle's C calls release the GIL; rows are
+    independent given the tie-group amax, and every output is in flat row order, so
+    the concatenation is the one-call result)."""
+    if pool is None:
+        return oracle_outputs(fmt, x_cpu, amax_g)
+    parts = list(pool.map(lambda ab: oracle_outputs(fmt, x_cpu[ab[0]:ab[1]], amax_g),
+                          row_parts(x_cpu.shape[0], host_threads())))
+    cat = lambda k: None if parts[0][k] is None else np.concatenate([p[k] for p in parts])  # noqa: E731
+    return cat(0), cat(1), cat(2)

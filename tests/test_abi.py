@@ -61,7 +61,7 @@ int main(void) {
     memset(&t, 0, sizeof t);
     t.x = (const void*)0x1000; t.rows = 4; t.cols = 48; t.y = (void*)0x2000;
     t.codes = (void*)0x3000; t.scales = (void*)0x4000;
-    if (qf_version() != ((1 << 16) | 6)) return 1;
+    if (qf_version() != ((1 << 16) | 7)) return 1;
     if (strncmp(qf_status_string(QF_ERR_SHAPE), "QF_ERR_SHAPE", 12) != 0) return 2;
     if (qf_fakequant(QF_MXFP4, &t, 1, NULL, 0, NULL, NULL) != QF_ERR_SHAPE) return 3;
     if (qf_last_error()[0] == 0) return 4;
@@ -92,7 +92,7 @@ def test_struct_layout_matches_header(qf):
 def test_status_strings(qf):
     for s in range(7):
         assert qf.lib.qf_status_string(s).decode().startswith("QF_")
-    assert qf.lib.qf_version() == (1 << 16) | 6
+    assert qf.lib.qf_version() == (1 << 16) | 7
 
 
 def _tensor(qf, x=0x1000, rows=4, cols=64, group=0, y=0x2000, codes=0x3000, scales=0x4000,

@@ -151,3 +151,78 @@ def test_large_call_matches_two_calls():
     for i in range(len(xs)):
         assert torch.equal(y1[i].view(torch.int16), y2[i].view(torch.int16)), i
         assert torch.equal(c1[i], c2[i]) and torch.equal(s1[i], s2[i]), i
+
+
+def _guarded_call(xs, groups, ng, ws, tracked=None):
+    """One qf_amax_fakequant call into fresh guarded outputs (every byte 0xA5 beforehand,
+    the FP32 outputs NaN); returns the buffers."""
+    outs = [outputs("nvfp4", x) for x in xs]
+    amax = torch.full((ng,), float("nan"), device=DEV)
+    so = torch.full((ng,), float("nan"), device=DEV)
+    qf.qf_amax_fakequant(xs, [o[0].view(x.shape) for o, x in zip(outs, xs)],
+                         [o[1].view() for o in outs], [o[2].view() for o in outs], groups, amax,
+                         tracked=tracked, group_scale_out=so, workspace=ws)
+    return outs, amax, so
+
+
+def _untouched(outs, amax, so, label):
+    torch.cuda.synchronize()
+    for i, o in enumerate(outs):
+        for nm, g in zip(("y", "codes", "scales"), o):
+            assert bool((g.raw == 0xA5).all()), f"{label}: tensor {i} {nm} was written"
+    assert bool(torch.isnan(amax).all()) and bool(torch.isnan(so).all()), f"{label}: amax / s_t written"
+
+
+def test_barrier_timeout_is_reported_and_recovers():
+    """The bounded grid barrier runs out with every CTA present (the testing aid makes
+    it wait for one CTA more than the grid holds, at most 1000 polls).  Expected: no
+    output is written, the error flag is sticky (a second call on the workspace does
+    nothing), qf_workspace_check reports QF_ERR_TIMEOUT and clears it, the workspace
+    is all zero again, and the next call is bit-exact to the oracle."""
+    wl = workloads.nvfp4_tied(rows_scale=1 / 16, with_grads=False)
+    xs = [x.to(DEV) for x in wl["tensors"]]
+    groups, ng = wl["groups"], wl["n_groups"]
+    ws = qf.alloc_workspace(ng, DEV)
+    try:
+        qf.qf_test_barrier_timeout(1000)
+        outs, amax, so = _guarded_call(xs, groups, ng, ws)
+        _untouched(outs, amax, so, "timed-out call")
+    finally:
+        qf.qf_test_barrier_timeout(0)
+    # sticky: this call finds the flag at entry and does no work
+    outs2, amax2, so2 = _guarded_call(xs, groups, ng, ws)
+    _untouched(outs2, amax2, so2, "call after the timeout")
+    assert int(ws[4:].count_nonzero()) == 0, "counters / slots not reset by the timed-out calls"
+    with pytest.raises(qf.QfError) as e:
+        qf.qf_workspace_check(ws)
+    assert e.value.status == 6                           # QF_ERR_TIMEOUT
+    assert int(ws.count_nonzero()) == 0, "workspace not zero after the check"
+    qf.qf_workspace_check(ws)                            # cleared: QF_OK now
+    res = _run(wl["tensors"], groups, ng, workspace=ws)
+    _check_oracle(wl["tensors"], groups, ng, res, label="after timeout")
+
+
+def _nan_case(where):
+    wl = workloads.nvfp4_activation(rows_scale=1 / 256)
+    x = wl["tensors"][0].clone()
+    tracked = [np.float32(1.5)]
+    if where == "x":
+        x.view(-1)[12345] = float("nan")
+    else:
+        tracked = [np.float32("nan")]
+    return [x], wl["groups"], wl["n_groups"], tracked
+
+
+@pytest.mark.parametrize("where", ["x", "tracked"])
+def test_nan_folds_alike_on_both_paths(where):
+    """A NaN in x or in the running amax is outside the formats, but the call gives the
+    same bytes whether it takes the single launch or the two launches: both fold the
+    amax as the max of FP32 bit patterns, so the NaN propagates."""
+    xs, groups, ng, tracked = _nan_case(where)
+    one = _run(xs, groups, ng, tracked=tracked)
+    two = _run(xs, groups, ng, tracked=tracked, workspace=None)
+    for k in ("y", "codes", "scales"):
+        assert_same(f"{where}: {k}", one[k][0], two[k][0])
+    for k in ("amax", "s_t", "tracked"):
+        assert_same(f"{where}: {k}", one[k].view(np.uint32), two[k].view(np.uint32))
+    assert np.isnan(one["tracked"][0]) and np.isnan(one["s_t"][0])

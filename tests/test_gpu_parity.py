@@ -257,15 +257,6 @@ def test_errors_launch_nothing():
 
 # ----------------------------------------------------------------------------- full sizes
 @pytest.mark.slow
-def test_full_mxfp4_w4a4_sampled_rows():
-    wl = workloads.mxfp4_w4a4()
-    res = run_fakequant("mxfp4", wl["tensors"])
-    for i, x in enumerate(wl["tensors"]):
-        compare_rows("mxfp4", x, res["y"][i], res["codes"][i], res["scales"][i],
-                     sample_rows(x.shape[0], 48, 100 + i), label=f"w4a4[{i}]")
-
-
-@pytest.mark.slow
 def test_full_nvfp4_weight_whole():
     wl = workloads.nvfp4_weight()
     res = run_fakequant("nvfp4", wl["tensors"])
@@ -273,50 +264,8 @@ def test_full_nvfp4_weight_whole():
     compare_full("nvfp4", wl["tensors"], res, am, label="w4096")
 
 
-@pytest.mark.slow
-def test_full_q4k_sampled_rows():
-    wl = workloads.q4k_weights()
-    res = run_fakequant("q4k", wl["tensors"])
-    for i, x in enumerate(wl["tensors"]):
-        compare_rows("q4k", x, res["y"][i], res["codes"][i], None,
-                     sample_rows(x.shape[0], 48, 200 + i), label=f"q4k[{i}]")
-
-
-@pytest.mark.slow
-def test_full_nvfp4_tied_sampled_rows():
-    wl = workloads.nvfp4_tied(with_grads=False)
-    res = run_fakequant("nvfp4", wl["tensors"], wl["groups"], 2)
-    am = oracle.tied_amax(wl["tensors"], wl["groups"], 2)
-    assert_same("tied amax", res["amax"].view(np.uint32), am.view(np.uint32))
-    for i, x in enumerate(wl["tensors"]):
-        compare_rows("nvfp4", x, res["y"][i], res["codes"][i], res["scales"][i],
-                     sample_rows(x.shape[0], 32, 300 + i), float(am[wl["groups"][i]]),
-                     label=f"tied[{i}]")
-
-
-@pytest.mark.slow
-def test_full_moe_grouped_sampled_experts():
-    wl = workloads.moe_experts()
-    ts, groups, ng = wl["tensors"], wl["groups"], wl["n_groups"]
-    am = oracle.tied_amax(ts, groups, ng)
-    for fmt in ("nvfp4", "mxfp4", "q4k"):
-        res = run_fakequant(fmt, ts, groups, ng)
-        if fmt == "nvfp4":
-            assert_same("moe amax", res["amax"].view(np.uint32), am.view(np.uint32))
-        for i in (0, 1, 2, 190, 191, 380, 381, 382, 383):
-            compare_rows(fmt, ts[i], res["y"][i], res["codes"][i], res["scales"][i],
-                         sample_rows(ts[i].shape[0], 8, i), float(am[groups[i]]),
-                         label=f"moe {fmt} t{i}")
-
-
-@pytest.mark.slow
-def test_full_activation_tracked():
-    a = workloads.nvfp4_activation()["tensors"][0]
-    am = oracle.amax(a)
-    res = run_fakequant("nvfp4", [a], tracked=[0.0])
-    assert res["tracked"][0] == np.float32(am)
-    compare_rows("nvfp4", a, res["y"][0], res["codes"][0], res["scales"][0],
-                 sample_rows(a.shape[0], 48, 400), float(am), label="act")
+# The other full-size configurations are compared whole, every output byte, in
+# tests/test_gpu_fullsize.py.
 
 
 # ----------------------------------------------------------------------------- FP32 latent input
@@ -394,15 +343,6 @@ def test_q4k_mse_pack_and_clipped_ste():
     qf.qf_ste_backward(g.to(DEV), out, mode=1, fmt="q4k_mse", x=x.to(DEV))
     torch.cuda.synchronize()
     assert_same("q4k mse ste", bits(out), oracle.ste_backward(g, 1, "q4k_mse", x))
-
-
-@pytest.mark.slow
-def test_full_q4k_mse_sampled_rows():
-    wl = workloads.q4k_weights()
-    res = run_fakequant("q4k_mse", wl["tensors"])
-    for i, x in enumerate(wl["tensors"]):
-        compare_rows("q4k_mse", x, res["y"][i], res["codes"][i], None,
-                     sample_rows(x.shape[0], 24, 500 + i), label=f"q4k mse[{i}]")
 
 
 def test_q4k_clipped_ste_at_both_ends_of_the_code_range():
