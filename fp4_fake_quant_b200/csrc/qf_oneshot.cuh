@@ -22,7 +22,7 @@
 //
 // Every fold of the amax (slots, the tracked running value) takes the max of the FP32
 // bit patterns as unsigned integers, as k_amax does: for values >= +0 that is the
-// float max, and a NaN (sign bit clear) wins, on both paths of the call alike.
+// float max, and a NaN running value stays NaN, on both paths of the call alike.
 //
 // Workspace layout (32-bit words): [0] error flags, [1] reserved (0), [2] arrive
 // count, [3] depart count, [4 + g] group g's running max |x| as FP32 bits.

@@ -140,7 +140,7 @@ typedef struct qf_tensor {
  *                     d_group_amax of qf_fakequant to quantize with it).  Its
  *                     values must be >= +0 (start it at +0): the max is taken on
  *                     the FP32 bit patterns as unsigned integers, which is the
- *                     float max there (a NaN, outside the formats, propagates).
+ *                     float max there (a NaN running value stays NaN).
  *   Only x, rows, cols, group and x_type of each tensor are read; cols may be any
  *   value >= 0 here.  n == 0 only clears d_group_amax.
  * Errors: t == NULL with n > 0, n < 0, n_groups <= 0, d_group_amax == NULL,
@@ -228,7 +228,7 @@ qf_status qf_fakequant(qf_format f, const qf_tensor* t, int n, const float* d_gr
  *   bit patterns as unsigned integers, as qf_amax_tied does; that is the float max for
  *   values >= +0, so the running amax must start at +0 (or any value >= +0).  A NaN in
  *   x or in d_tracked is outside the formats (inputs are finite), but both paths of
- *   this call give the same bytes for it: the NaN propagates into the amax.
+ *   this call give the same bytes for it (a NaN running value stays NaN).
  * Errors: as qf_fakequant; a workspace smaller than needed -> QF_ERR_INVALID_ARG,
  *   not 16-byte aligned -> QF_ERR_ALIGN.
  */

@@ -217,7 +217,8 @@ def _nan_case(where):
 def test_nan_folds_alike_on_both_paths(where):
     """A NaN in x or in the running amax is outside the formats, but the call gives the
     same bytes whether it takes the single launch or the two launches: both fold the
-    amax as the max of FP32 bit patterns, so the NaN propagates."""
+    running amax as the max of FP32 bit patterns (a NaN running value stays NaN), and
+    both take the block maxima of x alike."""
     xs, groups, ng, tracked = _nan_case(where)
     one = _run(xs, groups, ng, tracked=tracked)
     two = _run(xs, groups, ng, tracked=tracked, workspace=None)
@@ -225,4 +226,5 @@ def test_nan_folds_alike_on_both_paths(where):
         assert_same(f"{where}: {k}", one[k][0], two[k][0])
     for k in ("amax", "s_t", "tracked"):
         assert_same(f"{where}: {k}", one[k].view(np.uint32), two[k].view(np.uint32))
-    assert np.isnan(one["tracked"][0]) and np.isnan(one["s_t"][0])
+    if where == "tracked":
+        assert np.isnan(one["tracked"][0]) and np.isnan(one["s_t"][0])
