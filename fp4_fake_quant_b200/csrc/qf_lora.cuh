@@ -5,10 +5,11 @@
 // The merged weight is formed on the fly and never written unless asked for:
 //   acc = sum over k = 0..r-1, in increasing k, of B[i,k] * A[k,j]   (FP32)
 //   M   = BF16(W[i,j] + scale * acc)
-// A BF16 x BF16 product has at most 16 significant bits, so it is exact in FP32
-// and one FMA per term rounds exactly like the separate multiply and add; the
-// fixed order makes the result reproducible bit for bit (tensor cores are not
-// used because their accumulation order is not specified).
+// Each term is one fused multiply-add (acc + b*a rounded once; a BF16 x BF16 product
+// has at most 16 significant bits, so this is also the separate multiply and add
+// unless the product underflows); the fixed order makes the result reproducible bit
+// for bit (tensor cores are not used because their accumulation order is not
+// specified).
 //
 // Layout: lane l owns 4 consecutive columns, a warp a 128-column slab, a CTA
 // kLoraThreads / 32 slabs (1024 columns at 256 threads) by kLoraRows rows.  The warp
@@ -18,8 +19,7 @@
 //
 // The products run on sm_100's paired FP32 pipe: one fma.rn.f32x2 updates the
 // accumulators of two adjacent columns, each rounded exactly as a scalar
-// fma.rn.f32 would be (and, the products being exact, as a separate multiply and
-// add would be).  Operands and accumulators live in 64-bit registers from load to
+// fma.rn.f32 would be.  Operands and accumulators live in 64-bit registers from load to
 // use, so no pair is ever repacked.  B is stored in shared memory with every value
 // twice, so one 16-byte load yields the (b, b) operand pairs of two consecutive k.
 //
@@ -111,7 +111,7 @@ __device__ __forceinline__ float2 unpk2(uint64_t v) {
     asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
     return r;
 }
-// d = a * b + c on both halves, each rounded once (the products here are exact)
+// d = a * b + c on both halves, each rounded once (fused: the product is not rounded)
 __device__ __forceinline__ uint64_t fma2_pk(uint64_t a, uint64_t b, uint64_t c) {
     uint64_t d;
     asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));

@@ -316,7 +316,7 @@ qf_status qf_ste_backward(qf_format f, const void* grad_y, void* grad_x, int64_t
  * on a frozen BF16 base and quantizes the merged weight, not the base).
  * For tensor t with base W = t.x (BF16 [rows, cols]):
  *   acc = sum over k = 0..rank-1, in increasing k, of b[i,k] * a[k,j]   (FP32; each
- *         BF16 x BF16 product is exact in FP32, each sum is rounded)
+ *         term is one fused multiply-add, acc + b*a rounded once)
  *   M   = BF16( W[i,j] + scale * acc )      (an FP32 multiply, an FP32 add, RNE)
  * M is the merged weight a BF16 model holds after merging the adapter.
  *   b       BF16 [rows, rank] row-major (device)

@@ -647,7 +647,9 @@ void qfo_ste_backward_x(const uint16_t* grad_y, uint16_t* grad_x, int64_t numel,
 /* base and quantizes W + B A, not W.  Reading: the merged weight is what a  */
 /* BF16 model would hold after merging --                                    */
 /*   acc  = sum over k = 0..r-1, in increasing k, of B[i,k] * A[k,j]  (FP32; */
-/*          a BF16 x BF16 product is exact in FP32, each sum is rounded)     */
+/*          each term is one fused multiply-add: acc + B*A rounded once.    */
+/*          A BF16 x BF16 product has at most 16 significant bits, so this  */
+/*          equals multiply-then-add unless the product underflows FP32)    */
 /*   M    = BF16( W[i,j] + scale * acc )   (FP32 multiply, FP32 add, RNE)    */
 /* B is [rows, r] and A is [r, cols], both BF16 row-major; scale is FP32      */
 /* (alpha / r in the usual parameterisation).                                */
@@ -658,10 +660,9 @@ void qfo_lora_merge(const uint16_t* w, const uint16_t* b, const uint16_t* a, int
     for (int64_t i = 0; i < rows; ++i) {
         for (int64_t j = 0; j < cols; ++j) {
             float acc = 0.0f;
-            for (int k = 0; k < rank; ++k) {
-                float prod = qfo_bf16_to_f32(b[i * rank + k]) * qfo_bf16_to_f32(a[(int64_t)k * cols + j]);
-                acc = acc + prod;
-            }
+            for (int k = 0; k < rank; ++k)
+                acc = fmaf(qfo_bf16_to_f32(b[i * rank + k]),
+                           qfo_bf16_to_f32(a[(int64_t)k * cols + j]), acc);
             float d = scale * acc;
             m[i * cols + j] = qfo_f32_to_bf16(qfo_bf16_to_f32(w[i * cols + j]) + d);
         }

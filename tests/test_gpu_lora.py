@@ -213,3 +213,27 @@ def test_merge_accumulates_in_increasing_k(rank_pad):
         qf.qf_lora_merge([w], [(b, a, 1.0)], [m])
         torch.cuda.synchronize()
         assert np.all(bits(m) == want), (order, [hex(v) for v in bits(m)[:4]])
+
+
+def test_underflowing_product_is_fused_on_the_device():
+    """The oracle's worked case (products 2^-149 then 2^-150; W = 0, scale = 2^100):
+    the device's fused terms give the merged weight 2^-48, as the oracle does, in the
+    merge call and in the fused fake-quant."""
+    cols = 32
+    w = torch.zeros(1, cols, dtype=torch.bfloat16)
+    b = torch.tensor([[2.0 ** -75, 2.0 ** -75]], dtype=torch.bfloat16)
+    a = torch.tensor([[2.0 ** -74] * cols, [2.0 ** -75] * cols], dtype=torch.bfloat16)
+    scale = 2.0 ** 100
+    want = oracle.lora_merge(w, b, a, scale)
+    assert int(want[0, 0]) == 0x2780
+    wd = w.to(DEV)
+    m = torch.empty_like(wd)
+    qf.qf_lora_merge([wd], [(b.to(DEV), a.to(DEV), scale)], [m])
+    torch.cuda.synchronize()
+    assert_same("fused merge", bits(m), want)
+    y, c, s = qf.alloc_outputs("mxfp4", wd)
+    qf.qf_fakequant_lora("mxfp4", [wd], [(b.to(DEV), a.to(DEV), scale)], [y], [c], [s])
+    torch.cuda.synchronize()
+    yo, co, so = oracle.mxfp4(want)
+    assert_same("fused merge, MXFP4 y", bits(y), yo)
+    assert_same("fused merge, MXFP4 codes", u8(c), co)

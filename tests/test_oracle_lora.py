@@ -100,3 +100,42 @@ def test_accumulation_order_is_increasing_k():
     # the same products in decreasing k reach the other side of the BF16 tie
     rev = f32(oracle.lora_merge(w, b[:, ::-1].copy(), a[::-1, :].copy(), 1.0).astype(np.uint32))
     assert rev.reshape(-1).tolist() == [1.0 + 2.0 ** -7]
+
+
+def _fused_chain_reference(w, b, a, scale):
+    """The merge with each term rounded once (acc + b*a), emulated in float64: every
+    b*a of BF16 operands is exact in float64, and rounding acc + b*a first to binary64
+    and then to binary32 equals rounding it once to binary32 (the binary64 precision is
+    at least twice binary32's plus two, and both addends are binary32 values here)."""
+    wf, bf, af = f32(w), f32(b), f32(a)
+    rows, cols = wf.shape
+    r = bf.shape[1]
+    acc = np.zeros((rows, cols), np.float32)
+    for k in range(r):
+        prod = bf[:, k:k + 1].astype(np.float64) * af[k:k + 1, :].astype(np.float64)
+        acc = (acc.astype(np.float64) + prod).astype(np.float32)
+    d = (np.float32(scale) * acc).astype(np.float32)
+    return bf16((wf + d).astype(np.float32))
+
+
+def test_merge_is_one_rounding_per_term_on_random_adapters():
+    rng = np.random.default_rng(11)
+    rows, cols, r = 16, 128, 16
+    w = workloads.bf16_bits(workloads.normal_with_outliers(rows, cols, 0.02, 1e-3, 20, 12, 0))
+    b = bf16(rng.standard_normal((rows, r)) * 0.01)
+    a = bf16(rng.standard_normal((r, cols)) * 0.02)
+    got = oracle.lora_merge(w, b, a, 2.0)
+    assert np.array_equal(got, _fused_chain_reference(w, b, a, 2.0))
+
+
+def test_underflowing_product_is_fused_into_the_sum():
+    """A worked case where a product underflows FP32.  Terms: b0*a0 = 2^-149 (the
+    smallest subnormal) and b1*a1 = 2^-150.  Fused: acc = RN(2^-149 + 2^-150), a tie
+    between 2^-149 and 2^-148 that goes to the even 2^-148.  Multiplying first would
+    round 2^-150 to 0 (a tie, to even) and leave acc = 2^-149.  With W = 0 and
+    scale = 2^100 the merged weight is 2^-48 (0x2780) fused, 2^-49 (0x2700) if not."""
+    w = np.zeros((1, 2), np.uint16)
+    b = bf16(np.float32([[2.0 ** -75, 2.0 ** -75]] * 1))
+    a = bf16(np.float32([[2.0 ** -74, 2.0 ** -74], [2.0 ** -75, 2.0 ** -75]]))
+    got = oracle.lora_merge(w, b, a, 2.0 ** 100)
+    assert got.tolist() == [[0x2780, 0x2780]]
