@@ -373,6 +373,42 @@ qf_status lora_launch_r(const std::vector<qf::LoraTensor>& v, const float* am, f
     return QF_OK;
 }
 
+// k_lora_amax over the tensors of a call (units of kLoraAmaxRows rows x kLoraCols
+// columns); folds each tie group's exact max |M| into d_group_amax, which must hold
+// exact values only (zeros, or an earlier fold of the same group).
+qf_status lora_amax_launch(const std::vector<qf::LoraTensor>& v, float* am, cudaStream_t s) {
+    for (size_t b = 0; b < v.size(); b += kLoraLargeT) {
+        const size_t cnt = std::min<size_t>(kLoraLargeT, v.size() - b);
+        auto fill = [&](auto& P) {
+            memset(&P, 0, sizeof P);
+            int64_t u = 0;
+            for (size_t i = 0; i < cnt; ++i) {
+                qf::LoraTensor d = v[b + i];
+                d.unit_begin = u;
+                u += ((d.rows + qf::kLoraAmaxRows - 1) / qf::kLoraAmaxRows) * d.col_groups;
+                P.t[i] = d;
+            }
+            P.total_units = u;
+            P.n = (int)cnt;
+            P.group_amax = am;
+        };
+        if (cnt <= (size_t)kLoraSmallT) {
+            qf::LoraTable<kLoraSmallT> P;
+            fill(P);
+            qf::k_lora_amax<kLoraSmallT>
+                <<<(unsigned)std::max<int64_t>(1, P.total_units), qf::kLoraThreads, 0, s>>>(P);
+        } else {
+            qf::LoraTable<kLoraLargeT> P;
+            fill(P);
+            qf::k_lora_amax<kLoraLargeT>
+                <<<(unsigned)std::max<int64_t>(1, P.total_units), qf::kLoraThreads, 0, s>>>(P);
+        }
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+    }
+    return QF_OK;
+}
+
 template <int MODE>
 qf_status lora_launch(const std::vector<qf::LoraTensor>& v, int max_rank, const float* am,
                       float* so, int ng, cudaStream_t s) {
@@ -587,7 +623,7 @@ qf_status qf_amax_tied_lora(const qf_tensor* t, const qf_lora* l, int n, float* 
     cudaError_t e = cudaMemsetAsync(d_group_amax, 0, sizeof(float) * (size_t)n_groups, s);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
     if (v.empty()) return QF_OK;
-    return lora_launch<qf::kLoraAmax>(v, max_rank, d_group_amax, nullptr, n_groups, s);
+    return lora_amax_launch(v, d_group_amax, s);
 }
 
 qf_status qf_fakequant_lora(qf_format f, const qf_tensor* t, const qf_lora* l, int n,
@@ -638,7 +674,7 @@ qf_status qf_amax_fakequant_lora(const qf_tensor* t, const qf_lora* l, int n,
     if (v.empty() || !all_y) {
         // no room for the merged weight: form it twice (amax pass, then fused pass)
         if (!v.empty()) {
-            st = lora_launch<qf::kLoraAmax>(v, max_rank, d_group_amax, nullptr, n_groups, s);
+            st = lora_amax_launch(v, d_group_amax, s);
             if (st != QF_OK) return st;
         }
         if (v.empty() && !d_group_scale_out) return QF_OK;

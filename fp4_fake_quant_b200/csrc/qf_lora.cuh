@@ -383,4 +383,211 @@ __global__ void __launch_bounds__(kLoraThreads) k_lora(const __grid_constant__ L
     }
 }
 
+
+// ------------------------------------------------------------------ merged-weight amax
+// k_lora_amax: the exact max |M| of a tie group's merged weights, M = BF16(W + s * acc),
+// with the rank-r merge evaluated only where it can decide the result.
+//
+// Bounds.  With R_i = sum_k |b_ik| (FP32) and C_j = max_k |a_kj|, every term satisfies
+// |b_ik a_kj| <= |b_ik| C_j, so |sum_k b_ik a_kj| <= R_i C_j.  The fused sum, the
+// scaling, the add and the BF16 rounding each add at most one rounding (or, where the
+// value is subnormal, an absolute error below 2^-133), so for
+//   D_ij = K_i C_j + 2^-120 + |s| 2^-140,   K_i = |s| R_i (1 + 2^-6)
+//   (D_ij = 0 when K_i or C_j is 0: every product is then an exact zero and M = W)
+// every element satisfies
+//   lb = (|W| - D_ij)(1 - 2^-7) - 2^-120  <=  |M|  <=  (|W| + D_ij)(1 + 2^-7) = ub,
+// with the FP32 rounding of these expressions themselves inside the margins (2^-6 and
+// 2^-7 against a few 2^-24).  An element whose ub is below a lower bound of the group's
+// max |M| cannot be that max.  The lower bounds used: the lb of any element, and the
+// exact |M| of any evaluated element, including the group's current amax (the output
+// only ever receives exact values).
+//
+// Pass 1 reads the CTA's tile (kLoraAmaxRows rows x 1024 columns) and keeps, per row and
+// lane, the max |W| of the lane's 32 elements; the CTA's best lb follows from it.
+// Pass 2 revisits only the (row, lane) pieces whose bound reaches that lower bound,
+// re-reads their 32 elements (from L2) and evaluates the merge exactly, with the merge
+// kernel's arithmetic, where the element's own bound still reaches it.  The result is the
+// max over the evaluated elements: exact, since the max element is always evaluated.
+#ifndef QF_LORA_AMAX_ROWS
+#define QF_LORA_AMAX_ROWS 128
+#endif
+constexpr int kLoraAmaxRows = QF_LORA_AMAX_ROWS;     // a multiple of 2 * kLoraThreads / 32
+constexpr float kBoundUp = 1.0f + 0x1p-7f;
+constexpr float kBoundDown = 1.0f - 0x1p-7f;
+constexpr float kBoundWiden = 1.0f + 0x1p-6f;
+constexpr float kBoundTiny = 0x1p-120f;
+
+// |M| of element (i, j) as FP32: the merge of k_lora, one element at a time
+__device__ __forceinline__ float lora_merged_mag(const LoraTensor& T, int64_t i, int64_t j,
+                                                 float w) {
+    const uint16_t* bp = T.b + i * T.rank;
+    const uint16_t* ap = T.a + j;
+    float acc = 0.0f;
+    for (int k = 0; k < T.rank; ++k)
+        acc = __fmaf_rn(bf16_lo(bp[k]), bf16_lo(ap[k * T.cols]), acc);
+    const uint32_t m = cvt_bf16x2(0.0f, __fadd_rn(w, __fmul_rn(T.scale, acc)));
+    return __uint_as_float((m & 0x7FFFu) << 16);
+}
+
+__device__ __forceinline__ uint32_t max_abs_bf16x8(uint32_t m, uint4 v) {
+    m = max_u16x2(m, v.x & 0x7FFF7FFFu);
+    m = max_u16x2(m, v.y & 0x7FFF7FFFu);
+    m = max_u16x2(m, v.z & 0x7FFF7FFFu);
+    return max_u16x2(m, v.w & 0x7FFF7FFFu);
+}
+
+template <int MAXT>
+__global__ void __launch_bounds__(kLoraThreads) k_lora_amax(const __grid_constant__ LoraTable<MAXT> P) {
+    constexpr int kWarps = kLoraThreads / 32;
+    constexpr int kRpw = kLoraAmaxRows / kWarps;         // rows per warp, read two at a time
+    constexpr int kChunks = kLoraCols / 8;                // 16-byte column chunks per tile row
+    static_assert(kLoraAmaxRows % (2 * kWarps) == 0, "row pairs per warp");
+    static_assert(kLoraThreads >= 2 * kChunks && kLoraThreads >= kLoraAmaxRows, "prologue shape");
+    __shared__ float s_k[kLoraAmaxRows];                  // K_i
+    __shared__ float s_c[kLoraCols];                      // C_j
+    __shared__ uint4 s_cpart[2][kChunks];                 // per-chunk |a| maxima, two k halves
+    __shared__ uint32_t s_lb, s_best;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    if (blockIdx.x >= P.total_units) return;
+    const LoraTensor& T = P.t[lora_locate(P, blockIdx.x)];
+    const int64_t local = blockIdx.x - T.unit_begin;
+    const int64_t r0 = (local / T.col_groups) * kLoraAmaxRows;
+    const int64_t c_base = (local % T.col_groups) * kLoraCols;
+    const int nrows = (int)min(T.rows - r0, (int64_t)kLoraAmaxRows);
+    const int ncols = (int)min(T.cols - c_base, (int64_t)kLoraCols);   // a multiple of 16
+    const int nchunks = ncols / 8;
+    const int64_t cols = T.cols;
+    const int rank = T.rank;
+    const float sabs = fabsf(T.scale);
+    const float tiny = __fadd_rn(kBoundTiny, __fmul_rn(sabs, 0x1p-140f));
+    unsigned int* gamax = reinterpret_cast<unsigned int*>(const_cast<float*>(P.group_amax)) + T.group;
+
+    // ---- prologue: C_j (16-byte loads of A, k split over two threads per chunk), K_i,
+    // and the group's amax so far
+    {
+        const int c = threadIdx.x >> 1, h = threadIdx.x & 1;
+        if (c < nchunks) {
+            const uint16_t* ap = T.a + c_base + 8 * c;
+            uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
+#pragma unroll 4
+            for (int k = h; k < rank; k += 2) {
+                const uint4 v = ld_stream<1>(ap + k * cols);
+                m0 = max_u16x2(m0, v.x & 0x7FFF7FFFu);
+                m1 = max_u16x2(m1, v.y & 0x7FFF7FFFu);
+                m2 = max_u16x2(m2, v.z & 0x7FFF7FFFu);
+                m3 = max_u16x2(m3, v.w & 0x7FFF7FFFu);
+            }
+            s_cpart[h][c] = make_uint4(m0, m1, m2, m3);
+        }
+    }
+    if (threadIdx.x < nrows) {
+        const uint16_t* bp = T.b + (r0 + threadIdx.x) * rank;
+        float r = 0.0f;
+#pragma unroll 8
+        for (int k = 0; k < rank; ++k) r = __fadd_rn(r, fabsf(bf16_lo(bp[k])));
+        s_k[threadIdx.x] = __fmul_rn(__fmul_rn(sabs, r), kBoundWiden);
+    }
+    if (threadIdx.x == 0) {
+        s_best = *reinterpret_cast<volatile unsigned int*>(gamax);
+        s_lb = 0u;
+    }
+    __syncthreads();
+    if (threadIdx.x < nchunks) {
+        const uint4 p0 = s_cpart[0][threadIdx.x], p1 = s_cpart[1][threadIdx.x];
+        const uint32_t m[4] = {max_u16x2(p0.x, p1.x), max_u16x2(p0.y, p1.y),
+                               max_u16x2(p0.z, p1.z), max_u16x2(p0.w, p1.w)};
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            s_c[8 * threadIdx.x + e] = __uint_as_float(((m[e >> 1] >> (16 * (e & 1))) & 0xFFFFu) << 16);
+    }
+    __syncthreads();
+
+    // this lane's columns: c_base + 256 q + 8 lane + e, q < 4, e < 8
+    float cmax = 0.0f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        if (256 * q + 8 * lane < ncols)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) cmax = fmaxf(cmax, s_c[256 * q + 8 * lane + e]);
+    auto dbound = [&](float k, float c) {
+        return (k > 0.0f && c > 0.0f) ? __fadd_rn(__fmul_rn(k, c), tiny) : 0.0f;
+    };
+    const uint16_t* wlane = T.w + r0 * cols + c_base + 8 * lane;
+
+    // ---- pass 1: max |W| per (row, lane), two rows (eight 16-byte loads) at a time;
+    // the best lower bound
+    float mrow[kRpw];
+    float lb_best = 0.0f;
+#pragma unroll
+    for (int t = 0; t < kRpw; t += 2) {
+        const int i0 = wid + kWarps * t, i1 = i0 + kWarps;
+        uint4 v[2][4];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                v[h][q] = (i0 + h * kWarps < nrows && 256 * q + 8 * lane < ncols)
+                              ? ld_stream<0>(wlane + (i0 + h * kWarps) * cols + 256 * q)
+                              : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            uint32_t m = 0;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) m = max_abs_bf16x8(m, v[h][q]);
+            const int i = h ? i1 : i0;
+            mrow[t + h] = __uint_as_float(bf16x2_max_bits(m));
+            if (i < nrows) {
+                const float lb = __fsub_rn(__fmul_rn(__fsub_rn(mrow[t + h], dbound(s_k[i], cmax)),
+                                                     kBoundDown), kBoundTiny);
+                lb_best = fmaxf(lb_best, lb);
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lb_best = fmaxf(lb_best, __shfl_xor_sync(kFull, lb_best, o));
+    if (lane == 0 && lb_best > 0.0f) atomicMax(&s_lb, __float_as_uint(lb_best));
+    __syncthreads();
+
+    // ---- pass 2: exact merges where the bound reaches the lower bound.  The (row, lane)
+    // pieces to revisit are marked first (unrolled, so mrow stays in registers); the
+    // rare revisits then run as plain loops.
+    float best = __uint_as_float(s_best);                 // exact: the group's amax so far
+    const float L = fmaxf(__uint_as_float(s_lb), best);
+    uint32_t cand = 0;
+#pragma unroll
+    for (int t = 0; t < kRpw; ++t) {
+        const int i = wid + kWarps * t;
+        const float rowub = __fmul_rn(__fadd_rn(mrow[t], dbound(i < nrows ? s_k[i] : 0.0f, cmax)),
+                                      kBoundUp);
+        if (i < nrows && rowub >= L && rowub > best) cand |= 1u << t;
+    }
+#pragma unroll 1
+    while (cand) {
+        const int t = __ffs(cand) - 1;
+        cand &= cand - 1;
+        const int i = wid + kWarps * t;
+        const float ki = s_k[i];
+#pragma unroll 1
+        for (int q = 0; q < 4; ++q) {
+            const int c0 = 256 * q + 8 * lane;
+            if (c0 >= ncols) continue;
+            const uint4 v = ld_stream<1>(wlane + i * cols + 256 * q);
+            const uint64_t lo = v.x | (uint64_t)v.y << 32, hi = v.z | (uint64_t)v.w << 32;
+#pragma unroll 1
+            for (int e = 0; e < 8; ++e) {
+                const uint32_t wb = (uint32_t)(((e < 4 ? lo : hi) >> (16 * (e & 3))) & 0xFFFFu);
+                const float x = __uint_as_float((wb & 0x7FFFu) << 16);
+                const float ub = __fmul_rn(__fadd_rn(x, dbound(ki, s_c[c0 + e])), kBoundUp);
+                if (ub >= L && ub > best)
+                    best = fmaxf(best, lora_merged_mag(T, r0 + i, c_base + c0 + e,
+                                                       __uint_as_float(wb << 16)));
+            }
+        }
+    }
+    // ---- the CTA's best exact value into the group's amax
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) best = fmaxf(best, __shfl_xor_sync(kFull, best, o));
+    if (lane == 0 && best > 0.0f) atomicMax(gamax, __float_as_uint(best));
+}
+
 }  // namespace qf

@@ -145,3 +145,59 @@ def test_global_scale_edge_cases():
     assert export.nvfp4_global_scale(0.0) == 1.0                  # every block scale is 0
     assert export.nvfp4_global_scale(2688.0) == 1.0
     assert export.nvfp4_global_scale(1e-44) == 1.0                # 2688 / a overflows FP32
+
+
+def _ct_decompress_nvfp4(codes, scales, rows, cols, amax):
+    from compressed_tensors.compressors.nvfp4.base import NVFP4PackedCompressor
+    from compressed_tensors.quantization import QuantizationScheme
+    from compressed_tensors.quantization.quant_scheme import PRESET_SCHEMES
+    t = export.compressed_tensors_nvfp4("w", torch.from_numpy(codes), torch.from_numpy(scales),
+                                        rows, cols, amax)
+    sd = {k.split(".", 1)[1]: v for k, v in t.items()}
+    scheme = QuantizationScheme(targets=["Linear"], **PRESET_SCHEMES["NVFP4"])
+    w = NVFP4PackedCompressor.decompress(sd, scheme)["weight"].to(torch.bfloat16)
+    return workloads.bf16_bits(w).reshape(-1)
+
+
+def test_compressed_tensors_nvfp4_decoder_relation():
+    """What the engine's decoder computes, and how it relates to the training path's y.
+
+    compressed-tensors rebuilds each weight as BF16(code * RN(sb / g)) with the global
+    scale g = RN(2688 / amax); the training path's y is BF16(code * RN(sb * s_t)) with
+    s_t = RN(amax / 2688).  The two block scales differ in the last FP32 bit for about
+    a third of (sb, amax) pairs, which changes y only when code * S lies within one FP32
+    unit of a BF16 rounding midpoint.  On the tied projections at 1/64 of the rows the
+    count of differing elements is the one the committed script
+    (tests/golden/make_ct_nvfp4_decoder_diff.py) recorded, as it is at full size; and a
+    constructed block (amax 0.01495361328125, sb 11 * 2^-9, code 1.5) shows a difference
+    of one BF16 unit that the decoder's formula explains."""
+    import json
+    import os
+    import ml_dtypes
+    gold = json.load(open(os.path.join(os.path.dirname(__file__), "golden",
+                                       "ct_nvfp4_decoder_diff.json")))
+    wl = workloads.nvfp4_tied(rows_scale=1 / 64, with_grads=False)
+    am = oracle.tied_amax(wl["tensors"], wl["groups"], wl["n_groups"])
+    n = d = 0
+    for x, gi in zip(wl["tensors"], wl["groups"]):
+        rows, cols = x.shape
+        y, codes, scales, _ = oracle.nvfp4(x, float(am[gi]))
+        w = _ct_decompress_nvfp4(codes, scales, rows, cols, float(am[gi]))
+        n, d = n + y.size, d + int(np.count_nonzero(w != y))
+    assert (n, d) == (gold["rows_scale_1_64"]["elements"], gold["rows_scale_1_64"]["differing"])
+
+    amax = np.float32(0.01495361328125)                     # a BF16 value
+    x = np.zeros((1, 32), np.float32)
+    x[0, 0] = amax                                          # block 0: the group max
+    x[0, 16] = np.float32(6.966292858123779e-07)            # block 1: sb = 11 * 2^-9
+    x[0, 17] = np.float32(1.7881393432617188e-07)           # code 1.5 in block 1
+    xb = x.astype(ml_dtypes.bfloat16).view(np.uint16)
+    y, codes, scales, s_t = oracle.nvfp4(xb, float(amax))
+    assert scales[1] == 11 and (codes[8] >> 4) == 3
+    w = _ct_decompress_nvfp4(codes, scales, 1, 32, float(amax))
+    sb = np.float32(11 * 2.0 ** -9)
+    g = np.float32(np.float32(2688.0) / amax)
+    want_ct = np.float32(np.float32(1.5) * np.float32(sb / g)).astype(ml_dtypes.bfloat16).view(np.uint16)
+    want_y = np.float32(np.float32(1.5) * np.float32(sb * np.float32(s_t))).astype(ml_dtypes.bfloat16).view(np.uint16)
+    assert w[17] == want_ct and y[17] == want_y and int(want_ct) != int(want_y)
+    assert abs(int(w[17]) - int(y[17])) == 1                # one BF16 unit apart

@@ -237,3 +237,76 @@ def test_underflowing_product_is_fused_on_the_device():
     yo, co, so = oracle.mxfp4(want)
     assert_same("fused merge, MXFP4 y", bits(y), yo)
     assert_same("fused merge, MXFP4 codes", u8(c), co)
+
+
+# ----------------------------------------------------------------------------- merged amax
+# qf_amax_tied_lora evaluates the merge only where a bound on |M| reaches a lower bound
+# of the group's max; these cases make the bounds decide the result, or make them
+# useless, and compare the group amax with the oracle's (merge, then max |M|).
+def _amax_case(ts, ads, groups, ng):
+    want = np.zeros(ng, np.float32)
+    for (w, (b, a, s)), g in zip(zip(ts, ads), groups):
+        want[g] = max(want[g], np.float32(oracle.amax(oracle.lora_merge(w, b, a, s))))
+    amax = torch.full((ng,), float("nan"), device=DEV)
+    qf.qf_amax_tied_lora([w.to(DEV) for w in ts], [(b.to(DEV), a.to(DEV), s) for b, a, s in ads],
+                         groups, amax)
+    torch.cuda.synchronize()
+    assert_same("merged amax", amax.cpu().numpy().view(np.uint32), want.view(np.uint32))
+
+
+def _bf16(a):
+    return torch.from_numpy(np.asarray(a, np.float32)).to(torch.bfloat16)
+
+
+def test_merged_amax_where_the_merge_moves_the_max():
+    """The largest |W| shrinks and the second largest grows past it: the max is not at
+    the argmax of |W|, and both lie inside each other's bounds."""
+    rows, cols, r = 64, 1024, 4
+    w = np.zeros((rows, cols), np.float32)
+    w[5, 100], w[40, 900] = 1.0, 0.98
+    b = np.zeros((rows, r), np.float32)
+    a = np.zeros((r, cols), np.float32)
+    b[5, 0], a[0, 100] = 0.25, -0.125                      # M[5,100] = 1 - 2 * 0.03125
+    b[40, 1], a[1, 900] = 0.25, 0.125                       # M[40,900] = 0.98 + 0.0625
+    _amax_case([_bf16(w)], [(_bf16(b), _bf16(a), 2.0)], [0], 1)
+
+
+@pytest.mark.parametrize("case", ["zero_base", "zero_adapter", "zero_scale", "negative_scale",
+                                  "huge_scale", "ties", "subnormal_base", "all_zero"])
+def test_merged_amax_edge_cases(case):
+    rows, cols, r = 70, 1040, 8                            # a ragged row tile and column group
+    w = workloads.normal_with_outliers(rows, cols, 0.02, 1e-3, 20.0, 31, 0)
+    b = workloads.normal_with_outliers(rows, r, 0.01, 0.0, 1.0, 31, 1)
+    a = workloads.normal_with_outliers(r, cols, 0.02, 0.0, 1.0, 31, 2)
+    s = 2.0
+    if case == "zero_base":          # the max comes from the merge alone: no pruning possible
+        w = torch.zeros_like(w)
+    elif case == "zero_adapter":     # B = 0 (the usual initialisation): M = W exactly
+        b = torch.zeros_like(b)
+    elif case == "zero_scale":
+        s = 0.0
+    elif case == "negative_scale":
+        s = -3.0
+    elif case == "huge_scale":       # the bounds overflow to inf: every element is evaluated
+        s = 1e30
+    elif case == "ties":             # many elements share the largest |W|
+        w = torch.where(w.abs() > 0.03, torch.sign(w) * 0.5, w).to(torch.bfloat16)
+    elif case == "subnormal_base":   # BF16 subnormals with a tiny adapter
+        w = (w.float() * 1e-37).to(torch.bfloat16)
+        b = (b.float() * 1e-20).to(torch.bfloat16)
+        a = (a.float() * 1e-19).to(torch.bfloat16)
+    elif case == "all_zero":
+        w, b = torch.zeros_like(w), torch.zeros_like(b)
+    _amax_case([w], [(b, a, s)], [0], 1)
+
+
+def test_merged_amax_many_tensors_and_groups():
+    """Expert-like tensors in several tie groups, each spread over many CTAs."""
+    ts, ads, groups = [], [], []
+    for e in range(4):
+        for j, (rr, c) in enumerate([(200, 2048), (200, 2048), (512, 768)]):
+            w, b, a = _case(rr, c, 16, 700 + 3 * e + j)
+            ts.append(w)
+            ads.append((b, a, 2.0))
+            groups.append(2 * e + (j == 2))
+    _amax_case(ts, ads, groups, 8)
