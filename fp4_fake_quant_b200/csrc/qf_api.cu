@@ -29,6 +29,9 @@ constexpr int kFp4U = QF_FP4_U;  // 256-element sub-tiles per warp unit
 #define QF_AMAX_U 4
 #endif
 constexpr int kAmaxU = QF_AMAX_U;
+#ifndef QF_NV_REVERSE
+#define QF_NV_REVERSE 1         // NVFP4 fused pass: units from the last one down (k_nv)
+#endif
 #ifndef QF_NOALLOC_MAX_GROUPS
 #define QF_NOALLOC_MAX_GROUPS 4092     // 4 header words + 4092 slots = 16 KB of static scratch
 #endif
@@ -158,7 +161,7 @@ template <typename KS, typename KL>
 qf_status launch_chunks(KS small_kernel, KL large_kernel, int threads, int waves,
                         const std::vector<DevTensor>& v, int64_t unit_elems, const float* amax,
                         float* scale_out, float* tracked, int n_groups, cudaStream_t s,
-                        bool dependent = false) {
+                        bool dependent = false, bool reverse = false) {
     Launch Ls, Ll;
     qf_status st = launch_shape(small_kernel, threads, waves, &Ls);
     if (st != QF_OK) return st;
@@ -180,6 +183,7 @@ qf_status launch_chunks(KS small_kernel, KL large_kernel, int threads, int waves
             Table<kSmallT> P;
             fill_table(P, v, b, cnt, unit_elems);
             P.group_amax = amax; P.group_scale_out = so; P.tracked = tracked; P.n_groups = n_groups;
+            P.reverse = reverse;
             if (dependent) {
                 cudaError_t e = launch_dependent(small_kernel, grid_for(Ls, P.total_units), threads, P, s);
                 if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx");
@@ -190,6 +194,7 @@ qf_status launch_chunks(KS small_kernel, KL large_kernel, int threads, int waves
             Table<kLargeT> Q;              // ~27 KB kernel parameter
             fill_table(Q, v, b, cnt, unit_elems);
             Q.group_amax = amax; Q.group_scale_out = so; Q.tracked = tracked; Q.n_groups = n_groups;
+            Q.reverse = reverse;
             if (dependent) {
                 cudaError_t e = launch_dependent(large_kernel, grid_for(Ll, Q.total_units), threads, Q, s);
                 if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx");
@@ -247,10 +252,12 @@ template <typename XT>
 qf_status launch_format_t(qf_format f, int mode, const std::vector<DevTensor>& v,
                           const float* am, float* so, int ng, cudaStream_t s) {
     if (f == QF_NVFP4) {
+        // the fused pass usually follows the tie-group amax pass over the same tensors:
+        // from the last unit down, its first reads are still in L2
         if (mode == 0)
             return launch_chunks(nv_block_kernel<XT, kSmallT>(), nv_block_kernel<XT, kLargeT>(),
                                  QF_NVB_THREADS, QF_NVB_WAVES, v, 512 * nvb_u<XT>(), am, so, nullptr,
-                                 ng, s);
+                                 ng, s, false, QF_NV_REVERSE);
         return launch_chunks(qf::k_nv_ste<XT, nvb_u<XT>(), kSmallT, QF_NVB_THREADS>,
                              qf::k_nv_ste<XT, nvb_u<XT>(), kLargeT, QF_NVB_THREADS>,
                              QF_NVB_THREADS, QF_NVB_WAVES, v, 512 * nvb_u<XT>(), am, nullptr,
@@ -711,7 +718,7 @@ qf_status qf_amax_fakequant_lora(const qf_tensor* t, const qf_lora* l, int n,
                          qf::k_nv<uint16_t, nvb_u<uint16_t>(), kLargeT, QF_NVB_THREADS,
                                   QF_NVB_PREFETCH, 3>,
                          QF_NVB_THREADS, QF_NVB_WAVES, w, 512 * nvb_u<uint16_t>(), d_group_amax,
-                         d_group_scale_out, nullptr, n_groups, s);
+                         d_group_scale_out, nullptr, n_groups, s, false, QF_NV_REVERSE);
 }
 
 qf_status qf_amax_tied(const qf_tensor* t, int n, float* d_group_amax, int n_groups,
@@ -821,13 +828,13 @@ qf_status qf_amax_fakequant(const qf_tensor* t, int n, float* d_group_amax, int 
                              qf::k_nv<float, nvb_u<float>(), kLargeT, QF_NVB_THREADS,
                                       QF_NVB_PREFETCH, QF_FP4_LD, true>,
                              QF_NVB_THREADS, QF_NVB_WAVES, v, 512 * nvb_u<float>(), am,
-                             d_group_scale_out, nullptr, n_groups, s, true);
+                             d_group_scale_out, nullptr, n_groups, s, true, QF_NV_REVERSE);
     return launch_chunks(qf::k_nv<uint16_t, nvb_u<uint16_t>(), kSmallT, QF_NVB_THREADS,
                                   QF_NVB_PREFETCH, QF_FP4_LD, true>,
                          qf::k_nv<uint16_t, nvb_u<uint16_t>(), kLargeT, QF_NVB_THREADS,
                                   QF_NVB_PREFETCH, QF_FP4_LD, true>,
                          QF_NVB_THREADS, QF_NVB_WAVES, v, 512 * nvb_u<uint16_t>(), am,
-                         d_group_scale_out, nullptr, n_groups, s, true);
+                         d_group_scale_out, nullptr, n_groups, s, true, QF_NV_REVERSE);
 }
 
 qf_status qf_amax_fakequant_noalloc(const qf_tensor* t, int n, float* d_group_amax,

@@ -68,6 +68,9 @@
 #ifndef QF_Q4K_WAVES
 #define QF_Q4K_WAVES 1
 #endif
+#ifndef QF_Q4K_PREFETCH
+#define QF_Q4K_PREFETCH 0       // 1: register prefetch of each warp's next unit (BF16 input)
+#endif
 #ifndef QF_Q4K_MINB
 #define QF_Q4K_MINB 0           // > 0: minimum resident CTAs per SM asked of the register allocator
 #endif
@@ -120,6 +123,7 @@ struct Table {
     float* tracked;             // qf_amax_tied running amax (nullable)
     int32_t n;
     int32_t n_groups;
+    int32_t reverse;            // k_nv: visit the units from the last one down (see there)
 };
 
 // ------------------------------------------------------------------ PTX helpers
@@ -567,6 +571,12 @@ __device__ __forceinline__ void nv_encode_unit(const DevTensor& T, int64_t e0, i
 // x is loaded before griddepcontrol.wait -- x was final before the amax kernel
 // started -- and the group amax is read only after it, so the loads of this grid's
 // first wave overlap the end of the amax grid.
+//
+// P.reverse: the warps take the units from the last one down.  A pass that follows one
+// over the same data (the tie-group amax, or the merge that wrote x) ends with its last
+// units' lines in L2, so the first units this grid reads come from L2, and lines it
+// overwrites in place need not be written back first.  The results do not depend on the
+// order.
 template <typename XT, int U, int MAXT, int THREADS, int PREFETCH, int LD = QF_FP4_LD,
           bool DEP_AMAX = false>
 __global__ void __launch_bounds__(THREADS) k_nv(const __grid_constant__ Table<MAXT> P) {
@@ -574,12 +584,16 @@ __global__ void __launch_bounds__(THREADS) k_nv(const __grid_constant__ Table<MA
     const int64_t warp = (int64_t(blockIdx.x) * THREADS + threadIdx.x) >> 5;
     const int64_t nwarps = (int64_t(gridDim.x) * THREADS) >> 5;
     constexpr int kUnit = 512 * U;
+    const bool rev = P.reverse != 0;
+    // the unit a warp's logical index stands for, and the tensor that owns it
+    auto phys = [&](int64_t lu) { return rev ? P.total_units - 1 - lu : lu; };
+    auto owner = [&](int hint, int64_t pu) { return rev ? locate_tensor(P, pu) : find_tensor(P, hint, pu); };
     int64_t u = warp;
     int ti = 0;
     Elems<XT, 16> cur[U], nxt[U];
     if (u < P.total_units) {
-        ti = locate_tensor(P, u);
-        nv_load_unit<XT, U, LD>(P.t[ti], (u - P.t[ti].unit_begin) * kUnit, lane, cur);
+        ti = locate_tensor(P, phys(u));
+        nv_load_unit<XT, U, LD>(P.t[ti], (phys(u) - P.t[ti].unit_begin) * kUnit, lane, cur);
     }
     if (DEP_AMAX) asm volatile("griddepcontrol.wait;" ::: "memory");
     if (blockIdx.x == 0 && P.group_scale_out) {
@@ -593,8 +607,8 @@ __global__ void __launch_bounds__(THREADS) k_nv(const __grid_constant__ Table<MA
         const int64_t un = u + nwarps;
         int tn = ti;
         if (PREFETCH && un < P.total_units) {
-            tn = find_tensor(P, ti, un);
-            nv_load_unit<XT, U, LD>(P.t[tn], (un - P.t[tn].unit_begin) * kUnit, lane, nxt);
+            tn = owner(ti, phys(un));
+            nv_load_unit<XT, U, LD>(P.t[tn], (phys(un) - P.t[tn].unit_begin) * kUnit, lane, nxt);
         }
         const DevTensor& T = P.t[ti];
         if (ti != cur_t) {
@@ -602,7 +616,7 @@ __global__ void __launch_bounds__(THREADS) k_nv(const __grid_constant__ Table<MA
             six_st = __fmul_rn(6.0f, s_t);
             cur_t = ti;
         }
-        nv_encode_unit<XT, U>(T, (u - T.unit_begin) * kUnit, lane, cur, s_t, six_st);
+        nv_encode_unit<XT, U>(T, (phys(u) - T.unit_begin) * kUnit, lane, cur, s_t, six_st);
         if (un >= P.total_units) break;
         u = un;
         if (PREFETCH) {
@@ -610,8 +624,8 @@ __global__ void __launch_bounds__(THREADS) k_nv(const __grid_constant__ Table<MA
 #pragma unroll
             for (int i = 0; i < U; ++i) cur[i] = nxt[i];
         } else {
-            ti = find_tensor(P, ti, u);
-            nv_load_unit<XT, U, LD>(P.t[ti], (u - P.t[ti].unit_begin) * kUnit, lane, cur);
+            ti = owner(ti, phys(u));
+            nv_load_unit<XT, U, LD>(P.t[ti], (phys(u) - P.t[ti].unit_begin) * kUnit, lane, cur);
         }
     }
 }
@@ -898,6 +912,21 @@ __global__ void QF_Q4K_BOUNDS(THREADS) k_q4k(const __grid_constant__ Table<MAXT>
     const int64_t warp = (int64_t(blockIdx.x) * THREADS + threadIdx.x) >> 5;
     const int64_t nwarps = (int64_t(gridDim.x) * THREADS) >> 5;
     int ti = warp < P.total_units ? locate_tensor(P, warp) : 0;
+    // QF_Q4K_PREFETCH (BF16 input): the next unit's loads are issued before this unit is
+    // encoded, so each warp keeps two units' loads in flight
+    constexpr bool kPf = QF_Q4K_PREFETCH && kBf16;
+    uint4 vn[4];
+    auto load_raw = [&](int64_t u, int t, uint4 (&v)[4]) {
+        const DevTensor& T = P.t[t];
+        const int64_t e0 = (u - T.unit_begin) * 1024;
+        const int64_t left = (T.numel - e0) >> 8;
+        const int nsb = left < 4 ? (int)left : 4;
+        const XT* xp = static_cast<const XT*>(T.x);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            v[k] = k < nsb ? ld_stream<0>(xp + e0 + 256 * k + 8 * lane) : make_uint4(0, 0, 0, 0);
+    };
+    if (kPf && warp < P.total_units) load_raw(warp, ti, vn);
     for (int64_t u = warp; u < P.total_units; u += nwarps) {
         ti = find_tensor(P, ti, u);
         const DevTensor& T = P.t[ti];
@@ -909,9 +938,16 @@ __global__ void QF_Q4K_BOUNDS(THREADS) k_q4k(const __grid_constant__ Table<MAXT>
         Elems<XT, 32> x;
         if constexpr (kBf16) {
             uint4 v[4];
+            if constexpr (kPf) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-                v[k] = k < nsb ? ld_stream<0>(xp + e0 + 256 * k + 8 * lane) : make_uint4(0, 0, 0, 0);
+                for (int k = 0; k < 4; ++k) v[k] = vn[k];
+                const int64_t un = u + nwarps;
+                if (un < P.total_units) load_raw(un, find_tensor(P, ti, un), vn);
+            } else {
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    v[k] = k < nsb ? ld_stream<0>(xp + e0 + 256 * k + 8 * lane) : make_uint4(0, 0, 0, 0);
+            }
             __syncwarp();
 #pragma unroll
             for (int k = 0; k < 4; ++k) sts128(sm_lane + k * kQ4kRow, v[k]);

@@ -54,6 +54,12 @@ constexpr int kLoraCols = kLoraThreads / 32 * 128;   // columns per CTA unit (12
 #ifndef QF_LORA_PF
 #define QF_LORA_PF 4            // with register prefetch: L2 prefetch distance, 4-row steps
 #endif
+#ifndef QF_LORA_PIPE
+#define QF_LORA_PIPE 1          // merge modes: the software-pipelined 2-row loop (unit_pipe)
+#endif
+#ifndef QF_LORA_FUSED
+#define QF_LORA_FUSED 1         // pipelined merge: one fused rounding where scale = 2^e, e >= 0
+#endif
 #ifndef QF_LORA_FULL
 #define QF_LORA_FULL 1          // guard-free copy of the unit loop for whole tiles: 0 none,
 #endif                          // 1 merge / amax modes, 2 every mode
@@ -135,7 +141,7 @@ struct FullTile { static constexpr bool value = B; };
 // R: compile-time rank capacity (the runtime rank is <= R; A and B are zero-padded,
 // which adds exact zeros to an accumulator that is never -0, so results do not change).
 template <int MODE, int R, int MAXT>
-__global__ void __launch_bounds__(kLoraThreads) k_lora(const __grid_constant__ LoraTable<MAXT> P) {
+__global__ void __launch_bounds__(kLoraThreads, R <= 16 ? 2 : 1) k_lora(const __grid_constant__ LoraTable<MAXT> P) {
     __shared__ __align__(16) uint64_t bsm[kLoraRows][R];     // (b, b) FP32 pairs
     // W ring: every lane copies its own 8 bytes of each row into its own slots and reads
     // only those back, so the ring needs no barrier (48 KB of static shared memory caps
@@ -361,10 +367,139 @@ __global__ void __launch_bounds__(kLoraThreads) k_lora(const __grid_constant__ L
         }
         if constexpr (kStages > 0) cp_async_wait<0>();
     };
+    // Merge modes, software-pipelined over 2-row steps: each iteration forms the rank-r
+    // products of the next two rows while it finishes the current two (merge with W,
+    // BF16 rounding, store, max), so within every warp the FMA pipe's work and the rest
+    // interleave instead of alternating in bursts.  W comes through the same per-lane
+    // cp.async ring, viewed as 2-row stages (twice as many).
+    auto unit_pipe = [&](auto tag, auto ftag) {
+        constexpr bool FULL = decltype(tag)::value;
+        constexpr bool FUSED = decltype(ftag)::value;   // W + scale * acc in one rounding
+        const uint64_t s2 = pk2(scale, scale);
+        constexpr int kS = 2 * kRing;                   // ring depth in 2-row steps
+        const int n = FULL ? kLoraRows : nrows;
+        const int nst = (n + 1) >> 1;
+        auto row = [&](int i) { return FULL ? i : min(i, n - 1); };
+        const uint32_t ring = (uint32_t)__cvta_generic_to_shared(&wring[0][0][threadIdx.x]);
+        auto issue = [&](int st) {
+            if (st < nst) {
+                const uint32_t dst = ring + (uint32_t)((st % kS) * 2 * kLoraThreads * 8);
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+                    cp_async8(dst + h * kLoraThreads * 8,
+                              (FULL || colok) ? (const void*)(wbase + row(2 * st + h) * cols)
+                                              : (const void*)T.w,
+                              (FULL || colok) ? 8u : 0u);
+            }
+            cp_async_commit();
+        };
+        auto chains = [&](int st, uint64_t (&acc)[2][2]) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int i = row(2 * st + h);
+                acc[h][0] = 0;
+                acc[h][1] = 0;
+#pragma unroll
+                for (int k = 0; k < R; k += 2) {
+                    const ulonglong2 bk = *reinterpret_cast<const ulonglong2*>(&bsm[i][k]);
+                    acc[h][0] = fma2_pk(bk.x, a[k][0], acc[h][0]);
+                    acc[h][1] = fma2_pk(bk.x, a[k][1], acc[h][1]);
+                    acc[h][0] = fma2_pk(bk.y, a[k + 1][0], acc[h][0]);
+                    acc[h][1] = fma2_pk(bk.y, a[k + 1][1], acc[h][1]);
+                }
+            }
+        };
+        uint16_t* yrow = kWritesMerged ? T.y + r0 * cols + col0 : nullptr;
+        // one step: the next rows' products into nxt, this step's rows finished from cur
+        auto step = [&](int st, uint64_t (&cur)[2][2], uint64_t (&nxt)[2][2]) {
+            cp_async_wait<kS - 2>();                    // this step's W has landed
+            const uint32_t src = ring + (uint32_t)((st % kS) * 2 * kLoraThreads * 8);
+            const uint2 w[2] = {lds64(src), lds64(src + kLoraThreads * 8)};
+            issue(st + kS - 1);                         // refills the stage read last step
+            if (st + 1 < nst) chains(st + 1, nxt);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t x0, x1;
+                if constexpr (FUSED) {
+                    // scale * acc is exact here (see kFusedMerge), so one fused rounding of
+                    // W + scale * acc equals the rounded product followed by the rounded add
+                    const float2 m01 = unpk2(fma2_pk(s2, cur[h][0],
+                                                     pk2(bf16_lo(w[h].x), bf16_hi(w[h].x))));
+                    const float2 m23 = unpk2(fma2_pk(s2, cur[h][1],
+                                                     pk2(bf16_lo(w[h].y), bf16_hi(w[h].y))));
+                    x0 = cvt_bf16x2(m01.y, m01.x);
+                    x1 = cvt_bf16x2(m23.y, m23.x);
+                } else {
+                    // scalar: a paired product must not feed an add (see mul2_rn)
+                    const float2 s01 = unpk2(cur[h][0]), s23 = unpk2(cur[h][1]);
+                    x0 = cvt_bf16x2(__fadd_rn(bf16_hi(w[h].x), __fmul_rn(scale, s01.y)),
+                                    __fadd_rn(bf16_lo(w[h].x), __fmul_rn(scale, s01.x)));
+                    x1 = cvt_bf16x2(__fadd_rn(bf16_hi(w[h].y), __fmul_rn(scale, s23.y)),
+                                    __fadd_rn(bf16_lo(w[h].y), __fmul_rn(scale, s23.x)));
+                }
+                if (kWritesMerged && (FULL || (colok && 2 * st + h < n)))
+                    *reinterpret_cast<uint2*>(yrow + h * cols) = make_uint2(x0, x1);
+                if (kFoldsAmax)
+                    run = max_u16x2(run, max_u16x2(x0 & 0x7FFF7FFFu, x1 & 0x7FFF7FFFu));
+            }
+            if (kWritesMerged) yrow += 2 * cols;
+        };
+#pragma unroll
+        for (int st = 0; st < kS - 1; ++st) issue(st);
+        uint64_t accA[2][2], accB[2][2];
+        chains(0, accA);
+#pragma unroll 1
+        for (int st = 0; st < nst; st += 2) {           // two steps per pass: the
+            step(st, accA, accB);                       // accumulators swap roles
+            if (st + 1 < nst) step(st + 1, accB, accA);
+        }
+        cp_async_wait<0>();
+    };
     constexpr bool kSplitFull = QF_LORA_FULL == 2 || (QF_LORA_FULL == 1 && MODE != kLoraNV &&
                                                       MODE != kLoraMX);
-    if (kSplitFull && nrows == kLoraRows && colok) unit(FullTile<true>{});
-    else unit(FullTile<false>{});
+    constexpr bool kPipe = QF_LORA_PIPE && kStages > 0 && (MODE == kLoraMerge ||
+                                                            MODE == kLoraMergeAmax);
+    if constexpr (kPipe) {
+        // kFusedMerge: with scale = 2^e, e >= 0, scale * acc is exact unless it overflows;
+        // |acc| <= sum_k |b_k| |a_k| (1 + 2^-20) <= Rmax Cmax (1 + 2^-20) over the CTA's
+        // rows and columns, so scale Rmax Cmax (1 + 2^-6) < 2^126 rules the overflow out
+        // and the merge may round W + scale * acc once (a paired FMA per two elements)
+        __shared__ uint32_t s_rmax, s_cmax;
+        if (threadIdx.x == 0) s_rmax = s_cmax = 0u;
+        __syncthreads();
+        if (threadIdx.x < kLoraRows) {
+            float r = 0.0f;
+#pragma unroll
+            for (int k = 0; k < R; ++k) r = __fadd_rn(r, fabsf(unpk2(bsm[threadIdx.x][k]).x));
+            atomicMax(&s_rmax, __float_as_uint(r));
+        }
+        uint32_t cm = 0;
+#pragma unroll
+        for (int k = 0; k < R; ++k) {
+            const float2 p = unpk2(a[k][0]), q = unpk2(a[k][1]);
+            cm = max(cm, max(max(__float_as_uint(p.x), __float_as_uint(p.y)),
+                             max(__float_as_uint(q.x), __float_as_uint(q.y))) & 0x7FFFFFFFu);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) cm = max(cm, __shfl_xor_sync(kFull, cm, o));
+        if (lane == 0) atomicMax(&s_cmax, cm);
+        __syncthreads();
+        const uint32_t sb = __float_as_uint(scale);
+        const bool pow2 = (sb & 0x807FFFFFu) == 0u && (sb >> 23) >= 127u && (sb >> 23) < 255u;
+        const float bound = __fmul_rn(__fmul_rn(__fmul_rn(scale, __uint_as_float(s_rmax)),
+                                                __uint_as_float(s_cmax)), 1.0f + 0x1p-6f);
+        const bool fused = QF_LORA_FUSED && pow2 && bound < 0x1p126f;
+        if (nrows == kLoraRows && colok) {
+            if (fused) unit_pipe(FullTile<true>{}, FullTile<true>{});
+            else unit_pipe(FullTile<true>{}, FullTile<false>{});
+        } else {
+            if (fused) unit_pipe(FullTile<false>{}, FullTile<true>{});
+            else unit_pipe(FullTile<false>{}, FullTile<false>{});
+        }
+    } else {
+        if (kSplitFull && nrows == kLoraRows && colok) unit(FullTile<true>{});
+        else unit(FullTile<false>{});
+    }
 
     if (kFoldsAmax) {
         // one atomic per CTA (its unit lies in one tensor), not one per warp

@@ -57,6 +57,114 @@ __device__ __forceinline__ uint32_t ld_relaxed_gpu(const uint32_t* p) {
     return v;
 }
 
+// ---- the parts both one-launch kernels share
+
+// A sticky error left by an earlier call on this workspace: the CTA does no work.
+__device__ __forceinline__ bool oneshot_skip(const uint32_t* ws) {
+    __shared__ int s_skip;
+    if (threadIdx.x == 0) s_skip = ld_relaxed_gpu(ws + kOneshotErrWord) != 0u;
+    __syncthreads();
+    const bool skip = s_skip;
+    __syncthreads();
+    return skip;
+}
+
+// Combine the warps' last (group, max) pairs in the CTA; one atomicMax per CTA and group.
+template <int THREADS>
+__device__ __forceinline__ void oneshot_fold(uint32_t* slot, int g, uint32_t a) {
+    constexpr int kWarps = THREADS / 32;
+    __shared__ int wgrp[kWarps];
+    __shared__ uint32_t wmax[kWarps];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    if (lane == 0) {
+        wgrp[wid] = g;
+        wmax[wid] = a;
+    }
+    __syncthreads();
+    if (threadIdx.x < kWarps) {
+        const int w = threadIdx.x, gw = wgrp[w];
+        bool first = gw >= 0;
+        uint32_t m = wmax[w];
+        for (int o = 0; o < kWarps; ++o) {
+            if (wgrp[o] != gw) continue;
+            if (o < w) first = false;
+            m = max(m, wmax[o]);
+        }
+        if (first) atomicMax(slot + gw, m);
+    }
+    __syncthreads();
+}
+
+// The bounded grid barrier; returns whether this CTA may go on to phase 2.
+__device__ __forceinline__ bool oneshot_barrier(uint32_t* ws, bool skip, uint32_t test_polls) {
+    __shared__ int s_go;
+    if (threadIdx.x == 0) {
+        __threadfence();                                    // this CTA's slot updates first
+        atomicAdd(ws + kOneshotArriveWord, 1u);
+        bool done = false;
+        if (!skip) {
+            const uint32_t target = gridDim.x + (test_polls ? 1u : 0u);
+            const uint32_t limit = test_polls ? test_polls : kOneshotSpinLimit;
+            uint32_t polls = 0;
+            done = ld_acquire_gpu(ws + kOneshotArriveWord) >= target;
+            while (!done && ++polls < limit) {
+                __nanosleep(256);
+                done = ld_acquire_gpu(ws + kOneshotArriveWord) >= target;
+            }
+            if (!done) atomicOr(ws + kOneshotErrWord, kOneshotErrTimeout);
+        }
+        s_go = done;
+    }
+    __syncthreads();
+    return s_go;
+}
+
+// The effective amax of a group: this call's max, folded with the running value when
+// one is kept (FP32 bit patterns as unsigned integers, as k_amax folds them).
+template <int MAXT>
+__device__ __forceinline__ float oneshot_eff_amax(const Table<MAXT>& P, const uint32_t* slot,
+                                                  int grp) {
+    uint32_t a = ld_relaxed_gpu(slot + grp);
+    if (P.tracked) a = max(a, __float_as_uint(P.tracked[grp]));
+    return __uint_as_float(a);
+}
+
+// CTA 0 writes the group statistics: this call's amax, the running amax, s_t.
+template <int MAXT, int THREADS>
+__device__ __forceinline__ void oneshot_stats(const Table<MAXT>& P, const uint32_t* slot) {
+    if (blockIdx.x != 0) return;
+    for (int q = threadIdx.x; q < P.n_groups; q += THREADS) {
+        const float cur = __uint_as_float(ld_relaxed_gpu(slot + q));
+        const float e = oneshot_eff_amax(P, slot, q);
+        const_cast<float*>(P.group_amax)[q] = cur;
+        if (P.tracked) P.tracked[q] = e;
+        if (P.group_scale_out) P.group_scale_out[q] = nv_tensor_scale(e);
+    }
+}
+
+// Every CTA departs, whether it passed the barrier or gave up; the last one out leaves
+// the slots and counters zeroed for the next call.
+template <int THREADS>
+__device__ __forceinline__ void oneshot_depart(uint32_t* ws, int n_groups) {
+    __shared__ int s_last;
+    uint32_t* slot = ws + kOneshotHeaderWords;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        s_last = atomicAdd(ws + kOneshotDepartWord, 1u) == gridDim.x - 1;
+    }
+    __syncthreads();
+    if (s_last) {
+        __threadfence();
+        for (int q = threadIdx.x; q < n_groups; q += THREADS) slot[q] = 0u;
+        if (threadIdx.x == 0) {
+            ws[kOneshotArriveWord] = 0u;
+            ws[kOneshotDepartWord] = 0u;
+        }
+    }
+}
+
+// ---- k_nv_oneshot: the second pass re-reads x from L2
 // P.group_amax: output, this call's tie-group amax.  P.tracked (nullable): running
 // amax, max-accumulated in place; when given, s_t comes from the updated running
 // value (the activation reading), otherwise from this call's amax.
@@ -74,13 +182,7 @@ __global__ void __launch_bounds__(THREADS, QF_ONESHOT_MINB)
     const int64_t warp = int64_t(blockIdx.x) * kWarps + wid;
     const int64_t nwarps = int64_t(gridDim.x) * kWarps;
     uint32_t* slot = ws + kOneshotHeaderWords;
-    __shared__ int s_flag;
-
-    // a sticky error left by an earlier call: do nothing, so the caller's check sees it
-    if (threadIdx.x == 0) s_flag = ld_relaxed_gpu(ws + kOneshotErrWord) != 0u;
-    __syncthreads();
-    const bool skip = s_flag;
-    __syncthreads();
+    const bool skip = oneshot_skip(ws);
 
     // ---- phase 1: max |x| per tie group over this warp's units
     int ti = warp < P.total_units && !skip ? locate_tensor(P, warp) : 0;
@@ -106,65 +208,10 @@ __global__ void __launch_bounds__(THREADS, QF_ONESHOT_MINB)
 #pragma unroll
         for (int s = 0; s < U; ++s) run = max(run, v[s].amax_bits());
     }
-    __shared__ int wgrp[kWarps];
-    __shared__ uint32_t wmax[kWarps];
-    {
-        const uint32_t a = warp_max();
-        if (lane == 0) {
-            wgrp[wid] = g;
-            wmax[wid] = a;
-        }
-    }
-    __syncthreads();
-    if (threadIdx.x < kWarps) {
-        const int w = threadIdx.x, gw = wgrp[w];
-        bool first = gw >= 0;
-        uint32_t m = wmax[w];
-        for (int o = 0; o < kWarps; ++o) {
-            if (wgrp[o] != gw) continue;
-            if (o < w) first = false;
-            m = max(m, wmax[o]);
-        }
-        if (first) atomicMax(slot + gw, m);
-    }
-    __syncthreads();
+    oneshot_fold<THREADS>(slot, g, warp_max());
 
-    // ---- grid barrier (bounded)
-    if (threadIdx.x == 0) {
-        __threadfence();                                    // this CTA's slot updates first
-        atomicAdd(ws + kOneshotArriveWord, 1u);
-        bool done = false;
-        if (!skip) {
-            const uint32_t target = gridDim.x + (test_polls ? 1u : 0u);
-            const uint32_t limit = test_polls ? test_polls : kOneshotSpinLimit;
-            uint32_t polls = 0;
-            done = ld_acquire_gpu(ws + kOneshotArriveWord) >= target;
-            while (!done && ++polls < limit) {
-                __nanosleep(256);
-                done = ld_acquire_gpu(ws + kOneshotArriveWord) >= target;
-            }
-            if (!done) atomicOr(ws + kOneshotErrWord, kOneshotErrTimeout);
-        }
-        s_flag = done;
-    }
-    __syncthreads();
-    const bool go = s_flag;                                 // false: outputs left unwritten
-
-    // ---- group statistics out (CTA 0)
-    auto eff_amax = [&](int grp) {
-        uint32_t a = ld_relaxed_gpu(slot + grp);
-        if (P.tracked) a = max(a, __float_as_uint(P.tracked[grp]));
-        return __uint_as_float(a);
-    };
-    if (go && blockIdx.x == 0) {
-        for (int q = threadIdx.x; q < P.n_groups; q += THREADS) {
-            const float cur = __uint_as_float(ld_relaxed_gpu(slot + q));
-            const float e = eff_amax(q);
-            const_cast<float*>(P.group_amax)[q] = cur;
-            if (P.tracked) P.tracked[q] = e;
-            if (P.group_scale_out) P.group_scale_out[q] = nv_tensor_scale(e);
-        }
-    }
+    const bool go = oneshot_barrier(ws, skip, test_polls);   // false: outputs left unwritten
+    if (go) oneshot_stats<MAXT, THREADS>(P, slot);
 
     // ---- phase 2: encode the same units (their lines are in L2 now)
     if (go && warp < P.total_units) {
@@ -175,7 +222,7 @@ __global__ void __launch_bounds__(THREADS, QF_ONESHOT_MINB)
             ti = find_tensor(P, ti, u);
             const DevTensor& T = P.t[ti];
             if (ti != cur_t) {
-                s_t = nv_tensor_scale(eff_amax(T.group));
+                s_t = nv_tensor_scale(oneshot_eff_amax(P, slot, T.group));
                 six_st = __fmul_rn(6.0f, s_t);
                 cur_t = ti;
             }
@@ -185,23 +232,7 @@ __global__ void __launch_bounds__(THREADS, QF_ONESHOT_MINB)
             nv_encode_unit<XT, U>(T, e0, lane, v, s_t, six_st);
         }
     }
-
-    // ---- depart (every CTA, whether it passed the barrier or gave up); the last CTA
-    // out leaves the slots and counters zeroed for the next call
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        s_flag = atomicAdd(ws + kOneshotDepartWord, 1u) == gridDim.x - 1;
-    }
-    __syncthreads();
-    if (s_flag) {
-        __threadfence();
-        for (int q = threadIdx.x; q < P.n_groups; q += THREADS) slot[q] = 0u;
-        if (threadIdx.x == 0) {
-            ws[kOneshotArriveWord] = 0u;
-            ws[kOneshotDepartWord] = 0u;
-        }
-    }
+    oneshot_depart<THREADS>(ws, P.n_groups);
 }
 
 }  // namespace qf

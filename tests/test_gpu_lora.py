@@ -310,3 +310,35 @@ def test_merged_amax_many_tensors_and_groups():
             ads.append((b, a, 2.0))
             groups.append(2 * e + (j == 2))
     _amax_case(ts, ads, groups, 8)
+
+
+@pytest.mark.parametrize("case", ["pow2_1", "pow2_8", "half", "pow2_overflow_guard", "odd"])
+def test_merge_paths_for_scale_kinds(case):
+    """The merge rounds W + scale * acc once when scale is a power of two >= 1 and a bound
+    rules out overflow, else as a rounded product and a rounded add; both must give the
+    oracle's bytes.  In the guard case (adapters scaled by 1e5, scale 2^100) the bound on
+    scale * acc exceeds 2^126, so the two-rounding path must run, while the values stay
+    finite (about 5e37 at most)."""
+    rows, cols, r = 130, 2048, 16
+    w, b, a = _case(rows, cols, r, 900)
+    scale = {"pow2_1": 1.0, "pow2_8": 8.0, "half": 0.5, "pow2_overflow_guard": 2.0 ** 100,
+             "odd": 3.0}[case]
+    if case == "pow2_overflow_guard":
+        b = (b.float() * 1e5).to(torch.bfloat16)
+        a = (a.float() * 1e5).to(torch.bfloat16)
+    merged = oracle.lora_merge(w, b, a, scale)
+    wd = w.to(DEV)
+    ad = [(b.to(DEV), a.to(DEV), scale)]
+    m = torch.empty_like(wd)
+    qf.qf_lora_merge([wd], ad, [m])
+    yo, co, so = qf.alloc_outputs("nvfp4", wd)
+    amax = torch.empty(1, device=DEV)
+    qf.qf_amax_fakequant_lora([wd], ad, [yo], [co], [so], [0], amax)
+    torch.cuda.synchronize()
+    assert np.isfinite(oracle.bf16_to_f32(merged)).all()
+    assert_same(f"{case} merge", bits(m), merged)
+    am = np.float32(oracle.amax(merged))
+    assert_same(f"{case} amax", amax.cpu().numpy().view(np.uint32), np.float32([am]).view(np.uint32))
+    y, c, s, _ = oracle.nvfp4(merged, am)
+    assert_same(f"{case} y", bits(yo), y)
+    assert_same(f"{case} codes", u8(co), c)

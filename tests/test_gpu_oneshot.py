@@ -75,6 +75,16 @@ def test_tied_groups_small(dtype):
     _check_oracle(wl["tensors"], wl["groups"], wl["n_groups"], res, label=f"tied {dtype}")
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_near_the_l2_limit(dtype):
+    """Inputs close to the single-launch limit of L2 / 3 (BF16: 1/7 of the tied
+    projections, 40.7 MB; FP32: 1/14, also 40.7 MB)."""
+    wl = workloads.nvfp4_tied(rows_scale=1 / 7 if dtype == "bf16" else 1 / 14, with_grads=False,
+                              dtype=dtype)
+    res = _run(wl["tensors"], wl["groups"], wl["n_groups"])
+    _check_oracle(wl["tensors"], wl["groups"], wl["n_groups"], res, label=f"tied {dtype}")
+
+
 @pytest.mark.parametrize("scale", [0.5, 4.0])
 def test_tracked_amax(scale):
     """Activations: s_t comes from max(tracked, amax), and tracked is updated in place."""
@@ -173,7 +183,8 @@ def _untouched(outs, amax, so, label):
     assert bool(torch.isnan(amax).all()) and bool(torch.isnan(so).all()), f"{label}: amax / s_t written"
 
 
-def test_barrier_timeout_is_reported_and_recovers():
+@pytest.mark.parametrize("rows_scale", [1 / 16, 1 / 7])
+def test_barrier_timeout_is_reported_and_recovers(rows_scale):
     """The bounded grid barrier runs out with every CTA present (the testing aid makes
     it wait for one CTA more than the grid holds, at most 1000 polls).  Expected: no
     output is written, the error flag is sticky (a second call on the workspace does
