@@ -241,11 +241,13 @@ template <typename XT, int MAXT, int MODE>
 constexpr auto mx_kernel() {
     return qf::k_fp4<false, XT, kFp4U, MAXT, MODE, QF_MX_THREADS, QF_MX_PREFETCH>;
 }
-template <typename XT>
-constexpr int q4k_threads() { return sizeof(XT) == 2 ? QF_Q4K_THREADS : QF_Q4K_F32_THREADS; }
+template <typename XT, bool MSE = false>
+constexpr int q4k_threads() {
+    return sizeof(XT) == 2 ? (MSE ? QF_Q4K_MSE_THREADS : QF_Q4K_THREADS) : QF_Q4K_F32_THREADS;
+}
 template <typename XT, int MAXT, int MODE, bool MSE>
 constexpr auto q4k_kernel() {
-    return qf::k_q4k<XT, MAXT, MODE, q4k_threads<XT>(), MSE>;
+    return qf::k_q4k<XT, MAXT, MODE, q4k_threads<XT, MSE>(), MSE>;
 }
 
 template <typename XT>
@@ -273,11 +275,11 @@ qf_status launch_format_t(qf_format f, int mode, const std::vector<DevTensor>& v
     if (f == QF_Q4K_MSE) {
         if (mode == 0)
             return launch_chunks(q4k_kernel<XT, kSmallT, 0, true>(),
-                                 q4k_kernel<XT, kLargeT, 0, true>(), q4k_threads<XT>(),
+                                 q4k_kernel<XT, kLargeT, 0, true>(), q4k_threads<XT, true>(),
                                  QF_Q4K_WAVES, v, 1024, nullptr, nullptr, nullptr, 0, s);
         return launch_chunks(q4k_kernel<XT, kSmallT, 1, true>(), q4k_kernel<XT, kLargeT, 1, true>(),
-                             q4k_threads<XT>(), QF_Q4K_WAVES, v, 1024, nullptr, nullptr, nullptr, 0,
-                             s);
+                             q4k_threads<XT, true>(), QF_Q4K_WAVES, v, 1024, nullptr, nullptr,
+                             nullptr, 0, s);
     }
     if (mode == 0)
         return launch_chunks(q4k_kernel<XT, kSmallT, 0, false>(),

@@ -68,6 +68,12 @@
 #ifndef QF_Q4K_WAVES
 #define QF_Q4K_WAVES 1
 #endif
+#ifndef QF_Q4K_MSE_HOIST
+#define QF_Q4K_MSE_HOIST 1      // MSE search: x + min_j formed once per sub-block, not per trial
+#endif
+#ifndef QF_Q4K_MSE_THREADS
+#define QF_Q4K_MSE_THREADS QF_Q4K_THREADS
+#endif
 #ifndef QF_Q4K_PREFETCH
 #define QF_Q4K_PREFETCH 0       // 1: register prefetch of each warp's next unit (BF16 input)
 #endif
@@ -725,15 +731,17 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
 // -(x - dq)).  x + min_j >= +0 always (min_j >= -min x), so with a finite reciprocal
 // the scaled value is >= +0 and only the upper clamp can act: LOWER = false drops the
 // lower one.  LOWER = true keeps it for a reciprocal that overflowed (0 * inf).
+// XM: the sub-block's x + min_j, formed once for all trials (QF_Q4K_MSE_HOIST), or NULL.
 template <typename XT, bool LOWER>
-__device__ __forceinline__ float2 q4k_sub_err2(const Elems<XT, 32>& x, float2 scale, float min_j) {
+__device__ __forceinline__ float2 q4k_sub_err2(const Elems<XT, 32>& x, float2 scale, float min_j,
+                                               const float* XM) {
     const float2 inv = make_float2(__frcp_rn(scale.x), __frcp_rn(scale.y));
     const float2 rnd = make_float2(kRound, kRound), nrnd = make_float2(-kRound, -kRound);
     float2 err = make_float2(0.0f, 0.0f);
 #pragma unroll
     for (int k = 0; k < 32; ++k) {
         const float xk = x.get(k);
-        const float xm = __fadd_rn(xk, min_j);
+        const float xm = QF_Q4K_MSE_HOIST ? XM[k] : __fadd_rn(xk, min_j);
         const float2 t = mul2_rn(make_float2(xm, xm), inv);
         const float2 c = LOWER ? make_float2(fminf(fmaxf(t.x, 0.0f), 15.0f), fminf(fmaxf(t.y, 0.0f), 15.0f))
                                : make_float2(fminf(t.x, 15.0f), fminf(t.y, 15.0f));
@@ -754,7 +762,10 @@ template <typename XT, bool LOWER>
 __device__ __forceinline__ float q4k_search_scale_t(const Elems<XT, 32>& x, float range,
                                                     float best, float s18, float min_j) {
     const float s14 = __fdiv_rn(range, 14.0f);
-    const float2 e0 = q4k_sub_err2<XT, LOWER>(x, make_float2(best, s14), min_j);
+    float xm[32];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) xm[k] = QF_Q4K_MSE_HOIST ? __fadd_rn(x.get(k), min_j) : 0.0f;
+    const float2 e0 = q4k_sub_err2<XT, LOWER>(x, make_float2(best, s14), min_j, xm);
     float best_err = e0.x;
     if (e0.y < best_err) {
         best_err = e0.y;
@@ -767,7 +778,7 @@ __device__ __forceinline__ float q4k_search_scale_t(const Elems<XT, 32>& x, floa
         const float na = p == 0 ? 14.5f : p == 1 ? 16.0f : p == 2 ? 17.0f : 18.0f;
         const float nb = p == 0 ? 15.5f : p == 1 ? 16.5f : p == 2 ? 17.5f : 18.0f;
         const float2 sc = make_float2(p == 3 ? s18 : __fdiv_rn(range, na), __fdiv_rn(range, nb));
-        const float2 err = q4k_sub_err2<XT, LOWER>(x, sc, min_j);
+        const float2 err = q4k_sub_err2<XT, LOWER>(x, sc, min_j, xm);
         if (err.x < best_err) {
             best_err = err.x;
             best = sc.x;
