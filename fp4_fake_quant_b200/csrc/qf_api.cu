@@ -365,16 +365,21 @@ qf_status lora_launch_r(const std::vector<qf::LoraTensor>& v, const float* am, f
             P.group_scale_out = sout;
             P.n_groups = ng;
         };
+        // merge modes up to rank 16: 8 columns per lane (k_lora8), same units
+        constexpr bool k8 = QF_LORA8 && R <= 16 && (MODE == qf::kLoraMerge ||
+                                                    MODE == qf::kLoraMergeAmax);
         if (cnt <= (size_t)kLoraSmallT) {
             qf::LoraTable<kLoraSmallT> P;
             fill(P);
-            qf::k_lora<MODE, R, kLoraSmallT>
-                <<<(unsigned)std::max<int64_t>(1, P.total_units), qf::kLoraThreads, 0, s>>>(P);
+            const unsigned grid = (unsigned)std::max<int64_t>(1, P.total_units);
+            if constexpr (k8) qf::k_lora8<MODE, R, kLoraSmallT><<<grid, qf::kLora8Threads, 0, s>>>(P);
+            else qf::k_lora<MODE, R, kLoraSmallT><<<grid, qf::kLoraThreads, 0, s>>>(P);
         } else {
             qf::LoraTable<kLoraLargeT> P;
             fill(P);
-            qf::k_lora<MODE, R, kLoraLargeT>
-                <<<(unsigned)std::max<int64_t>(1, P.total_units), qf::kLoraThreads, 0, s>>>(P);
+            const unsigned grid = (unsigned)std::max<int64_t>(1, P.total_units);
+            if constexpr (k8) qf::k_lora8<MODE, R, kLoraLargeT><<<grid, qf::kLora8Threads, 0, s>>>(P);
+            else qf::k_lora<MODE, R, kLoraLargeT><<<grid, qf::kLoraThreads, 0, s>>>(P);
         }
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "kernel launch");

@@ -519,6 +519,195 @@ __global__ void __launch_bounds__(kLoraThreads, R <= 16 ? 2 : 1) k_lora(const __
 }
 
 
+// ------------------------------------------------------------------ merge, 8 columns per lane
+// k_lora8: the merge modes (kLoraMerge, kLoraMergeAmax) for rank <= 16 with each lane
+// owning 8 consecutive columns (a 128-thread CTA still covers 1024 columns by
+// kLoraRows rows, the unit of k_lora).  Against 4 columns per lane, every broadcast
+// load of two (b, b) pairs feeds 8 paired FMAs instead of 4 and the per-row work is
+// shared by twice the elements; the A slab takes 128 registers per lane (R = 16).
+// Arithmetic, results and the fused-rounding rule are those of k_lora's merge.
+#ifndef QF_LORA8
+#define QF_LORA8 1
+#endif
+#ifndef QF_LORA8_STAGES
+#define QF_LORA8_STAGES 4       // W ring depth in 2-row steps (16 bytes per lane and row)
+#endif
+#ifndef QF_LORA8_MINB
+#define QF_LORA8_MINB 3
+#endif
+constexpr int kLora8Threads = 128;
+
+__device__ __forceinline__ void cp_async16_cg(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                 "r"(src_bytes) : "memory");
+}
+
+template <int MODE, int R, int MAXT>
+__global__ void __launch_bounds__(kLora8Threads, QF_LORA8_MINB)
+    k_lora8(const __grid_constant__ LoraTable<MAXT> P) {
+    static_assert(MODE == kLoraMerge || MODE == kLoraMergeAmax, "merge modes only");
+    static_assert(R <= 16, "the A slab of rank 32 does not fit in registers");
+    constexpr int kS = QF_LORA8_STAGES;
+    constexpr bool kWritesMerged = true;
+    constexpr bool kFoldsAmax = MODE == kLoraMergeAmax;
+    __shared__ __align__(16) uint64_t bsm[kLoraRows][R];                 // (b, b) FP32 pairs
+    __shared__ __align__(16) uint4 wring[kS][2][kLora8Threads];
+    __shared__ uint32_t s_rmax, s_cmax;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int64_t cu = blockIdx.x;
+    if (cu >= P.total_units) return;
+    const LoraTensor& T = P.t[lora_locate(P, cu)];
+    const int64_t local = cu - T.unit_begin;
+    const int64_t r0 = (local / T.col_groups) * kLoraRows;
+    const int64_t c_base = (local % T.col_groups) * kLoraCols;
+    const int64_t rows_left = T.rows - r0;
+    const int nrows = rows_left < kLoraRows ? (int)rows_left : kLoraRows;
+    const int64_t cols = T.cols;
+    const int64_t col0 = c_base + wid * 256 + lane * 8;
+    const bool colok = col0 < cols;            // cols % 16 == 0: 8 columns all in or all out
+    const int rank = T.rank;
+    const float scale = T.scale;
+
+    for (int idx = threadIdx.x; idx < kLoraRows * R; idx += kLora8Threads) {
+        const int i = idx / R, k = idx % R;
+        const float b = (i < nrows && k < rank) ? bf16_lo(T.b[(r0 + i) * rank + k]) : 0.0f;
+        bsm[i][k] = pk2(b, b);
+    }
+    // this lane's 8 columns of A as four FP32 pairs per k, zero-padded to R
+    uint64_t a[R][4];
+#pragma unroll
+    for (int k = 0; k < R; ++k) {
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (k < rank && colok) v = *reinterpret_cast<const uint4*>(T.a + k * cols + col0);
+        a[k][0] = pk2(bf16_lo(v.x), bf16_hi(v.x));
+        a[k][1] = pk2(bf16_lo(v.y), bf16_hi(v.y));
+        a[k][2] = pk2(bf16_lo(v.z), bf16_hi(v.z));
+        a[k][3] = pk2(bf16_lo(v.w), bf16_hi(v.w));
+    }
+    if (threadIdx.x == 0) s_rmax = s_cmax = 0u;
+    __syncthreads();
+    // the fused-rounding rule of k_lora (kFusedMerge): scale = 2^e, e >= 0, and
+    // scale * Rmax * Cmax * (1 + 2^-6) < 2^126 over the CTA's rows and columns
+    if (threadIdx.x < kLoraRows) {
+        float r = 0.0f;
+#pragma unroll
+        for (int k = 0; k < R; ++k) r = __fadd_rn(r, fabsf(unpk2(bsm[threadIdx.x][k]).x));
+        atomicMax(&s_rmax, __float_as_uint(r));
+    }
+    uint32_t cm = 0;
+#pragma unroll
+    for (int k = 0; k < R; ++k)
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const float2 q = unpk2(a[k][p]);
+            cm = max(cm, max(__float_as_uint(q.x), __float_as_uint(q.y)) & 0x7FFFFFFFu);
+        }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cm = max(cm, __shfl_xor_sync(kFull, cm, o));
+    if (lane == 0) atomicMax(&s_cmax, cm);
+    __syncthreads();
+    const uint32_t sbits = __float_as_uint(scale);
+    const bool pow2 = (sbits & 0x807FFFFFu) == 0u && (sbits >> 23) >= 127u && (sbits >> 23) < 255u;
+    const float bound = __fmul_rn(__fmul_rn(__fmul_rn(scale, __uint_as_float(s_rmax)),
+                                            __uint_as_float(s_cmax)), 1.0f + 0x1p-6f);
+    const bool fused = QF_LORA_FUSED && pow2 && bound < 0x1p126f;
+
+    uint32_t run = 0;
+    const uint16_t* wbase = T.w + r0 * cols + col0;
+    auto unit = [&](auto tag, auto ftag) {
+        constexpr bool FULL = decltype(tag)::value;
+        constexpr bool FUSED = decltype(ftag)::value;
+        const uint64_t s2 = pk2(scale, scale);
+        const int n = FULL ? kLoraRows : nrows;
+        const int nst = (n + 1) >> 1;
+        auto row = [&](int i) { return FULL ? i : min(i, n - 1); };
+        const uint32_t ring = (uint32_t)__cvta_generic_to_shared(&wring[0][0][threadIdx.x]);
+        auto issue = [&](int st) {
+            if (st < nst) {
+                const uint32_t dst = ring + (uint32_t)((st % kS) * 2 * kLora8Threads * 16);
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+                    cp_async16_cg(dst + h * kLora8Threads * 16,
+                                  (FULL || colok) ? (const void*)(wbase + row(2 * st + h) * cols)
+                                                  : (const void*)T.w,
+                                  (FULL || colok) ? 16u : 0u);
+            }
+            cp_async_commit();
+        };
+#pragma unroll
+        for (int st = 0; st < kS - 1; ++st) issue(st);
+        uint16_t* yrow = T.y + r0 * cols + col0;
+#pragma unroll 1
+        for (int st = 0; st < nst; ++st) {
+            cp_async_wait<kS - 2>();                        // this step's W has landed
+            const uint32_t src = ring + (uint32_t)((st % kS) * 2 * kLora8Threads * 16);
+            const uint4 w[2] = {lds128(src), lds128(src + kLora8Threads * 16)};
+            issue(st + kS - 1);                             // refills the stage read last step
+            uint64_t acc[2][4];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int i = row(2 * st + h);
+#pragma unroll
+                for (int p = 0; p < 4; ++p) acc[h][p] = 0;
+#pragma unroll
+                for (int k = 0; k < R; k += 2) {
+                    const ulonglong2 bk = *reinterpret_cast<const ulonglong2*>(&bsm[i][k]);
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) acc[h][p] = fma2_pk(bk.x, a[k][p], acc[h][p]);
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) acc[h][p] = fma2_pk(bk.y, a[k + 1][p], acc[h][p]);
+                }
+            }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t wv[4] = {w[h].x, w[h].y, w[h].z, w[h].w};
+                uint32_t xo[4];
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    if constexpr (FUSED) {
+                        const float2 m = unpk2(fma2_pk(s2, acc[h][p], pk2(bf16_lo(wv[p]), bf16_hi(wv[p]))));
+                        xo[p] = cvt_bf16x2(m.y, m.x);
+                    } else {
+                        // scalar: a paired product must not feed an add (see mul2_rn)
+                        const float2 sp = unpk2(acc[h][p]);
+                        xo[p] = cvt_bf16x2(__fadd_rn(bf16_hi(wv[p]), __fmul_rn(scale, sp.y)),
+                                           __fadd_rn(bf16_lo(wv[p]), __fmul_rn(scale, sp.x)));
+                    }
+                }
+                if (kWritesMerged && (FULL || (colok && 2 * st + h < n)))
+                    *reinterpret_cast<uint4*>(yrow + h * cols) = make_uint4(xo[0], xo[1], xo[2], xo[3]);
+                if (kFoldsAmax)
+                    run = max_u16x2(max_u16x2(run, max_u16x2(xo[0] & 0x7FFF7FFFu, xo[1] & 0x7FFF7FFFu)),
+                                    max_u16x2(xo[2] & 0x7FFF7FFFu, xo[3] & 0x7FFF7FFFu));
+            }
+            yrow += 2 * cols;
+        }
+        cp_async_wait<0>();
+    };
+    if (nrows == kLoraRows && colok) {
+        if (fused) unit(FullTile<true>{}, FullTile<true>{});
+        else unit(FullTile<true>{}, FullTile<false>{});
+    } else {
+        if (fused) unit(FullTile<false>{}, FullTile<true>{});
+        else unit(FullTile<false>{}, FullTile<false>{});
+    }
+
+    if (kFoldsAmax) {
+        __shared__ uint32_t wmax[kLora8Threads / 32];
+        run = bf16x2_max_bits(run);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) run = max(run, __shfl_xor_sync(kFull, run, o));
+        if (lane == 0) wmax[wid] = run;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            for (int w = 1; w < kLora8Threads / 32; ++w) run = max(run, wmax[w]);
+            if (run != 0)
+                atomicMax(reinterpret_cast<unsigned int*>(const_cast<float*>(P.group_amax)) + T.group,
+                          run);
+        }
+    }
+}
+
 // ------------------------------------------------------------------ merged-weight amax
 // k_lora_amax: the exact max |M| of a tie group's merged weights, M = BF16(W + s * acc),
 // with the rank-r merge evaluated only where it can decide the result.
