@@ -7,8 +7,9 @@ of channels x50 -- quantized in ONE grouped qf_fakequant launch that writes
 dequantized BF16, packed E2M1 nibbles and E8M0 block scales.  A step is that
 launch.  Other workloads (`--workload`): nvfp4_tied, q4k, nvfp4_weight,
 activation, moe_nvfp4, moe_mxfp4, moe_q4k, nvfp4_tied_f32, q4k_f32 (FP32 master
-weights), lora_nvfp4 (LoRA-merged weights), q4k_mse (MSE-searched Q4_K fit); an
-NVFP4 step is the tied-amax pass followed by the fused pass.
+weights), lora_nvfp4 (LoRA-merged weights), lora_amax (their tie-group amax alone),
+q4k_mse (MSE-searched Q4_K fit); an NVFP4 step is the tied-amax pass followed by the
+fused pass.
 
   value      GB/s of algorithmic bytes per step (read BF16 + write BF16 + codes +
              scales = 4.5625 / 4.53125 / 4.5625 B per element for NVFP4 / MXFP4 /
@@ -52,7 +53,8 @@ UNIT = "GB/s"
 BYTES_PER_ELEM = {"nvfp4": 2 + 2 + 0.5 + 1 / 16, "mxfp4": 2 + 2 + 0.5 + 1 / 32,
                   "q4k": 2 + 2 + 144 / 256, "q4k_mse": 2 + 2 + 144 / 256}
 WORKLOADS = ("w4a4", "nvfp4_tied", "q4k", "nvfp4_weight", "activation", "moe_nvfp4",
-             "moe_mxfp4", "moe_q4k", "nvfp4_tied_f32", "q4k_f32", "lora_nvfp4", "q4k_mse")
+             "moe_mxfp4", "moe_q4k", "nvfp4_tied_f32", "q4k_f32", "lora_nvfp4", "lora_amax",
+             "q4k_mse")
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -232,6 +234,11 @@ def make_workload(name: str, qf, dev, seed_shift: int = 0):
         desc = ("LoRA-QAD NVFP4: tied Q/K/V and gate/up bases with rank-16 adapters (scale 2); "
                 "qf_amax_fakequant_lora: the merged weight formed once (written to y with its "
                 "group amax), then fake-quant+pack of y in place")
+    elif name == "lora_amax":
+        wl, fmt = workloads.nvfp4_tied(seed=3 + seed_shift, with_grads=False), "nvfp4"
+        desc = ("LoRA-QAD NVFP4 tie-group amax of the merged weights (qf_amax_tied_lora): tied "
+                "Q/K/V and gate/up bases with rank-16 adapters (scale 2), W read once, the merge "
+                "evaluated exactly only where a bound reaches the group's max")
     elif name == "activation":
         wl, fmt = workloads.nvfp4_activation(seed=5 + seed_shift), "nvfp4"
         desc = ("NVFP4 activation 32768x4096 Student-t(3) with tracked amax: amax pass "
@@ -249,6 +256,20 @@ def make_workload(name: str, qf, dev, seed_shift: int = 0):
     W = dict(name=name, fmt=fmt, desc=desc, xs=xs, xs_h=xs_h, outs=[t for t in Y + C + S if
              t is not None], numel=numel, fq_bytes=numel * (BYTES_PER_ELEM[fmt] + in_b - 2),
              n_tensors=len(xs), in_bytes=in_b, groups=groups, n_groups=ng)
+    if name == "lora_amax":
+        r = 16
+        ads = [(workloads.normal_with_outliers(x.shape[0], r, 0.01, 0, 1, 9 + seed_shift, 2 * i)
+                .to(dev), workloads.normal_with_outliers(r, x.shape[1], 0.02, 0, 1, 9 + seed_shift,
+                                                         2 * i + 1).to(dev), 2.0)
+               for i, x in enumerate(xs)]
+        amax = torch.zeros(ng, dtype=torch.float32, device=dev)
+        W["pre"] = None
+        W["fq"] = qf.prepare_amax_tied_lora(xs, ads, groups, amax)
+        W["fq_bytes"] = W["step_bytes"] = 2 * numel          # W read once
+        W["launches"] = 1
+        W["kernel"] = "k_lora_amax"
+        W["adapters"] = ads
+        return W
     if name == "lora_nvfp4":
         r = 16
         ads = [(workloads.normal_with_outliers(x.shape[0], r, 0.01, 0, 1, 9 + seed_shift, 2 * i)
@@ -268,7 +289,7 @@ def make_workload(name: str, qf, dev, seed_shift: int = 0):
         W["fq_bytes"] = W["step_bytes"]
         W["two_call"] = lambda: (pre2(), fq2())
         W["launches"] = 2
-        W["kernel"] = "k_lora_merge_amax+k_nv"
+        W["kernel"] = "k_lora8+k_nv"
         W["adapters"] = ads
         return W
     if name == "nvfp4_weight":

@@ -347,6 +347,10 @@ constexpr int kLoraLargeT = 256;
 template <int MODE, int R>
 qf_status lora_launch_r(const std::vector<qf::LoraTensor>& v, const float* am, float* so, int ng,
                         cudaStream_t s) {
+    // merge modes up to rank 16: 8 columns per lane (k_lora8), kLora8Rows-row units
+    constexpr bool k8 = QF_LORA8 && R <= 16 && (MODE == qf::kLoraMerge ||
+                                                MODE == qf::kLoraMergeAmax);
+    constexpr int64_t kRowsPerUnit = k8 ? qf::kLora8Rows : qf::kLoraRows;
     for (size_t b = 0; b < v.size(); b += kLoraLargeT) {
         const size_t cnt = std::min<size_t>(kLoraLargeT, v.size() - b);
         float* sout = b == 0 ? so : nullptr;
@@ -356,7 +360,7 @@ qf_status lora_launch_r(const std::vector<qf::LoraTensor>& v, const float* am, f
             for (size_t i = 0; i < cnt; ++i) {
                 qf::LoraTensor d = v[b + i];
                 d.unit_begin = u;
-                u += ((d.rows + qf::kLoraRows - 1) / qf::kLoraRows) * d.col_groups;
+                u += ((d.rows + kRowsPerUnit - 1) / kRowsPerUnit) * d.col_groups;
                 P.t[i] = d;
             }
             P.total_units = u;
@@ -365,9 +369,6 @@ qf_status lora_launch_r(const std::vector<qf::LoraTensor>& v, const float* am, f
             P.group_scale_out = sout;
             P.n_groups = ng;
         };
-        // merge modes up to rank 16: 8 columns per lane (k_lora8), same units
-        constexpr bool k8 = QF_LORA8 && R <= 16 && (MODE == qf::kLoraMerge ||
-                                                    MODE == qf::kLoraMergeAmax);
         if (cnt <= (size_t)kLoraSmallT) {
             qf::LoraTable<kLoraSmallT> P;
             fill(P);

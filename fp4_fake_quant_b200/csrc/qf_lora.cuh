@@ -522,7 +522,7 @@ __global__ void __launch_bounds__(kLoraThreads, R <= 16 ? 2 : 1) k_lora(const __
 // ------------------------------------------------------------------ merge, 8 columns per lane
 // k_lora8: the merge modes (kLoraMerge, kLoraMergeAmax) for rank <= 16 with each lane
 // owning 8 consecutive columns (a 128-thread CTA still covers 1024 columns by
-// kLoraRows rows, the unit of k_lora).  Against 4 columns per lane, every broadcast
+// kLora8Rows rows).  Against 4 columns per lane, every broadcast
 // load of two (b, b) pairs feeds 8 paired FMAs instead of 4 and the per-row work is
 // shared by twice the elements; the A slab takes 128 registers per lane (R = 16).
 // Arithmetic, results and the fused-rounding rule are those of k_lora's merge.
@@ -536,6 +536,10 @@ __global__ void __launch_bounds__(kLoraThreads, R <= 16 ? 2 : 1) k_lora(const __
 #define QF_LORA8_MINB 3
 #endif
 constexpr int kLora8Threads = 128;
+#ifndef QF_LORA8_ROWS
+#define QF_LORA8_ROWS 64
+#endif
+constexpr int kLora8Rows = QF_LORA8_ROWS;   // rows per CTA unit of k_lora8 (an even number)
 
 __device__ __forceinline__ void cp_async16_cg(uint32_t dst, const void* src, uint32_t src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
@@ -550,7 +554,7 @@ __global__ void __launch_bounds__(kLora8Threads, QF_LORA8_MINB)
     constexpr int kS = QF_LORA8_STAGES;
     constexpr bool kWritesMerged = true;
     constexpr bool kFoldsAmax = MODE == kLoraMergeAmax;
-    __shared__ __align__(16) uint64_t bsm[kLoraRows][R];                 // (b, b) FP32 pairs
+    __shared__ __align__(16) uint64_t bsm[kLora8Rows][R];                 // (b, b) FP32 pairs
     __shared__ __align__(16) uint4 wring[kS][2][kLora8Threads];
     __shared__ uint32_t s_rmax, s_cmax;
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
@@ -558,17 +562,17 @@ __global__ void __launch_bounds__(kLora8Threads, QF_LORA8_MINB)
     if (cu >= P.total_units) return;
     const LoraTensor& T = P.t[lora_locate(P, cu)];
     const int64_t local = cu - T.unit_begin;
-    const int64_t r0 = (local / T.col_groups) * kLoraRows;
+    const int64_t r0 = (local / T.col_groups) * kLora8Rows;
     const int64_t c_base = (local % T.col_groups) * kLoraCols;
     const int64_t rows_left = T.rows - r0;
-    const int nrows = rows_left < kLoraRows ? (int)rows_left : kLoraRows;
+    const int nrows = rows_left < kLora8Rows ? (int)rows_left : kLora8Rows;
     const int64_t cols = T.cols;
     const int64_t col0 = c_base + wid * 256 + lane * 8;
     const bool colok = col0 < cols;            // cols % 16 == 0: 8 columns all in or all out
     const int rank = T.rank;
     const float scale = T.scale;
 
-    for (int idx = threadIdx.x; idx < kLoraRows * R; idx += kLora8Threads) {
+    for (int idx = threadIdx.x; idx < kLora8Rows * R; idx += kLora8Threads) {
         const int i = idx / R, k = idx % R;
         const float b = (i < nrows && k < rank) ? bf16_lo(T.b[(r0 + i) * rank + k]) : 0.0f;
         bsm[i][k] = pk2(b, b);
@@ -588,7 +592,7 @@ __global__ void __launch_bounds__(kLora8Threads, QF_LORA8_MINB)
     __syncthreads();
     // the fused-rounding rule of k_lora (kFusedMerge): scale = 2^e, e >= 0, and
     // scale * Rmax * Cmax * (1 + 2^-6) < 2^126 over the CTA's rows and columns
-    if (threadIdx.x < kLoraRows) {
+    if (threadIdx.x < kLora8Rows) {
         float r = 0.0f;
 #pragma unroll
         for (int k = 0; k < R; ++k) r = __fadd_rn(r, fabsf(unpk2(bsm[threadIdx.x][k]).x));
@@ -618,7 +622,7 @@ __global__ void __launch_bounds__(kLora8Threads, QF_LORA8_MINB)
         constexpr bool FULL = decltype(tag)::value;
         constexpr bool FUSED = decltype(ftag)::value;
         const uint64_t s2 = pk2(scale, scale);
-        const int n = FULL ? kLoraRows : nrows;
+        const int n = FULL ? kLora8Rows : nrows;
         const int nst = (n + 1) >> 1;
         auto row = [&](int i) { return FULL ? i : min(i, n - 1); };
         const uint32_t ring = (uint32_t)__cvta_generic_to_shared(&wring[0][0][threadIdx.x]);
@@ -684,7 +688,7 @@ __global__ void __launch_bounds__(kLora8Threads, QF_LORA8_MINB)
         }
         cp_async_wait<0>();
     };
-    if (nrows == kLoraRows && colok) {
+    if (nrows == kLora8Rows && colok) {
         if (fused) unit(FullTile<true>{}, FullTile<true>{});
         else unit(FullTile<true>{}, FullTile<false>{});
     } else {
