@@ -14,6 +14,10 @@
 #include "qf.h"
 #include "qf_device.cuh"
 #include "qf_lora.cuh"
+
+#ifndef QF_LORA_STEP_TWO_PASS
+#define QF_LORA_STEP_TWO_PASS 0  // LoRA step up to rank 16: 1 = pruned amax + fused NVFP4 pass
+#endif
 #include "qf_oneshot.cuh"
 
 namespace {
@@ -347,9 +351,10 @@ constexpr int kLoraLargeT = 256;
 template <int MODE, int R>
 qf_status lora_launch_r(const std::vector<qf::LoraTensor>& v, const float* am, float* so, int ng,
                         cudaStream_t s) {
-    // merge modes up to rank 16: 8 columns per lane (k_lora8), kLora8Rows-row units
-    constexpr bool k8 = QF_LORA8 && R <= 16 && (MODE == qf::kLoraMerge ||
-                                                MODE == qf::kLoraMergeAmax);
+    // merge modes and NVFP4 up to rank 16: 8 columns per lane (k_lora8), kLora8Rows-row units
+    constexpr bool k8 = QF_LORA8 && R <= 16 &&
+                        (MODE == qf::kLoraMerge || MODE == qf::kLoraMergeAmax ||
+                         (QF_LORA8_NV && MODE == qf::kLoraNV));
     constexpr int64_t kRowsPerUnit = k8 ? qf::kLora8Rows : qf::kLoraRows;
     for (size_t b = 0; b < v.size(); b += kLoraLargeT) {
         const size_t cnt = std::min<size_t>(kLoraLargeT, v.size() - b);
@@ -686,8 +691,11 @@ qf_status qf_amax_fakequant_lora(const qf_tensor* t, const qf_lora* l, int n,
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
     bool all_y = true;
     for (const qf::LoraTensor& d : v) all_y &= d.y != nullptr;
-    if (v.empty() || !all_y) {
-        // no room for the merged weight: form it twice (amax pass, then fused pass)
+    // With room for it in y, the merged weight is written once with its amax and
+    // quantized in place.  Otherwise (or with QF_LORA_STEP_TWO_PASS up to rank 16) the
+    // step reads W twice: the pruned exact amax, then the merge-on-the-fly NVFP4 pass.
+    const bool two_pass = v.empty() || !all_y || (QF_LORA_STEP_TWO_PASS && max_rank <= 16);
+    if (two_pass) {
         if (!v.empty()) {
             st = lora_amax_launch(v, d_group_amax, s);
             if (st != QF_OK) return st;

@@ -520,14 +520,23 @@ __global__ void __launch_bounds__(kLoraThreads, R <= 16 ? 2 : 1) k_lora(const __
 
 
 // ------------------------------------------------------------------ merge, 8 columns per lane
-// k_lora8: the merge modes (kLoraMerge, kLoraMergeAmax) for rank <= 16 with each lane
-// owning 8 consecutive columns (a 128-thread CTA still covers 1024 columns by
-// kLora8Rows rows).  Against 4 columns per lane, every broadcast
+// k_lora8: the merge modes (kLoraMerge, kLoraMergeAmax) and the NVFP4 mode for rank
+// <= 16 with each lane owning 8 consecutive columns (a 128-thread CTA still covers 1024
+// columns by kLora8Rows rows).  Against 4 columns per lane, every broadcast
 // load of two (b, b) pairs feeds 8 paired FMAs instead of 4 and the per-row work is
 // shared by twice the elements; the A slab takes 128 registers per lane (R = 16).
-// Arithmetic, results and the fused-rounding rule are those of k_lora's merge.
+// Arithmetic, results and the fused-rounding rule are those of k_lora's merge.  In the
+// NVFP4 mode a 16-element block spans a lane pair, and the merged BF16 values of each
+// row go through the 8-element-lane NVFP4 codec (fp4_lane): block max over the pair,
+// E4M3 block scale, E2M1 codes and the dequantized BF16 values, as in k_lora.
 #ifndef QF_LORA8
 #define QF_LORA8 1
+#endif
+#ifndef QF_LORA8_NV
+#define QF_LORA8_NV 1           // NVFP4 mode of the merge-on-the-fly pass in k_lora8
+#endif
+#ifndef QF_LORA8_NV_MINB
+#define QF_LORA8_NV_MINB 2
 #endif
 #ifndef QF_LORA8_STAGES
 #define QF_LORA8_STAGES 4       // W ring depth in 2-row steps (16 bytes per lane and row)
@@ -547,18 +556,24 @@ __device__ __forceinline__ void cp_async16_cg(uint32_t dst, const void* src, uin
 }
 
 template <int MODE, int R, int MAXT>
-__global__ void __launch_bounds__(kLora8Threads, QF_LORA8_MINB)
+__global__ void __launch_bounds__(kLora8Threads, MODE == kLoraNV ? QF_LORA8_NV_MINB : QF_LORA8_MINB)
     k_lora8(const __grid_constant__ LoraTable<MAXT> P) {
-    static_assert(MODE == kLoraMerge || MODE == kLoraMergeAmax, "merge modes only");
+    static_assert(MODE == kLoraMerge || MODE == kLoraMergeAmax || MODE == kLoraNV,
+                  "merge modes and NVFP4 only");
     static_assert(R <= 16, "the A slab of rank 32 does not fit in registers");
     constexpr int kS = QF_LORA8_STAGES;
-    constexpr bool kWritesMerged = true;
+    constexpr bool kNV = MODE == kLoraNV;
+    constexpr bool kWritesMerged = !kNV;
     constexpr bool kFoldsAmax = MODE == kLoraMergeAmax;
     __shared__ __align__(16) uint64_t bsm[kLora8Rows][R];                 // (b, b) FP32 pairs
     __shared__ __align__(16) uint4 wring[kS][2][kLora8Threads];
     __shared__ uint32_t s_rmax, s_cmax;
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int64_t cu = blockIdx.x;
+    if (kNV && cu == 0 && P.group_scale_out) {
+        for (int g = threadIdx.x; g < P.n_groups; g += kLora8Threads)
+            P.group_scale_out[g] = nv_tensor_scale(P.group_amax[g]);
+    }
     if (cu >= P.total_units) return;
     const LoraTensor& T = P.t[lora_locate(P, cu)];
     const int64_t local = cu - T.unit_begin;
@@ -616,6 +631,11 @@ __global__ void __launch_bounds__(kLora8Threads, QF_LORA8_MINB)
                                             __uint_as_float(s_cmax)), 1.0f + 0x1p-6f);
     const bool fused = QF_LORA_FUSED && pow2 && bound < 0x1p126f;
 
+    float s_t = 0.0f, six_st = 0.0f;
+    if (kNV) {
+        s_t = nv_tensor_scale(P.group_amax[T.group]);
+        six_st = __fmul_rn(6.0f, s_t);
+    }
     uint32_t run = 0;
     const uint16_t* wbase = T.w + r0 * cols + col0;
     auto unit = [&](auto tag, auto ftag) {
@@ -640,7 +660,9 @@ __global__ void __launch_bounds__(kLora8Threads, QF_LORA8_MINB)
         };
 #pragma unroll
         for (int st = 0; st < kS - 1; ++st) issue(st);
-        uint16_t* yrow = T.y + r0 * cols + col0;
+        // the merge modes step a row pointer; the NVFP4 mode a flat element index
+        uint16_t* yrow = kWritesMerged ? T.y + r0 * cols + col0 : nullptr;
+        int64_t erow = kNV ? r0 * cols + col0 : 0;
 #pragma unroll 1
         for (int st = 0; st < nst; ++st) {
             cp_async_wait<kS - 2>();                        // this step's W has landed
@@ -678,13 +700,29 @@ __global__ void __launch_bounds__(kLora8Threads, QF_LORA8_MINB)
                                            __fadd_rn(bf16_lo(wv[p]), __fmul_rn(scale, sp.x)));
                     }
                 }
-                if (kWritesMerged && (FULL || (colok && 2 * st + h < n)))
+                const bool keep = FULL || (colok && 2 * st + h < n);
+                if constexpr (kNV) {
+                    const int64_t e = erow + h * cols;
+                    // every lane runs the codec (its block max is a pair shuffle); rows past
+                    // the end repeat the last row and are not stored
+                    Elems<uint16_t, 8> xe;
+                    xe.v[0] = make_uint4(xo[0], xo[1], xo[2], xo[3]);
+                    Fp4Lane o;
+                    fp4_lane<true, true>(xe, s_t, six_st, o);
+                    if (keep) {
+                        if (T.y) *reinterpret_cast<uint4*>(T.y + e) = o.y;
+                        if (T.codes) *reinterpret_cast<uint32_t*>(T.codes + (e >> 1)) = o.codes;
+                        if (T.scales && (lane & 1) == 0) T.scales[e >> 4] = (uint8_t)o.scale;
+                    }
+                }
+                if (kWritesMerged && keep)
                     *reinterpret_cast<uint4*>(yrow + h * cols) = make_uint4(xo[0], xo[1], xo[2], xo[3]);
                 if (kFoldsAmax)
                     run = max_u16x2(max_u16x2(run, max_u16x2(xo[0] & 0x7FFF7FFFu, xo[1] & 0x7FFF7FFFu)),
                                     max_u16x2(xo[2] & 0x7FFF7FFFu, xo[3] & 0x7FFF7FFFu));
             }
-            yrow += 2 * cols;
+            if (kWritesMerged) yrow += 2 * cols;
+            if (kNV) erow += 2 * cols;
         }
         cp_async_wait<0>();
     };
