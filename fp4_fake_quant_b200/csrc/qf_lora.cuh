@@ -769,11 +769,15 @@ __global__ void __launch_bounds__(kLora8Threads, MODE == kLoraNV ? QF_LORA8_NV_M
 // only ever receives exact values).
 //
 // Pass 1 reads the CTA's tile (kLoraAmaxRows rows x 1024 columns) and keeps, per row and
-// lane, the max |W| of the lane's 32 elements; the CTA's best lb follows from it.
-// Pass 2 revisits only the (row, lane) pieces whose bound reaches that lower bound,
-// re-reads their 32 elements (from L2) and evaluates the merge exactly, with the merge
-// kernel's arithmetic, where the element's own bound still reaches it.  The result is the
-// max over the evaluated elements: exact, since the max element is always evaluated.
+// lane, the max |W| of the lane's 32 elements; the CTA's best lb follows from it.  Its
+// first row pair is requested before the prologue (the adapters' maxima) and every
+// later pair one step ahead, so the tile's reads stay in flight.
+// Pass 2 revisits only the (row, lane) pieces whose bound reaches that lower bound and
+// re-reads their 32 elements (from L2); the elements whose own bound still reaches it go
+// to a per-warp queue in shared memory, and the warp evaluates the queue 32 elements at
+// a time, one per lane, with the merge kernel's arithmetic (each element's rank-r terms
+// fetched 8 at a time).  The result is the max over the evaluated elements: exact, since
+// the max element is always evaluated.
 #ifndef QF_LORA_AMAX_ROWS
 #define QF_LORA_AMAX_ROWS 128
 #endif
@@ -783,14 +787,27 @@ constexpr float kBoundDown = 1.0f - 0x1p-7f;
 constexpr float kBoundWiden = 1.0f + 0x1p-6f;
 constexpr float kBoundTiny = 0x1p-120f;
 
-// |M| of element (i, j) as FP32: the merge of k_lora, one element at a time
+// |M| of element (i, j) as FP32: the merge of k_lora, one element at a time, with the
+// terms' operands fetched 8 at a time (8 loads of B's row and 8 of A's column in flight
+// together); the terms are still added one by one in increasing k.
 __device__ __forceinline__ float lora_merged_mag(const LoraTensor& T, int64_t i, int64_t j,
-                                                 float w) {
+                                                  float w) {
     const uint16_t* bp = T.b + i * T.rank;
     const uint16_t* ap = T.a + j;
     float acc = 0.0f;
-    for (int k = 0; k < T.rank; ++k)
-        acc = __fmaf_rn(bf16_lo(bp[k]), bf16_lo(ap[k * T.cols]), acc);
+#pragma unroll 1
+    for (int k0 = 0; k0 < T.rank; k0 += 8) {
+        float bv[8], av[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const bool ok = k0 + u < T.rank;
+            bv[u] = ok ? bf16_lo(bp[k0 + u]) : 0.0f;
+            av[u] = ok ? bf16_lo(ap[(int64_t)(k0 + u) * T.cols]) : 0.0f;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            if (k0 + u < T.rank) acc = __fmaf_rn(bv[u], av[u], acc);
+    }
     const uint32_t m = cvt_bf16x2(0.0f, __fadd_rn(w, __fmul_rn(T.scale, acc)));
     return __uint_as_float((m & 0x7FFFu) << 16);
 }
@@ -802,8 +819,11 @@ __device__ __forceinline__ uint32_t max_abs_bf16x8(uint32_t m, uint4 v) {
     return max_u16x2(m, v.w & 0x7FFF7FFFu);
 }
 
+#ifndef QF_LORA_AMAX_MINB
+#define QF_LORA_AMAX_MINB 3     // 3 CTAs per SM (80 registers): 61.5 us against 77.9 at 2
+#endif
 template <int MAXT>
-__global__ void __launch_bounds__(kLoraThreads) k_lora_amax(const __grid_constant__ LoraTable<MAXT> P) {
+__global__ void __launch_bounds__(kLoraThreads, QF_LORA_AMAX_MINB) k_lora_amax(const __grid_constant__ LoraTable<MAXT> P) {
     constexpr int kWarps = kLoraThreads / 32;
     constexpr int kRpw = kLoraAmaxRows / kWarps;         // rows per warp, read two at a time
     constexpr int kChunks = kLoraCols / 8;                // 16-byte column chunks per tile row
@@ -813,6 +833,9 @@ __global__ void __launch_bounds__(kLoraThreads) k_lora_amax(const __grid_constan
     __shared__ float s_c[kLoraCols];                      // C_j
     __shared__ uint4 s_cpart[2][kChunks];                 // per-chunk |a| maxima, two k halves
     __shared__ uint32_t s_lb, s_best;
+    constexpr int kQueue = 64;                            // pass-2 queue entries per warp
+    __shared__ uint2 s_q[kWarps][kQueue];                 // (row << 16 | column, W bits)
+    __shared__ uint32_t s_qn[kWarps];
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     if (blockIdx.x >= P.total_units) return;
     const LoraTensor& T = P.t[lora_locate(P, blockIdx.x)];
@@ -827,6 +850,22 @@ __global__ void __launch_bounds__(kLoraThreads) k_lora_amax(const __grid_constan
     const float sabs = fabsf(T.scale);
     const float tiny = __fadd_rn(kBoundTiny, __fmul_rn(sabs, 0x1p-140f));
     unsigned int* gamax = reinterpret_cast<unsigned int*>(const_cast<float*>(P.group_amax)) + T.group;
+    const uint16_t* wlane = T.w + r0 * cols + c_base + 8 * lane;
+    // pass 1's reads, a row pair (eight 16-byte loads per lane) per step: rows
+    // wid + kWarps t and wid + kWarps (t + 1); the first pair is requested now
+    auto load_pair = [&](int t, uint4 (&v)[2][4]) {
+        const int i0 = wid + kWarps * t;
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                v[h][q] = (i0 + h * kWarps < nrows && 256 * q + 8 * lane < ncols)
+                              ? ld_stream<0>(wlane + (i0 + h * kWarps) * cols + 256 * q)
+                              : make_uint4(0, 0, 0, 0);
+    };
+    uint4 vbuf[2][2][4];
+    load_pair(0, vbuf[0]);
+    if (lane == 0) s_qn[wid] = 0u;
 
     // ---- prologue: C_j (16-byte loads of A, k split over two threads per chunk), K_i,
     // and the group's amax so far
@@ -878,23 +917,16 @@ __global__ void __launch_bounds__(kLoraThreads) k_lora_amax(const __grid_constan
     auto dbound = [&](float k, float c) {
         return (k > 0.0f && c > 0.0f) ? __fadd_rn(__fmul_rn(k, c), tiny) : 0.0f;
     };
-    const uint16_t* wlane = T.w + r0 * cols + c_base + 8 * lane;
 
-    // ---- pass 1: max |W| per (row, lane), two rows (eight 16-byte loads) at a time;
-    // the best lower bound
+    // ---- pass 1: max |W| per (row, lane), a row pair per step with the next pair's
+    // loads in flight; the best lower bound
     float mrow[kRpw];
     float lb_best = 0.0f;
 #pragma unroll
     for (int t = 0; t < kRpw; t += 2) {
         const int i0 = wid + kWarps * t, i1 = i0 + kWarps;
-        uint4 v[2][4];
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                v[h][q] = (i0 + h * kWarps < nrows && 256 * q + 8 * lane < ncols)
-                              ? ld_stream<0>(wlane + (i0 + h * kWarps) * cols + 256 * q)
-                              : make_uint4(0, 0, 0, 0);
+        if (t + 2 < kRpw) load_pair(t + 2, vbuf[((t >> 1) + 1) & 1]);
+        const uint4 (&v)[2][4] = vbuf[(t >> 1) & 1];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             uint32_t m = 0;
@@ -927,27 +959,57 @@ __global__ void __launch_bounds__(kLoraThreads) k_lora_amax(const __grid_constan
                                       kBoundUp);
         if (i < nrows && rowub >= L && rowub > best) cand |= 1u << t;
     }
+    // the elements of those pieces whose own bound reaches L, into the warp's queue (an
+    // element past its capacity is evaluated on the spot)
 #pragma unroll 1
     while (cand) {
         const int t = __ffs(cand) - 1;
         cand &= cand - 1;
         const int i = wid + kWarps * t;
         const float ki = s_k[i];
+        uint4 vq[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            vq[q] = 256 * q + 8 * lane < ncols ? ld_stream<1>(wlane + i * cols + 256 * q)
+                                               : make_uint4(0, 0, 0, 0);
 #pragma unroll 1
         for (int q = 0; q < 4; ++q) {
             const int c0 = 256 * q + 8 * lane;
             if (c0 >= ncols) continue;
-            const uint4 v = ld_stream<1>(wlane + i * cols + 256 * q);
-            const uint64_t lo = v.x | (uint64_t)v.y << 32, hi = v.z | (uint64_t)v.w << 32;
+            const uint64_t lo = vq[q].x | (uint64_t)vq[q].y << 32;
+            const uint64_t hi = vq[q].z | (uint64_t)vq[q].w << 32;
 #pragma unroll 1
             for (int e = 0; e < 8; ++e) {
                 const uint32_t wb = (uint32_t)(((e < 4 ? lo : hi) >> (16 * (e & 3))) & 0xFFFFu);
                 const float x = __uint_as_float((wb & 0x7FFFu) << 16);
                 const float ub = __fmul_rn(__fadd_rn(x, dbound(ki, s_c[c0 + e])), kBoundUp);
-                if (ub >= L && ub > best)
-                    best = fmaxf(best, lora_merged_mag(T, r0 + i, c_base + c0 + e,
-                                                       __uint_as_float(wb << 16)));
+                if (ub >= L && ub > best) {
+                    const uint32_t pos = atomicAdd(&s_qn[wid], 1u);
+                    if (pos < (uint32_t)kQueue)
+                        s_q[wid][pos] = make_uint2((uint32_t)i << 16 | (uint32_t)(c0 + e), wb);
+                    else
+                        best = fmaxf(best, lora_merged_mag(T, r0 + i, c_base + c0 + e,
+                                                            __uint_as_float(wb << 16)));
+                }
             }
+        }
+    }
+    __syncwarp();
+    // the queue, 32 elements at a time, each skipped once the warp's best exceeds its bound
+    const int nq = (int)min(s_qn[wid], (uint32_t)kQueue);
+#pragma unroll 1
+    for (int b0 = 0; b0 < nq; b0 += 32) {
+        float wbest = best;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) wbest = fmaxf(wbest, __shfl_xor_sync(kFull, wbest, o));
+        if (b0 + lane < nq) {
+            const uint2 q = s_q[wid][b0 + lane];
+            const int i = (int)(q.x >> 16), c = (int)(q.x & 0xFFFFu);
+            const float x = __uint_as_float((q.y & 0x7FFFu) << 16);
+            const float ub = __fmul_rn(__fadd_rn(x, dbound(s_k[i], s_c[c])), kBoundUp);
+            if (ub > wbest)
+                best = fmaxf(best, lora_merged_mag(T, r0 + i, c_base + c,
+                                                    __uint_as_float(q.y << 16)));
         }
     }
     // ---- the CTA's best exact value into the group's amax
