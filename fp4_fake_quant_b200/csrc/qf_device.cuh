@@ -360,6 +360,52 @@ __device__ __forceinline__ void nv_block_scale(float amax_b, float s_t, float si
     }
 }
 
+// NVFP4 block scale from a tie group's tables.  The divisor 6 s_t of the block ratio is
+// one number per tie group, so its reciprocal yd = RN(1 / (6 s_t)) is taken once, and
+// q0 = RN(amax_b * yd) lies within two FP32 steps of the ratio RN(amax_b / (6 s_t))
+// wherever both fall in one binade (the product's relative error is below 2^-24, and
+// each rounding adds at most half a step).  The block byte is the ratio rounded to E4M3;
+// in E4M3's normal range [2^-6, 448] every rounding boundary has the low 20 mantissa bits
+// 0x80000, so where q0's low bits are more than 3 steps from that pattern, q0 and the
+// ratio round to the same byte, and below 2^-11 (or above 2^9) both give 0 (or the
+// saturated 448).  Everything else (near a boundary, E4M3's subnormal range, a NaN, or a
+// group whose 6 s_t lies outside [2^-80, 2^100], marked by yd = 0) takes the division of
+// nv_block_scale.  S and 1/S come from the group's table of the 128 E4M3 bytes, filled
+// with nv_block_scale's own operations.
+struct NvScaleTab {
+    float S[128];
+    float inv[128];
+};
+// entries i, i + n, ... of the table of tensor scale s_t (s_t != 0)
+__device__ __forceinline__ void nv_tab_fill(NvScaleTab& t, float s_t, int i, int n) {
+    for (int c = i; c < 128; c += n) {
+        const float S = __fmul_rn(f16_lo(cvt_e4m3x2_f16x2((uint32_t)c)), s_t);
+        t.S[c] = S;
+        t.inv[c] = S == 0.0f ? 0.0f : __frcp_rn(S);
+    }
+}
+// yd for a group, 0 where the division is always taken
+__device__ __forceinline__ float nv_ratio_recip(float six_st) {
+    return (six_st >= 0x1p-80f && six_st <= 0x1p100f) ? __frcp_rn(six_st) : 0.0f;
+}
+// whether q0 = RN(amax_b * yd) rounds to the block byte itself
+__device__ __forceinline__ bool nv_ratio_fast(float q0, float yd) {
+    const uint32_t low = __float_as_uint(q0) & 0xFFFFFu;
+    return yd != 0.0f && (q0 < 0x1p-11f || q0 > 0x1p9f || (q0 >= 0x1p-6f && low - 0x7FFFDu > 6u));
+}
+__device__ __forceinline__ void nv_block_scale_tab(float amax_b, float s_t, float six_st, float yd,
+                                                   const NvScaleTab& t, uint32_t& sb, float& S,
+                                                   float& inv) {
+    const float q0 = __fmul_rn(amax_b, yd);
+    if (__builtin_expect(nv_ratio_fast(q0, yd), 1)) {
+        sb = cvt_e4m3x2(0.0f, q0) & 0xFFu;
+        S = t.S[sb];
+        inv = t.inv[sb];
+    } else {
+        nv_block_scale(amax_b, s_t, six_st, sb, S, inv);
+    }
+}
+
 // ------------------------------------------------------------------ k_fp4 (MXFP4; STE)
 // Per-lane result of the FP4 codec for 8 elements.
 struct Fp4Lane {
@@ -369,16 +415,19 @@ struct Fp4Lane {
     float q[8];         // scaled values (for the clipped STE)
 };
 
-template <bool NV, bool WANT_Y, typename XT>
+// TAB (NVFP4): the block scale from the group's tables (nv_block_scale_tab; yd, tab given).
+template <bool NV, bool WANT_Y, bool TAB = false, typename XT>
 __device__ __forceinline__ void fp4_lane(const Elems<XT, 8>& x, float s_t, float six_st,
-                                         Fp4Lane& o) {
+                                         Fp4Lane& o, float yd = 0.0f,
+                                         const NvScaleTab* tab = nullptr) {
     uint32_t a = x.amax_bits();
     a = max(a, __shfl_xor_sync(kFull, a, 1));
     if (!NV) a = max(a, __shfl_xor_sync(kFull, a, 2));
     float S, inv;
     if (NV) {
         uint32_t sb;
-        nv_block_scale(__uint_as_float(a), s_t, six_st, sb, S, inv);
+        if constexpr (TAB) nv_block_scale_tab(__uint_as_float(a), s_t, six_st, yd, *tab, sb, S, inv);
+        else nv_block_scale(__uint_as_float(a), s_t, six_st, sb, S, inv);
         o.scale = sb;
     } else {
         // E8M0: e = floor(log2 amax) - 2 clamped to >= -127; byte = e + 127 = max(E - 2, 0)

@@ -538,6 +538,9 @@ __global__ void __launch_bounds__(kLoraThreads, R <= 16 ? 2 : 1) k_lora(const __
 #ifndef QF_LORA8_NV_MINB
 #define QF_LORA8_NV_MINB 2
 #endif
+#ifndef QF_LORA8_TAB
+#define QF_LORA8_TAB 1          // NVFP4 mode: block scales from the CTA's tables (nv_block_scale_tab)
+#endif
 #ifndef QF_LORA8_STAGES
 #define QF_LORA8_STAGES 4       // W ring depth in 2-row steps (16 bytes per lane and row)
 #endif
@@ -568,6 +571,7 @@ __global__ void __launch_bounds__(kLora8Threads, MODE == kLoraNV ? QF_LORA8_NV_M
     __shared__ __align__(16) uint64_t bsm[kLora8Rows][R];                 // (b, b) FP32 pairs
     __shared__ __align__(16) uint4 wring[kS][2][kLora8Threads];
     __shared__ uint32_t s_rmax, s_cmax;
+    __shared__ NvScaleTab s_tab[1];                                        // NVFP4 mode
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int64_t cu = blockIdx.x;
     if (kNV && cu == 0 && P.group_scale_out) {
@@ -604,6 +608,15 @@ __global__ void __launch_bounds__(kLora8Threads, MODE == kLoraNV ? QF_LORA8_NV_M
         a[k][3] = pk2(bf16_lo(v.w), bf16_hi(v.w));
     }
     if (threadIdx.x == 0) s_rmax = s_cmax = 0u;
+    float s_t = 0.0f, six_st = 0.0f, yd = 0.0f;
+    if (kNV) {
+        s_t = nv_tensor_scale(P.group_amax[T.group]);
+        six_st = __fmul_rn(6.0f, s_t);
+        if (QF_LORA8_TAB) {
+            yd = nv_ratio_recip(six_st);
+            if (yd != 0.0f) nv_tab_fill(s_tab[0], s_t, threadIdx.x, kLora8Threads);
+        }
+    }
     __syncthreads();
     // the fused-rounding rule of k_lora (kFusedMerge): scale = 2^e, e >= 0, and
     // scale * Rmax * Cmax * (1 + 2^-6) < 2^126 over the CTA's rows and columns
@@ -631,11 +644,6 @@ __global__ void __launch_bounds__(kLora8Threads, MODE == kLoraNV ? QF_LORA8_NV_M
                                             __uint_as_float(s_cmax)), 1.0f + 0x1p-6f);
     const bool fused = QF_LORA_FUSED && pow2 && bound < 0x1p126f;
 
-    float s_t = 0.0f, six_st = 0.0f;
-    if (kNV) {
-        s_t = nv_tensor_scale(P.group_amax[T.group]);
-        six_st = __fmul_rn(6.0f, s_t);
-    }
     uint32_t run = 0;
     const uint16_t* wbase = T.w + r0 * cols + col0;
     auto unit = [&](auto tag, auto ftag) {
@@ -708,7 +716,7 @@ __global__ void __launch_bounds__(kLora8Threads, MODE == kLoraNV ? QF_LORA8_NV_M
                     Elems<uint16_t, 8> xe;
                     xe.v[0] = make_uint4(xo[0], xo[1], xo[2], xo[3]);
                     Fp4Lane o;
-                    fp4_lane<true, true>(xe, s_t, six_st, o);
+                    fp4_lane<true, true, QF_LORA8_TAB>(xe, s_t, six_st, o, yd, &s_tab[0]);
                     if (keep) {
                         if (T.y) *reinterpret_cast<uint4*>(T.y + e) = o.y;
                         if (T.codes) *reinterpret_cast<uint32_t*>(T.codes + (e >> 1)) = o.codes;
