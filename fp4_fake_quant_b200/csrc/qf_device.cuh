@@ -746,6 +746,30 @@ __global__ void __launch_bounds__(THREADS) k_nv_ste(const __grid_constant__ Tabl
     }
 }
 
+// RN(x / c) for a constant divisor c > 0, given c_inv = RN(1 / c): q0 = RN(x * c_inv)
+// and one correction by the exact residual x - q0 c (Markstein's correction step, as in
+// P. Markstein, "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Dev. 34(1), 1990); a zero residual keeps q0 (and the sign of a
+// zero quotient).  Magnitudes outside [2^-100, 2^100], and NaN, take the division itself.
+// For each constant the kernels use, a GPU test compares it with the IEEE division on
+// every one of the 2^32 inputs.
+__device__ __forceinline__ float div_const(float x, float c, float c_inv) {
+    const float ax = fabsf(x);
+    if (__builtin_expect(ax <= 0x1p100f && (ax >= 0x1p-100f || ax == 0.0f), 1)) {
+        const float q0 = __fmul_rn(x, c_inv);
+        const float r = __fmaf_rn(-q0, c, x);
+        return r == 0.0f ? q0 : __fmaf_rn(r, c_inv, q0);
+    }
+    return __fdiv_rn(x, c);
+}
+#ifndef QF_DIVCONST
+#define QF_DIVCONST 1           // Q4_K fits: divisions by constants through div_const
+#endif
+// x / c for one of the Q4_K fits' constant divisors (c_inv = RN(1 / c))
+__device__ __forceinline__ float q4k_div(float x, float c, float c_inv) {
+    return QF_DIVCONST ? div_const(x, c, c_inv) : __fdiv_rn(x, c);
+}
+
 // ------------------------------------------------------------------ Q4_K
 // One lane per 32-element sub-block: a warp iteration covers 4 super-blocks (1024
 // elements) and lane l owns sub-block j = l / 4 of super-block b = l % 4, so the
@@ -810,7 +834,7 @@ __device__ __forceinline__ float2 q4k_sub_err2(const Elems<XT, 32>& x, float2 sc
 template <typename XT, bool LOWER>
 __device__ __forceinline__ float q4k_search_scale_t(const Elems<XT, 32>& x, float range,
                                                     float best, float s18, float min_j) {
-    const float s14 = __fdiv_rn(range, 14.0f);
+    const float s14 = q4k_div(range, 14.0f, 1.0f / 14.0f);
     float xm[32];
 #pragma unroll
     for (int k = 0; k < 32; ++k) xm[k] = QF_Q4K_MSE_HOIST ? __fadd_rn(x.get(k), min_j) : 0.0f;
@@ -826,7 +850,11 @@ __device__ __forceinline__ float q4k_search_scale_t(const Elems<XT, 32>& x, floa
     for (int p = 0; p < 4; ++p) {
         const float na = p == 0 ? 14.5f : p == 1 ? 16.0f : p == 2 ? 17.0f : 18.0f;
         const float nb = p == 0 ? 15.5f : p == 1 ? 16.5f : p == 2 ? 17.5f : 18.0f;
-        const float2 sc = make_float2(p == 3 ? s18 : __fdiv_rn(range, na), __fdiv_rn(range, nb));
+        const float ia = p == 0 ? 1.0f / 14.5f : p == 1 ? 1.0f / 16.0f : p == 2 ? 1.0f / 17.0f
+                                                                         : 1.0f / 18.0f;
+        const float ib = p == 0 ? 1.0f / 15.5f : p == 1 ? 1.0f / 16.5f : p == 2 ? 1.0f / 17.5f
+                                                                         : 1.0f / 18.0f;
+        const float2 sc = make_float2(p == 3 ? s18 : q4k_div(range, na, ia), q4k_div(range, nb, ib));
         const float2 err = q4k_sub_err2<XT, LOWER>(x, sc, min_j, xm);
         if (err.x < best_err) {
             best_err = err.x;
@@ -842,10 +870,10 @@ __device__ __forceinline__ float q4k_search_scale_t(const Elems<XT, 32>& x, floa
 template <typename XT>
 __device__ __forceinline__ float q4k_search_scale(const Elems<XT, 32>& x, float hi, float min_j) {
     const float range = __fadd_rn(hi, min_j);
-    const float best = __fdiv_rn(range, 15.0f);
+    const float best = q4k_div(range, 15.0f, 1.0f / 15.0f);
     if (best == 0.0f) return best;
     // range / 18 is the smallest trial scale: when its reciprocal is finite, so are all
-    const float s18 = __fdiv_rn(range, 18.0f);
+    const float s18 = q4k_div(range, 18.0f, 1.0f / 18.0f);
     if (__frcp_rn(s18) <= 3.402823466e38f)
         return q4k_search_scale_t<XT, false>(x, range, best, s18, min_j);
     return q4k_search_scale_t<XT, true>(x, range, best, s18, min_j);
@@ -862,15 +890,15 @@ __device__ __forceinline__ Q4kFit q4k_fit(const Elems<XT, 32>& x) {
     x.minmax(lo, hi);
     const float min_j = lo < 0.0f ? -lo : 0.0f;
     const float scale_j = MSE ? q4k_search_scale(x, hi, min_j)
-                              : __fdiv_rn(__fadd_rn(hi, min_j), 15.0f);
+                              : q4k_div(__fadd_rn(hi, min_j), 15.0f, 1.0f / 15.0f);
     float ms = scale_j, mm = min_j;
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {               // the 8 lanes of this super-block
         ms = fmaxf(ms, __shfl_xor_sync(kFull, ms, o));
         mm = fmaxf(mm, __shfl_xor_sync(kFull, mm, o));
     }
-    const __half dh = __float2half_rn(__fdiv_rn(ms, 63.0f));
-    const __half dmh = __float2half_rn(__fdiv_rn(mm, 63.0f));
+    const __half dh = __float2half_rn(q4k_div(ms, 63.0f, 1.0f / 63.0f));
+    const __half dmh = __float2half_rn(q4k_div(mm, 63.0f, 1.0f / 63.0f));
     const float d = __half2float(dh), dmin = __half2float(dmh);
     Q4kFit f;
     f.dbits = __half_as_ushort(dh);

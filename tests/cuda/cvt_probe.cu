@@ -98,7 +98,27 @@ __global__ void k_blockscale(const float* s_t, uint32_t n_f32, unsigned long lon
     atomicAdd(fast + blockIdx.y, nfast);
 }
 
+// div_const(x, c, RN(1/c)) against __fdiv_rn(x, c) on every binary32 x (bit patterns
+// lo .. lo + n - 1); counts mismatches (NaN results match any NaN) and records the first.
+__global__ void k_divconst(float c, float c_inv, uint32_t lo, uint64_t n,
+                           unsigned long long* bad, uint32_t* first) {
+    const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
+    for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+        const uint32_t u = lo + (uint32_t)i;
+        const float x = __uint_as_float(u);
+        const float a = qf::div_const(x, c, c_inv), b = __fdiv_rn(x, c);
+        const bool same = __float_as_uint(a) == __float_as_uint(b) || (isnan(a) && isnan(b));
+        if (!same && atomicAdd(bad, 1ull) == 0ull) *first = u;
+    }
+}
+
 }  // namespace
+
+extern "C" int probe_divconst(float c, float c_inv, uint32_t lo, uint64_t n,
+                              unsigned long long* bad, uint32_t* first) {
+    k_divconst<<<148 * 16, 256>>>(c, c_inv, lo, n, bad, first);
+    return cudaDeviceSynchronize() == cudaSuccess ? 0 : 2;
+}
 
 extern "C" int probe_blockscale(const float* s_t, int n_st, uint32_t n_f32,
                                 unsigned long long* bad, uint32_t* first,
