@@ -542,10 +542,7 @@ __global__ void __launch_bounds__(kLoraThreads, R <= 16 ? 2 : 1) k_lora(const __
 #define QF_LORA8_TAB 1          // NVFP4 mode: block scales from the CTA's tables (nv_block_scale_tab)
 #endif
 #ifndef QF_LORA8_STAGES
-#define QF_LORA8_STAGES 4       // W ring depth in steps (16 bytes per lane and row)
-#endif
-#ifndef QF_LORA8_RPS
-#define QF_LORA8_RPS 2          // rows per step: their rank-r products are formed together
+#define QF_LORA8_STAGES 4       // W ring depth in 2-row steps (16 bytes per lane and row)
 #endif
 #ifndef QF_LORA8_MINB
 #define QF_LORA8_MINB 3
@@ -572,9 +569,7 @@ __global__ void __launch_bounds__(kLora8Threads, MODE == kLoraNV ? QF_LORA8_NV_M
     constexpr bool kWritesMerged = !kNV;
     constexpr bool kFoldsAmax = MODE == kLoraMergeAmax;
     __shared__ __align__(16) uint64_t bsm[kLora8Rows][R];                 // (b, b) FP32 pairs
-    constexpr int kRps = QF_LORA8_RPS;                 // rows per step
-    static_assert(kLora8Rows % kRps == 0, "whole steps per unit");
-    __shared__ __align__(16) uint4 wring[kS][kRps][kLora8Threads];
+    __shared__ __align__(16) uint4 wring[kS][2][kLora8Threads];
     __shared__ uint32_t s_rmax, s_cmax;
     __shared__ NvScaleTab s_tab[1];                                        // NVFP4 mode
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
@@ -656,16 +651,16 @@ __global__ void __launch_bounds__(kLora8Threads, MODE == kLoraNV ? QF_LORA8_NV_M
         constexpr bool FUSED = decltype(ftag)::value;
         const uint64_t s2 = pk2(scale, scale);
         const int n = FULL ? kLora8Rows : nrows;
-        const int nst = (n + kRps - 1) / kRps;
+        const int nst = (n + 1) >> 1;
         auto row = [&](int i) { return FULL ? i : min(i, n - 1); };
         const uint32_t ring = (uint32_t)__cvta_generic_to_shared(&wring[0][0][threadIdx.x]);
         auto issue = [&](int st) {
             if (st < nst) {
-                const uint32_t dst = ring + (uint32_t)((st % kS) * kRps * kLora8Threads * 16);
+                const uint32_t dst = ring + (uint32_t)((st % kS) * 2 * kLora8Threads * 16);
 #pragma unroll
-                for (int h = 0; h < kRps; ++h)
+                for (int h = 0; h < 2; ++h)
                     cp_async16_cg(dst + h * kLora8Threads * 16,
-                                  (FULL || colok) ? (const void*)(wbase + row(kRps * st + h) * cols)
+                                  (FULL || colok) ? (const void*)(wbase + row(2 * st + h) * cols)
                                                   : (const void*)T.w,
                                   (FULL || colok) ? 16u : 0u);
             }
@@ -679,15 +674,13 @@ __global__ void __launch_bounds__(kLora8Threads, MODE == kLoraNV ? QF_LORA8_NV_M
 #pragma unroll 1
         for (int st = 0; st < nst; ++st) {
             cp_async_wait<kS - 2>();                        // this step's W has landed
-            const uint32_t src = ring + (uint32_t)((st % kS) * kRps * kLora8Threads * 16);
-            uint4 w[kRps];
-#pragma unroll
-            for (int h = 0; h < kRps; ++h) w[h] = lds128(src + h * kLora8Threads * 16);
+            const uint32_t src = ring + (uint32_t)((st % kS) * 2 * kLora8Threads * 16);
+            const uint4 w[2] = {lds128(src), lds128(src + kLora8Threads * 16)};
             issue(st + kS - 1);                             // refills the stage read last step
-            uint64_t acc[kRps][4];
+            uint64_t acc[2][4];
 #pragma unroll
-            for (int h = 0; h < kRps; ++h) {
-                const int i = row(kRps * st + h);
+            for (int h = 0; h < 2; ++h) {
+                const int i = row(2 * st + h);
 #pragma unroll
                 for (int p = 0; p < 4; ++p) acc[h][p] = 0;
 #pragma unroll
@@ -700,7 +693,7 @@ __global__ void __launch_bounds__(kLora8Threads, MODE == kLoraNV ? QF_LORA8_NV_M
                 }
             }
 #pragma unroll
-            for (int h = 0; h < kRps; ++h) {
+            for (int h = 0; h < 2; ++h) {
                 const uint32_t wv[4] = {w[h].x, w[h].y, w[h].z, w[h].w};
                 uint32_t xo[4];
 #pragma unroll
@@ -715,7 +708,7 @@ __global__ void __launch_bounds__(kLora8Threads, MODE == kLoraNV ? QF_LORA8_NV_M
                                            __fadd_rn(bf16_lo(wv[p]), __fmul_rn(scale, sp.x)));
                     }
                 }
-                const bool keep = FULL || (colok && kRps * st + h < n);
+                const bool keep = FULL || (colok && 2 * st + h < n);
                 if constexpr (kNV) {
                     const int64_t e = erow + h * cols;
                     // every lane runs the codec (its block max is a pair shuffle); rows past
@@ -736,8 +729,8 @@ __global__ void __launch_bounds__(kLora8Threads, MODE == kLoraNV ? QF_LORA8_NV_M
                     run = max_u16x2(max_u16x2(run, max_u16x2(xo[0] & 0x7FFF7FFFu, xo[1] & 0x7FFF7FFFu)),
                                     max_u16x2(xo[2] & 0x7FFF7FFFu, xo[3] & 0x7FFF7FFFu));
             }
-            if (kWritesMerged) yrow += kRps * cols;
-            if (kNV) erow += kRps * cols;
+            if (kWritesMerged) yrow += 2 * cols;
+            if (kNV) erow += 2 * cols;
         }
         cp_async_wait<0>();
     };
