@@ -23,8 +23,11 @@ fused pass.
              HBM copy bandwidth.
   cpu_baseline  the oracle (scalar C) on a bounded sample of the rows, on every host core
              of the affinity mask (rows split over threads), plus a one-core figure.
+  pack_only  the same launch writing codes and scales only (no BF16 dequant): the
+             input read plus 0.5625 / 0.53125 / 0.5625 B per element.
   per_format the other workloads, each timed per call with the L2 flushed
-             (L2Flush: L2 left holding only clean lines).
+             (L2Flush: L2 left holding only clean lines), with their pack-only launch.
+  per_format_summary  the line's last key: compact figures for every workload.
 
 `--impl reference` times the oracle on the host cores for the same metric (the
 reference arm).  Launch with torchrun for N > 1 GPUs (one process per GPU).
@@ -52,6 +55,8 @@ METRIC = "fake-quant+pack GB/s and Gelem/s per format; % of B200 HBM roofline"
 UNIT = "GB/s"
 BYTES_PER_ELEM = {"nvfp4": 2 + 2 + 0.5 + 1 / 16, "mxfp4": 2 + 2 + 0.5 + 1 / 32,
                   "q4k": 2 + 2 + 144 / 256, "q4k_mse": 2 + 2 + 144 / 256}
+# pack only (codes and scales, no BF16 dequant): output bytes per element beside the input
+PACK_BYTES = {"nvfp4": 0.5 + 1 / 16, "mxfp4": 0.5 + 1 / 32, "q4k": 144 / 256}
 WORKLOADS = ("w4a4", "nvfp4_tied", "q4k", "nvfp4_weight", "activation", "moe_nvfp4",
              "moe_mxfp4", "moe_q4k", "nvfp4_tied_f32", "q4k_f32", "lora_nvfp4", "lora_amax",
              "q4k_mse")
@@ -322,12 +327,15 @@ def make_workload(name: str, qf, dev, seed_shift: int = 0):
             W["pre"] = qf.prepare_amax_tied(xs, groups, amax)
             W["one_call"] = qf.prepare_amax_fakequant(xs, Y, C, S, groups, amax, group_scale_out=so)
         W["fq"] = qf.prepare_fakequant(fmt, xs, Y, C, S, groups, amax, so)
+        W["pack"] = qf.prepare_fakequant(fmt, xs, None, C, S, groups, amax, so, pack_only=True)
         W["step_bytes"] = W["fq_bytes"] + in_b * numel
         W["launches"] = 2 * chunks
         W["kernel"] = "k_nv"
     else:
         W["pre"] = None
         W["fq"] = qf.prepare_fakequant(fmt, xs, Y, C, S)
+        if fmt in PACK_BYTES:
+            W["pack"] = qf.prepare_fakequant(fmt, xs, None, C, S, pack_only=True)
         W["step_bytes"] = W["fq_bytes"]
         W["launches"] = chunks
         W["kernel"] = {"mxfp4": "k_fp4_mxfp4", "q4k": "k_q4k", "q4k_mse": "k_q4k_mse"}[fmt]
@@ -408,6 +416,7 @@ def run_ours(args, rank, world, local_rank):
                       "over 3 streams, H2D / kernel / D2H overlapped"}
         del pipe
 
+    pack = pack_timing(W, 20, 3, flush_buf if flush_buf is not None else (lambda: None))
     peak, peak_kind = peaks()
     achieved = W["fq_bytes"] / (kern_ms * 1e-3) / 1e9
     clocks = clk.summary()
@@ -447,6 +456,8 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": args.steps * W["launches"],
         "clocks": clocks,
     }
+    if pack is not None:
+        result["pack_only"] = pack
     del W, flush_buf
     torch.cuda.empty_cache()
     if rank == 0 and world == 1 and not args.no_per_format:
@@ -494,6 +505,12 @@ def format_summary(headline: str, result: dict, peak: float) -> dict:
         if "ste_identity_us" in d:
             ste = [_r(d["ste_identity_us"]), _r(d["ste_identity_GB/s"] / peak),
                    _r(d["ste_clipped_us"]), _r(d["ste_clipped_GB/s"] / peak)]
+    packs = {name: _r(d["pack_only"]["frac_of_hbm_peak"]) for name, d in result["per_format"].items()
+             if "pack_only" in d}
+    if "pack_only" in result:
+        packs = {headline: _r(result["pack_only"]["frac_of_hbm_peak"]), **packs}
+    if packs:
+        out["pack_only_frac"] = packs
     if moe:
         out["moe_grouped_vs_per_expert_us"] = {"cols": ["grouped", "per_expert_graph",
                                                         "per_expert_eager"], **moe}
@@ -542,6 +559,18 @@ class L2Flush:
         self.r.max()
 
 
+def pack_timing(W, iters, warm, flush):
+    """The pack-only launch (codes and scales, no BF16 dequant) of a workload that has
+    one, timed like the fused pass; its algorithmic bytes are the input read plus
+    PACK_BYTES per element.  Run after a whole step, so an NVFP4 amax is real."""
+    if "pack" not in W:
+        return None
+    t = timed_calls(W["pack"], iters, warm, flush)
+    gbs = W["numel"] * (W["in_bytes"] + PACK_BYTES[W["fmt"]]) / (t * 1e-3) / 1e9
+    return {"us": t * 1e3, "GB/s": gbs, "frac_of_hbm_peak": gbs / peaks()[0],
+            "bytes_per_element": W["in_bytes"] + PACK_BYTES[W["fmt"]]}
+
+
 def timed_calls(fn, iters, warm, flush):
     """Median device time (ms) of `fn` over `iters` calls, each after an L2 flush."""
     for _ in range(warm):
@@ -574,6 +603,7 @@ def per_format(qf, dev, args, l2, sm_max_mhz=None):
         pre_fn, fq_fn, fq_bytes = W["parts"] if "parts" in W else (W["pre"], W["fq"], W["fq_bytes"])
         run_step(W)
         t_fq = timed_calls(fq_fn, it, warm, flush)
+        pack = pack_timing(W, it, warm, flush)
         t_hot = timed_calls(fq_fn, it, warm, lambda: None)
         gbs = fq_bytes / (t_fq * 1e-3) / 1e9
         d = {"format": W["fmt"], "input": "fp32" if W["in_bytes"] == 4 else "bf16",
@@ -583,6 +613,8 @@ def per_format(qf, dev, args, l2, sm_max_mhz=None):
              # back-to-back calls without a flush: a tensor that fits in L2 is read from it
              "fused_hot_l2_us": t_hot * 1e3,
              "fused_hot_l2_GB/s": fq_bytes / (t_hot * 1e-3) / 1e9}
+        if pack is not None:
+            d["pack_only"] = pack
         if W["fmt"] == "q4k_mse":
             tops, how = fp32_peak_tops(dev, sm_max_mhz)
             ach = W["numel"] * MSE_OPS_PER_ELEM / (t_fq * 1e-3) / 1e12
