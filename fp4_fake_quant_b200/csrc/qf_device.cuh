@@ -77,6 +77,9 @@
 #ifndef QF_Q4K_PREFETCH
 #define QF_Q4K_PREFETCH 0       // 1: register prefetch of each warp's next unit (BF16 input)
 #endif
+#ifndef QF_Q4K_LD
+#define QF_Q4K_LD 1             // BF16 input: load form (ld_stream)
+#endif
 #ifndef QF_Q4K_MINB
 #define QF_Q4K_MINB 0           // > 0: minimum resident CTAs per SM asked of the register allocator
 #endif
@@ -92,7 +95,10 @@
 #define QF_AMAX_WAVES 1000
 #endif
 #ifndef QF_AMAX_LD
-#define QF_AMAX_LD 0
+#define QF_AMAX_LD 2            // amax pass: load form (ld_stream; 2 measured best)
+#endif
+#ifndef QF_COPY_LD
+#define QF_COPY_LD 1            // STE identity copy: load form (ld_stream; 1 measured best)
 #endif
 #ifndef QF_AMAX_ORDER
 #define QF_AMAX_ORDER 0         // 0: one contiguous unit range per CTA, 1: grid-stride sweep
@@ -238,6 +244,7 @@ __device__ __forceinline__ uint4 ld_stream(const void* p) {
     else if (LD == 2)
         asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
             : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+
     else
         asm volatile("ld.global.v4.u32 {%0,%1,%2,%3}, [%4];"
                      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p) : "memory");
@@ -1012,7 +1019,7 @@ __global__ void QF_Q4K_BOUNDS(THREADS) k_q4k(const __grid_constant__ Table<MAXT>
         const XT* xp = static_cast<const XT*>(T.x);
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-            v[k] = k < nsb ? ld_stream<0>(xp + e0 + 256 * k + 8 * lane) : make_uint4(0, 0, 0, 0);
+            v[k] = k < nsb ? ld_stream<QF_Q4K_LD>(xp + e0 + 256 * k + 8 * lane) : make_uint4(0, 0, 0, 0);
     };
     if (kPf && warp < P.total_units) load_raw(warp, ti, vn);
     for (int64_t u = warp; u < P.total_units; u += nwarps) {
@@ -1034,7 +1041,7 @@ __global__ void QF_Q4K_BOUNDS(THREADS) k_q4k(const __grid_constant__ Table<MAXT>
             } else {
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    v[k] = k < nsb ? ld_stream<0>(xp + e0 + 256 * k + 8 * lane) : make_uint4(0, 0, 0, 0);
+                    v[k] = k < nsb ? ld_stream<QF_Q4K_LD>(xp + e0 + 256 * k + 8 * lane) : make_uint4(0, 0, 0, 0);
             }
             __syncwarp();
 #pragma unroll
@@ -1201,7 +1208,7 @@ __global__ void __launch_bounds__(kThreads) k_copy(const uint16_t* __restrict__ 
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const int64_t i = base + j * kThreads;
-        if (i < nvec) v[j] = ld_stream<0>(src + 8 * i);
+        if (i < nvec) v[j] = ld_stream<QF_COPY_LD>(src + 8 * i);
     }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {

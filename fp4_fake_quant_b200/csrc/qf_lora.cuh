@@ -827,6 +827,9 @@ __device__ __forceinline__ uint32_t max_abs_bf16x8(uint32_t m, uint4 v) {
     return max_u16x2(m, v.w & 0x7FFF7FFFu);
 }
 
+#ifndef QF_LORA_AMAX_LD
+#define QF_LORA_AMAX_LD 0       // pass 1's loads of W (ld_stream form)
+#endif
 #ifndef QF_LORA_AMAX_MINB
 #define QF_LORA_AMAX_MINB 3     // 3 CTAs per SM (80 registers): 61.5 us against 77.9 at 2
 #endif
@@ -868,7 +871,7 @@ __global__ void __launch_bounds__(kLoraThreads, QF_LORA_AMAX_MINB) k_lora_amax(c
 #pragma unroll
             for (int q = 0; q < 4; ++q)
                 v[h][q] = (i0 + h * kWarps < nrows && 256 * q + 8 * lane < ncols)
-                              ? ld_stream<0>(wlane + (i0 + h * kWarps) * cols + 256 * q)
+                              ? ld_stream<QF_LORA_AMAX_LD>(wlane + (i0 + h * kWarps) * cols + 256 * q)
                               : make_uint4(0, 0, 0, 0);
     };
     uint4 vbuf[2][2][4];
