@@ -471,6 +471,11 @@ def run_ours(args, rank, world, local_rank):
     return result
 
 
+def _rows_part(frac: float) -> str:
+    """Words for a row sample: all rows, or the leading fraction of them."""
+    return "all rows" if frac >= 1 else f"the first {frac:.3g} of the rows"
+
+
 def _r(v, nd=3):
     """Round to `nd` significant digits (None stays None)."""
     if v is None:
@@ -831,7 +836,7 @@ def cpu_baseline(name, frac):
     bpe = BYTES_PER_ELEM[fmt] + sample[0].element_size() - 2      # FP32 input reads 4 B
     return {"value": n * bpe / dt_all / 1e9, "unit": UNIT, "cores": cores,
             "kind": "oracle",
-            "sample": f"first {frac:.3g} of the rows of every tensor ({n} elements), scalar C, "
+            "sample": f"{_rows_part(frac)} of every tensor ({n} elements), scalar C, "
                       f"rows split over {cores} host threads, {dt_all:.1f} s",
             "single_core_value": n1 * bpe / dt_one / 1e9,
             "single_core_sample": f"a quarter of that sample ({n1} elements) on one thread, "
@@ -863,7 +868,7 @@ def run_reference(args, world):
         step()
     dt = (time.perf_counter() - t0) / args.steps
     value = n * BYTES_PER_ELEM["mxfp4"] / dt / 1e9
-    desc = (f"oracle (scalar C) on the first {frac:.3g} of the rows of W and A ({n} elements) "
+    desc = (f"oracle (scalar C) on {_rows_part(frac)} of W and A ({n} elements) "
             f"per step, rows split over {cores} host threads")
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
